@@ -1,0 +1,363 @@
+"""Benchmark: SVQ 2.25-bpw batch-1 GEMV on a Qwen3-4B-shaped decoder layer.
+
+One step = one grouped launch of the seven SVQ linears of a decoder layer
+(q 2560->4096 (6,4), k/v 2560->1024 (7,3)/(8,2), o 4096->2560 (9,1),
+gate/up 2560->9728 (6,4)/(7,3), down 9728->2560 (8,2)) at batch 1, x fp16.
+Steps rotate through 14 independent layer copies (397 MB of packed codes, more
+than 3x the 126 MB L2), so every step streams its weights from HBM.  Launches
+are replayed from CUDA graphs; the timed region is bracketed by a barrier and
+device synchronisation and timed with CUDA events on the launching stream.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); the layer is not partitioned, each
+rank runs the same workload on its own GPU (replicas, weak scaling); the
+reported value is the sum of all ranks' bytes over the slowest rank's time.
+--impl reference: the CPU oracle on the host cores, same metric, each step a
+bounded sample (8 rows of one of the seven matrices).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "SVQ 2.25-bpw GEMV packed-weight GB/s and % HBM peak (batch 1, Qwen3-4B shapes)"
+UNIT = "GB/s"
+N_LAYERS = 14
+WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 1, one grouped launch per step"
+
+
+def layer_bytes():
+    packed = sum(N * K * 9 // 32 for _, N, K in synth.QWEN3_4B_SHAPES)
+    cb = sum((1 << b) * 16 for b in synth.QWEN3_4B_SPLITS)
+    params = sum(N * 4 for _, N, K in synth.QWEN3_4B_SHAPES)          # fp16 scale + offset
+    perm = sum(K * 4 for _, N, K in synth.QWEN3_4B_SHAPES)
+    x = sum(K * 2 for _, N, K in synth.QWEN3_4B_SHAPES)
+    y = sum(N * 4 for _, N, K in synth.QWEN3_4B_SHAPES)                # fp32 outputs
+    return packed, packed + cb + params + perm + x + y
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- CPU oracle (reference arm, cpu_baseline)
+def oracle_rows_sample(layer, step: int, rows: int = 8):
+    """(bytes, seconds) of the oracle on `rows` rows of one matrix (chosen by `step`)."""
+    import oracle
+    m, x = layer[step % 7]
+    nblk = m.N // rows
+    r0 = ((step // 7) % nblk) * rows
+    sub = synth.SvqMatrix(rows, m.K, m.b_d, np.ascontiguousarray(m.canonical[r0:r0 + rows]), m.codebook,
+                          np.ascontiguousarray(m.scale[r0:r0 + rows]),
+                          np.ascontiguousarray(m.offset[r0:r0 + rows]), m.perm)
+    t0 = time.perf_counter()
+    oracle.linear(sub, x)
+    dt = time.perf_counter() - t0
+    return rows * m.K * 9 // 32, dt
+
+
+def cpu_baseline(layer, budget_s: float = 12.0):
+    import oracle
+    oracle.linear(*layer[1])  # warm (builds the library)
+    nbytes, secs, steps = 0, 0.0, 0
+    rows = 64
+    while secs < budget_s:
+        b, dt = oracle_rows_sample(layer, steps, rows)
+        nbytes += b
+        secs += dt
+        steps += 1
+    return {"value": nbytes / secs / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{steps} calls of the fp64 C++ oracle, each {rows} rows of one of the seven layer "
+                      f"matrices (decode + fp64 dot), {nbytes} packed bytes in {secs:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    layer = synth.qwen3_4b_layer(0)
+    import oracle
+    oracle.linear(*layer[1])
+    for s in range(args.warmup):
+        oracle_rows_sample(layer, s)
+    nbytes, secs = 0, 0.0
+    for s in range(args.steps):
+        b, dt = oracle_rows_sample(layer, args.warmup + s)
+        nbytes += b
+        secs += dt
+    value = nbytes / secs / 1e9
+    cores = oracle.num_threads()
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD + " (CPU oracle: 8-row sample of one matrix per step)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "8 rows of one of the seven matrices per step, fp64 C++ oracle"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args, world, rank, local):
+    import torch
+
+    import bit_spherical_vector_b200 as svq
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    packed_b, alg_b = layer_bytes()
+
+    # Weights: N_LAYERS independent layer copies resident in HBM.
+    layers, Ws, xs_host = [], [], []
+    with torch.cuda.stream(stream):
+        for L in range(N_LAYERS):
+            layer = synth.qwen3_4b_layer(L)
+            layers.append(layer)
+            Ws.append([svq.SvqWeight.from_synth(m) for m, _ in layer])
+            xs_host.append([x for _, x in layer])
+    torch.cuda.synchronize()
+    for W in Ws:                      # drop the canonical upload buffers
+        for w in W:
+            w._canon_d = None
+
+    xs = [[torch.from_numpy(x.view(np.int16)).to(dev).view(torch.float16) for x in xl] for xl in xs_host]
+    ys = [[torch.empty((1, m.N), dtype=torch.float32, device=dev) for m, _ in layer] for layer in layers]
+    nb = max(svq.svq_linear_gemv_batched_workspace_size(W, 1) for W in Ws)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        svq.svq_workspace_init(ws)
+
+    def step(i):
+        L = i % N_LAYERS
+        svq.svq_linear_gemv_batched(Ws[L], xs[L], ys[L], ws)
+
+    # warm-up (eager), then capture one graph per layer and one graph of all layers
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+    torch.cuda.synchronize()
+    g_all = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_all, stream=stream):
+        for i in range(N_LAYERS):
+            step(i)
+    g_one = []
+    for L in range(N_LAYERS):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(L)
+        g_one.append(g)
+
+    def replay(k):
+        full, rem = divmod(k, N_LAYERS)
+        for _ in range(full):
+            g_all.replay()
+        for L in range(rem):
+            g_one[L].replay()
+
+    with torch.cuda.stream(stream):
+        replay(N_LAYERS * 4)          # graph warm-up
+    torch.cuda.synchronize()
+
+    # ---- device-timed region
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            replay(args.steps)
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    value = world * args.steps * packed_b / (ms_max * 1e-3) / 1e9
+    per_launch_s = ms * 1e-3 / args.steps
+    peak, peak_kind = read_peaks()
+    achieved = alg_b / per_launch_s / 1e9
+
+    # ---- end-to-end through the public API: pinned host x -> device, layer, y -> pinned host
+    e2e_steps = min(args.steps, 2000)
+    xh = [[torch.from_numpy(x.view(np.int16)).view(torch.float16).pin_memory() for x in xl] for xl in xs_host]
+    yh = [[torch.empty((1, m.N), dtype=torch.float32).pin_memory() for m, _ in layer] for layer in layers]
+    h2d = sum(x.numel() * 2 for x in xh[0])
+    d2h = sum(y.numel() * 4 for y in yh[0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(e2e_steps):
+            L = i % N_LAYERS
+            for xd, xhh in zip(xs[L], xh[L]):
+                xd.copy_(xhh, non_blocking=True)
+            svq.svq_linear_gemv_batched(Ws[L], xs[L], ys[L], ws)
+            for yd, yhh in zip(ys[L], yh[L]):
+                yhh.copy_(yd, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_value = world * e2e_steps * packed_b / (e2e_ms * 1e-3) / 1e9
+
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layer_packed_bytes": packed_b, "layer_algorithmic_bytes": alg_b,
+                   "layer_copies_rotated": N_LAYERS,
+                   "l2": f"inputs larger than L2: {N_LAYERS} layer copies, {N_LAYERS * packed_b / 1e6:.0f} MB "
+                         "of packed codes rotated",
+                   "hbm_pct_of_peak": 100.0 * value / world / peak, "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s",
+                     "kernel": "gemv_kernel<1> (grouped, 7 matrices)",
+                     "achieved_bytes": "all algorithmic bytes per launch (packed codes, codebooks, radius "
+                                       "params, perm, x, y)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(layers[0])
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=140000)
+    ap.add_argument("--warmup", type=int, default=1400)
+    ap.add_argument("--impl", default="svq", choices=["svq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_init() if args.impl == "svq" else (int(os.environ.get("WORLD_SIZE", "1")),
+                                                                 int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_gpu(args, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "svq":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

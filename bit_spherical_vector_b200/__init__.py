@@ -1,0 +1,210 @@
+"""Python binding of libsvq (include/svq.h): argument marshalling only.
+
+Every entry point takes torch CUDA tensors (device memory) and the current
+torch stream, passes raw pointers to the C ABI and raises SvqError on a
+non-zero status.  All computation happens in the CUDA kernels of libsvq.so;
+there is no CPU or PyTorch fallback.  If the library is missing the import of
+the binding functions fails loudly (call ``compile_library()`` or
+``python -m bit_spherical_vector_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "lib", "libsvq.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "svq.h")
+
+SVQ_OK, SVQ_ERR_INVALID_ARG, SVQ_ERR_UNSUPPORTED_SHAPE, SVQ_ERR_WORKSPACE, SVQ_ERR_CUDA, SVQ_ERR_TIMEOUT = range(6)
+SVQ_F16, SVQ_BF16, SVQ_F32 = 1, 2, 3
+
+
+class SvqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: status {status} ({status_string(status)})")
+        self.status = status
+
+
+class svq_matrix(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("b_d", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("packed", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
+                ("radius_scale", ctypes.c_void_p), ("radius_offset", ctypes.c_void_p),
+                ("perm", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def compile_library(force: bool = False) -> str:
+    """Compile libsvq.so in-tree (see bit_spherical_vector_b200/build.py)."""
+    import importlib
+    return importlib.import_module(__name__ + ".build").build(force=force)
+
+
+def lib():
+    """The loaded libsvq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libsvq.so not found at {LIB_PATH}; build it with "
+                          "`python -m bit_spherical_vector_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    MP = ctypes.POINTER(svq_matrix)
+    sig = {
+        "svq_status_string": ([I], ctypes.c_char_p),
+        "svq_version": ([], I),
+        "svq_packed_bytes": ([I, I], SZ),
+        "svq_canonical_bytes": ([I, I], SZ),
+        "svq_repack": ([P, I, I, I, P, P], I),
+        "svq_unpack_fields": ([P, I, I, I, P, P, P, P], I),
+        "svq_dequantize": ([MP, I, P, P], I),
+        "svq_linear_gemv_workspace_size": ([MP, I, ctypes.POINTER(SZ)], I),
+        "svq_workspace_init": ([P, SZ, P], I),
+        "svq_linear_gemv": ([MP, P, I, P, I, P, SZ, P], I),
+        "svq_linear_gemv_batched_workspace_size": ([MP, I, I, ctypes.POINTER(SZ)], I),
+        "svq_linear_gemv_batched": ([MP, I, ctypes.POINTER(P), I, ctypes.POINTER(P), I, P, SZ, P], I),
+        "svq_get_device_status": ([P], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().svq_status_string(int(status)).decode()
+    except ImportError:
+        return "library not loaded"
+
+
+def _check(status: int, what: str):
+    if status != SVQ_OK:
+        raise SvqError(status, what)
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _dtype_code(dtype) -> int:
+    import torch
+    return {torch.float16: SVQ_F16, torch.bfloat16: SVQ_BF16, torch.float32: SVQ_F32}[dtype]
+
+
+# ----------------------------------------------------------------------------- format
+def svq_packed_bytes(N: int, K: int) -> int:
+    return int(lib().svq_packed_bytes(N, K))
+
+
+def svq_canonical_bytes(N: int, K: int) -> int:
+    return int(lib().svq_canonical_bytes(N, K))
+
+
+def svq_repack(canonical, N: int, K: int, b_d: int, packed_out, stream=None):
+    _check(lib().svq_repack(_ptr(canonical), N, K, b_d, _ptr(packed_out), _stream(stream)), "svq_repack")
+
+
+def svq_unpack_fields(packed, N: int, K: int, b_d: int, signs, idx, code, stream=None):
+    _check(lib().svq_unpack_fields(_ptr(packed), N, K, b_d, _ptr(signs), _ptr(idx), _ptr(code),
+                                   _stream(stream)), "svq_unpack_fields")
+
+
+class SvqWeight:
+    """Device-resident SVQ matrix (packed codes, codebook, radius params, perm) and its
+    C descriptor.  Built from canonical host arrays by ``from_canonical``."""
+
+    def __init__(self, N, K, b_d, packed, codebook, scale, offset, perm):
+        self.N, self.K, self.b_d = N, K, b_d
+        self.packed, self.codebook, self.scale, self.offset, self.perm = packed, codebook, scale, offset, perm
+        self.desc = svq_matrix(N, K, b_d, 0, packed.data_ptr(), codebook.data_ptr(), scale.data_ptr(),
+                               offset.data_ptr(), perm.data_ptr())
+
+    @classmethod
+    def from_canonical(cls, N, K, b_d, canonical, codebook, scale, offset, perm, device="cuda", stream=None):
+        """canonical/codebook/scale/offset/perm: numpy arrays (uint8 / uint16 bit patterns / int32)."""
+        import numpy as np
+        import torch
+        dev = torch.device(device)
+        canon_d = torch.from_numpy(np.ascontiguousarray(canonical, np.uint8)).to(dev)
+        packed = torch.empty(svq_packed_bytes(N, K), dtype=torch.uint8, device=dev)
+        svq_repack(canon_d, N, K, b_d, packed, stream)
+        to16 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).to(dev)
+        w = cls(N, K, b_d, packed, to16(codebook), to16(scale), to16(offset),
+                torch.from_numpy(np.ascontiguousarray(perm, np.int32)).to(dev))
+        w._canon_d = canon_d   # keep alive until the repack has run
+        return w
+
+    @classmethod
+    def from_synth(cls, m, device="cuda", stream=None):
+        return cls.from_canonical(m.N, m.K, m.b_d, m.canonical, m.codebook, m.scale, m.offset, m.perm,
+                                  device, stream)
+
+
+def svq_dequantize(W: SvqWeight, out, stream=None):
+    _check(lib().svq_dequantize(ctypes.byref(W.desc), _dtype_code(out.dtype), _ptr(out), _stream(stream)),
+           "svq_dequantize")
+
+
+def svq_linear_gemv_workspace_size(W: SvqWeight, M: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().svq_linear_gemv_workspace_size(ctypes.byref(W.desc), M, ctypes.byref(n)),
+           "svq_linear_gemv_workspace_size")
+    return int(n.value)
+
+
+def svq_linear_gemv_batched_workspace_size(Ws, M: int) -> int:
+    arr = (svq_matrix * len(Ws))(*[w.desc for w in Ws])
+    n = ctypes.c_size_t(0)
+    _check(lib().svq_linear_gemv_batched_workspace_size(arr, len(Ws), M, ctypes.byref(n)),
+           "svq_linear_gemv_batched_workspace_size")
+    return int(n.value)
+
+
+def svq_workspace_init(ws, stream=None):
+    if ws is None or ws.numel() == 0:
+        return
+    _check(lib().svq_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "svq_workspace_init")
+
+
+def svq_linear_gemv(W: SvqWeight, x, y, ws=None, stream=None):
+    """y[M][N] = W x[M][K]^T with x fp16; y fp16 or fp32."""
+    M = x.shape[0]
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().svq_linear_gemv(ctypes.byref(W.desc), _ptr(x), M, _ptr(y), _dtype_code(y.dtype), _ptr(ws), nb,
+                                 _stream(stream)), "svq_linear_gemv")
+
+
+def svq_linear_gemv_batched(Ws, xs, ys, ws=None, stream=None):
+    n = len(Ws)
+    arr = (svq_matrix * n)(*[w.desc for w in Ws])
+    xp = (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs])
+    yp = (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys])
+    M = xs[0].shape[0]
+    nb = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().svq_linear_gemv_batched(arr, n, xp, M, yp, _dtype_code(ys[0].dtype), _ptr(ws), nb,
+                                         _stream(stream)), "svq_linear_gemv_batched")
+
+
+def svq_get_device_status(stream=None) -> int:
+    return int(lib().svq_get_device_status(_stream(stream)))
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/svq.h."""
+    import re
+    with open(HEADER) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"SVQ_API\s+[\w\s\*]+?\b(svq_\w+)\s*\(", src)))

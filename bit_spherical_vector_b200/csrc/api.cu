@@ -1,0 +1,172 @@
+// api.cu -- the extern "C" boundary of libsvq (declared in include/svq.h):
+// argument validation, workspace sizing, the device status word, dispatch to
+// the kernel launchers.  No entry point allocates or frees memory.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "layout.cuh"
+#include "svq.h"
+#include "svq_internal.h"
+
+namespace {
+
+__device__ int g_status_word;   // set by kernels whose bounded waits run out
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SVQ_OK : SVQ_ERR_CUDA; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+int check_matrix(const svq_matrix* W) {
+  if (!W) return SVQ_ERR_INVALID_ARG;
+  if (W->b_d < 1 || W->b_d > 10) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (W->K % 8 != 0 || !svq::layout_supported(W->N, W->K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!W->packed || !W->codebook || !W->radius_scale || !W->radius_offset || !W->perm)
+    return SVQ_ERR_INVALID_ARG;
+  if (!aligned(W->packed, 16) || !aligned(W->codebook, 16) || !aligned(W->radius_scale, 2) ||
+      !aligned(W->radius_offset, 2) || !aligned(W->perm, 4))
+    return SVQ_ERR_INVALID_ARG;
+  return SVQ_OK;
+}
+
+svq::GemvMatDesc desc_of(const svq_matrix& W, const uint16_t* x, void* y) {
+  svq::GemvMatDesc d;
+  d.N = W.N; d.K = W.K; d.b_d = W.b_d;
+  d.packed = W.packed; d.codebook = W.codebook; d.scale = W.radius_scale; d.offset = W.radius_offset;
+  d.perm = W.perm; d.x = x; d.y = y;
+  return d;
+}
+
+int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
+               svq::GemvMatDesc* descs, const uint16_t* const* x, void* const* y) {
+  if (!mats || n_mats < 1 || n_mats > svq::kGemvMaxMats) return SVQ_ERR_INVALID_ARG;
+  if (M < 1 || M > 16) return SVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_mats; ++i) {
+    const int st = check_matrix(&mats[i]);
+    if (st != SVQ_OK) return st;
+    descs[i] = desc_of(mats[i], x ? x[i] : nullptr, y ? y[i] : nullptr);
+  }
+  const int sms = num_sms();
+  if (sms <= 0) return SVQ_ERR_CUDA;
+  if (!svq::plan_gemv(descs, n_mats, M, sms, plan)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  return SVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* svq_status_string(int status) {
+  switch (status) {
+    case SVQ_OK: return "ok";
+    case SVQ_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad enum or batch size)";
+    case SVQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (needs K % 128 == 0, N % 4 == 0, 1 <= b_d <= 10)";
+    case SVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case SVQ_ERR_CUDA: return "CUDA runtime error";
+    case SVQ_ERR_TIMEOUT: return "a kernel's bounded wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int svq_version(void) { return 100; }
+
+size_t svq_packed_bytes(int N, int K) {
+  if (!svq::layout_supported(N, K)) return 0;
+  return svq::packed_bytes(N, K);
+}
+
+size_t svq_canonical_bytes(int N, int K) {
+  if (N <= 0 || K <= 0 || K % 8) return 0;
+  return (size_t)N * (((size_t)(K / 8) * 18 + 7) / 8);
+}
+
+int svq_repack(const uint8_t* canonical, int N, int K, int b_d, void* packed_out, svq_stream_t stream) {
+  if (!canonical || !packed_out) return SVQ_ERR_INVALID_ARG;
+  if (b_d < 1 || b_d > 10 || !svq::layout_supported(N, K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(packed_out, 16)) return SVQ_ERR_INVALID_ARG;
+  return cuda_status(svq::launch_repack(canonical, N, K, b_d, packed_out, (cudaStream_t)stream));
+}
+
+int svq_unpack_fields(const void* packed, int N, int K, int b_d, uint8_t* signs, uint16_t* idx,
+                      uint16_t* code, svq_stream_t stream) {
+  if (!packed || !signs || !idx || !code) return SVQ_ERR_INVALID_ARG;
+  if (b_d < 1 || b_d > 10 || !svq::layout_supported(N, K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(packed, 16) || !aligned(idx, 2) || !aligned(code, 2)) return SVQ_ERR_INVALID_ARG;
+  return cuda_status(svq::launch_unpack(packed, N, K, b_d, signs, idx, code, (cudaStream_t)stream));
+}
+
+int svq_dequantize(const svq_matrix* W, int out_dtype, void* w_out, svq_stream_t stream) {
+  const int st = check_matrix(W);
+  if (st != SVQ_OK) return st;
+  if (!w_out || !aligned(w_out, 16)) return SVQ_ERR_INVALID_ARG;
+  if (out_dtype != SVQ_F16 && out_dtype != SVQ_BF16) return SVQ_ERR_INVALID_ARG;
+  return cuda_status(svq::launch_dequant(W->packed, W->N, W->K, W->b_d, W->codebook, W->radius_scale,
+                                         W->radius_offset, out_dtype == SVQ_BF16, (uint16_t*)w_out,
+                                         (cudaStream_t)stream));
+}
+
+int svq_linear_gemv_batched_workspace_size(const svq_matrix* mats, int n_mats, int M, size_t* bytes) {
+  if (!bytes) return SVQ_ERR_INVALID_ARG;
+  svq::GemvPlan plan;
+  svq::GemvMatDesc descs[svq::kGemvMaxMats];
+  const int st = plan_group(mats, n_mats, M, &plan, descs, nullptr, nullptr);
+  if (st != SVQ_OK) return st;
+  *bytes = plan.ws_total;
+  return SVQ_OK;
+}
+
+int svq_linear_gemv_workspace_size(const svq_matrix* W, int M, size_t* bytes) {
+  return svq_linear_gemv_batched_workspace_size(W, 1, M, bytes);
+}
+
+int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t stream) {
+  if (bytes == 0) return SVQ_OK;
+  if (!workspace) return SVQ_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream));
+}
+
+int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const uint16_t* const* x, int M,
+                            void* const* y, int y_dtype, void* workspace, size_t workspace_bytes,
+                            svq_stream_t stream) {
+  if (!x || !y) return SVQ_ERR_INVALID_ARG;
+  if (y_dtype != SVQ_F16 && y_dtype != SVQ_F32) return SVQ_ERR_INVALID_ARG;
+  if (n_mats < 1 || n_mats > svq::kGemvMaxMats) return SVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n_mats; ++i) {
+    if (!x[i] || !y[i]) return SVQ_ERR_INVALID_ARG;
+    if (!aligned(x[i], 2) || !aligned(y[i], y_dtype == SVQ_F32 ? 4 : 2)) return SVQ_ERR_INVALID_ARG;
+  }
+  svq::GemvPlan plan;
+  svq::GemvMatDesc descs[svq::kGemvMaxMats];
+  const int st = plan_group(mats, n_mats, M, &plan, descs, x, y);
+  if (st != SVQ_OK) return st;
+  if (plan.ws_total > 0 && (!workspace || workspace_bytes < plan.ws_total || !aligned(workspace, 256)))
+    return SVQ_ERR_WORKSPACE;
+  return cuda_status(svq::launch_gemv(descs, plan, y_dtype == SVQ_F32, workspace, (cudaStream_t)stream));
+}
+
+int svq_linear_gemv(const svq_matrix* W, const uint16_t* x, int M, void* y, int y_dtype, void* workspace,
+                    size_t workspace_bytes, svq_stream_t stream) {
+  void* yy[1] = {y};
+  const uint16_t* xx[1] = {x};
+  if (!x || !y) return SVQ_ERR_INVALID_ARG;
+  return svq_linear_gemv_batched(W, 1, xx, M, yy, y_dtype, workspace, workspace_bytes, stream);
+}
+
+int svq_get_device_status(svq_stream_t stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SVQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return SVQ_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return SVQ_ERR_CUDA;
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,520 @@
+// gemm.cu -- SVQ prefill GEMM on the sm_100a tensor cores:
+//   y[m][n] = sum_j W[n][j] * X[m][perm[j]],  W decoded from SVQ codes on chip.
+//
+// Method ("SAGE", arXiv 2610.14745): subvector = radius * signs (.) codeword
+// (Figure 2 caption); activations are read in the ESG order (Figure 6 caption);
+// the pages' prefill kernel is a "64-row GEMM loop" in which an mma adds
+// A * B_j^T to an accumulator (Figure 6(b) caption) -- warp-level mma on the
+// GPU it was written for.  Here the same contraction runs on tcgen05:
+//
+//   * pass 1 (permute kernel): X_p[m][j] = X[m][perm[j]] into the workspace, so
+//     activation tiles become plain 2-D boxes for TMA;
+//   * pass 2 (this kernel, persistent, one CTA per SM, 10 warps):
+//       warp 0      TMA producer: X_p tiles [BN tokens x 64 k], 128-byte swizzle
+//       warp 1      TMEM allocator and the single MMA-issuing thread:
+//                   tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
+//                   N = BN tokens, K = 16 per instruction, fp32 accumulators
+//                   in TMEM (two buffers of BN columns)
+//       warps 2..5  decoders: packed codes -> 128 x 64 bf16/fp16 weight tile in
+//                   shared memory (K-major, 128-byte swizzle), codebook from
+//                   8 shared-memory replicas; each warp fills its own stages
+//       warps 6..9  epilogue: tcgen05.ld -> registers -> shared staging ->
+//                   coalesced stores of y (or split-K partials + fix-up)
+//   * weights are the A operand (swap-AB), so small token counts still map to
+//     the 128-row MMA; work units are (token tile, k-split, row tile).
+// Weight rows are placed in the A tile in the order rho = lane + 32 * r (lane
+// of the packed lane-block, r = its row 0..3), which makes the decoders'
+// 16-byte swizzled stores conflict free; the epilogue maps TMEM lane rho back to
+// weight row 4 * (rho % 32) + rho / 32.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "gemm_params.h"
+#include "layout.cuh"
+#include "sm100.cuh"
+#include "svq_internal.h"
+
+namespace svq {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 320;
+constexpr int kDecWarp0 = 2, kNumDec = 4;
+constexpr int kEpiWarp0 = 6, kNumEpi = 4;
+constexpr int kATileBytes = 128 * 128;           // 128 rows x 64 k x 2 bytes
+constexpr int kCbBytes = 32 * 1024;               // codebook replicas
+constexpr int kStageCols = 32;                    // epilogue columns per round
+constexpr int kStgBytes = kStageCols * 128 * 4;
+
+struct Smem {
+  // offsets (bytes from the 1024-aligned base)
+  uint32_t a, b, cb, stg, bars;
+};
+
+template <int BN, int NS>
+__host__ __device__ constexpr uint32_t smem_bytes() {
+  return NS * kATileBytes + NS * BN * 128 + kCbBytes + kStgBytes + 1024 /* barriers */ + 1024 /* align */;
+}
+
+struct Bars {
+  uint64_t full_a[8], full_b[8], empty[8], acc_full[2], acc_empty[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int last_flag;
+  int epi_ok;
+};
+
+__device__ __forceinline__ void record_timeout(const GemmKParams& p, Bars* bars) {
+  atomicExch(p.status, 5 /* SVQ_ERR_TIMEOUT */);
+  atomicExch(&bars->abort_flag, 1);
+}
+
+// Wait that gives up on timeout or when another role has aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const GemmKParams& p, Bars* bars) {
+  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63 && *(volatile int*)&bars->abort_flag) return false;
+  }
+  record_timeout(p, bars);
+  return false;
+}
+
+struct Unit {
+  int nt, mt, s, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit unit_of(const GemmKParams& p, int u) {
+  Unit w;
+  w.nt = u % p.n_tiles;
+  const int rest = u / p.n_tiles;
+  w.s = rest % p.S;
+  w.mt = rest / p.S;
+  const int KB = p.K / 64;
+  w.kb0 = (int)(((long long)KB * w.s) / p.S);
+  w.kb1 = (int)(((long long)KB * (w.s + 1)) / p.S);
+  return w;
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  uint32_t r;
+  if constexpr (BF16) {
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  } else {
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  }
+  return r;
+}
+
+// Decode one 64-column stage of one 128-row tile into the swizzled A tile.
+template <bool BF16>
+__device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int kb, uint8_t* a_tile,
+                                             const uint8_t* cbs, int lane) {
+  const int L = tile_lanes(p.N, nt);
+  if (lane >= L) return;
+  const int b = kb >> 1, h = kb & 1;
+  const uint8_t* blk = p.packed + tile_offset(p.K, nt) + (size_t)b * L * kLaneBlockBytes;
+  uint32_t w[kWords];
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(blk + ((size_t)c * L + lane) * 16));
+    w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+  }
+  const int bd = p.b_d;
+  const uint32_t imask = (1u << bd) - 1u;
+  const uint32_t cmask = (1u << (10 - bd)) - 1u;
+  const int rep = p.cb_replicas;
+  const uint8_t* cbq = cbs + (lane & (rep - 1)) * 16;
+  const int cb_stride = rep * 16;                      // bytes per codebook entry (all replicas)
+  const int n0 = nt * kTileRows + 4 * lane;
+  float sc[4], of[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    sc[r] = __half2float(__ushort_as_half(p.scale[n0 + r]));
+    of[r] = __half2float(__ushort_as_half(p.offset[n0 + r]));
+  }
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      if (hh != h) continue;
+      const int j = 8 * hh + jj;
+      const uint32_t S = w[j];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int v = 4 * j + r;
+        uint32_t pay;
+        if (v < 60) {
+          pay = w[16 + v / 3] >> (10 * (v % 3));
+        } else {
+          const int a = v - 60;
+          pay = ((w[16 + 5 * a] >> 30) << 8) | ((w[17 + 5 * a] >> 30) << 6) | ((w[18 + 5 * a] >> 30) << 4) |
+                ((w[19 + 5 * a] >> 30) << 2) | (w[20 + 5 * a] >> 30);
+        }
+        const uint32_t id = pay & imask;
+        const uint32_t code = (pay >> bd) & cmask;
+        const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
+        const float rad = __fmaf_rn(sc[r], (float)code, of[r]);
+        const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
+        uint32_t o4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __half2 hv = *reinterpret_cast<const __half2*>(&c4[q]);
+          const float lo = __fmul_rn(rad, __low2float(hv));
+          const float hi = __fmul_rn(rad, __high2float(hv));
+          o4[q] = pack2<BF16>(lo, hi) ^ ((S << (4 * r + q)) & 0x80008000u);
+        }
+        const int rho = lane + 32 * r;                   // A-tile row of weight row n0 + r
+        const int kc = jj;                               // 16-byte chunk within the 128-byte row
+        uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      }
+    }
+  }
+}
+
+template <int BN, int NS, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmKParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* a_st = base;
+  uint8_t* b_st = a_st + NS * kATileBytes;
+  uint8_t* cbs = b_st + NS * BN * 128;
+  float* stg = reinterpret_cast<float*>(cbs + kCbBytes);
+  Bars* bars = reinterpret_cast<Bars*>(reinterpret_cast<uint8_t*>(stg) + kStgBytes);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr uint32_t kTmemCols = (2 * BN) <= 32 ? 32 : (2 * BN) <= 64 ? 64 : (2 * BN) <= 128 ? 128
+                                 : (2 * BN) <= 256 ? 256 : 512;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&bars->full_a[s], 1);
+      mbar_init(&bars->full_b[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->acc_full[i], 1);
+      mbar_init(&bars->acc_empty[i], kNumEpi);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    bars->last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  // Codebook replicas: entry e, replica q at 16-byte slot e * rep + q.
+  {
+    const int rep = p.cb_replicas;
+    const int n = (1 << p.b_d) * rep;
+    for (int i = threadIdx.x; i < n; i += kThreads)
+      reinterpret_cast<uint4*>(cbs)[i] = __ldg(p.codebook + i / rep);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int n_units = p.n_tiles * p.m_tiles * p.S;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const Unit w = unit_of(p, u);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int s = it % NS;
+          const uint32_t ph = (it / NS) & 1;
+          if (it >= NS && !wait_bar(&bars->empty[s], ph ^ 1, p, bars)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars->full_b[s], BN * 128);
+          tma_load_2d(b_st + s * BN * 128, &tmap_x, &bars->full_b[s], kb * 64, w.mt * BN);
+        }
+      }
+      if (!ok) {
+        // Let copies already issued land before the CTA exits.
+        for (int k = std::max(0, it - NS); k < it; ++k) mbar_wait(&bars->full_b[k % NS], (k / NS) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(BF16 ? 1 : 0, BN);
+      int it = 0, acc_it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++acc_it) {
+        const Unit w = unit_of(p, u);
+        const int buf = acc_it & 1;
+        const uint32_t aph = (acc_it >> 1) & 1;
+        if (acc_it >= 2 && !wait_bar(&bars->acc_empty[buf], aph ^ 1, p, bars)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * BN;
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int s = it % NS;
+          const uint32_t ph = (it / NS) & 1;
+          if (!wait_bar(&bars->full_a[s], ph, p, bars) || !wait_bar(&bars->full_b[s], ph, p, bars)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc_sw128(smem_u32(a_st + s * kATileBytes));
+          const uint64_t bd = smem_desc_sw128(smem_u32(b_st + s * BN * 128));
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16)
+            mma_f16(d_tmem, ad + 2 * k16, bd + 2 * k16, idesc, (kb > w.kb0 || k16 > 0) ? 1u : 0u);
+          mma_commit(&bars->empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&bars->acc_full[buf]);
+      }
+      // All MMAs issued by this thread are complete before TMEM is released.
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0);
+    }
+  } else if (warp < kEpiWarp0) {
+    // ---------------- decoders
+    const int d = warp - kDecWarp0;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const Unit w = unit_of(p, u);
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+        if (it % kNumDec != d) continue;
+        const int s = it % NS;
+        const uint32_t ph = (it / NS) & 1;
+        int good = 1;
+        if (it >= NS && lane == 0) good = wait_bar(&bars->empty[s], ph ^ 1, p, bars) ? 1 : 0;
+        good = __shfl_sync(0xFFFFFFFFu, good, 0);
+        if (!good) { ok = false; break; }
+        decode_stage<BF16>(p, w.nt, kb, a_st + s * kATileBytes, cbs, lane);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->full_a[s]);
+      }
+    }
+  } else {
+    // ---------------- epilogue
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int e = warp - kEpiWarp0;          // 0..3
+    int acc_it = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++acc_it) {
+      const Unit w = unit_of(p, u);
+      const int buf = acc_it & 1;
+      const uint32_t aph = (acc_it >> 1) & 1;
+      if (threadIdx.x == kEpiWarp0 * 32) bars->epi_ok = wait_bar(&bars->acc_full[buf], aph, p, bars) ? 1 : 0;
+      named_bar_sync(1, kNumEpi * 32);
+      if (!bars->epi_ok) break;
+      tc_fence_after();
+      const int n0 = w.nt * kTileRows;
+      const int rows = min(kTileRows, p.N - n0);
+      const bool split = p.S > 1;
+      for (int c0 = 0; c0 < BN; c0 += kStageCols) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c0, v);
+        tmem_ld_wait();
+        const int nl = 4 * lane + q;         // weight row of TMEM lane 32q + lane
+#pragma unroll
+        for (int i = 0; i < 32; ++i) stg[i * 128 + nl] = __uint_as_float(v[i]);
+        named_bar_sync(1, kNumEpi * 32);
+        for (int i = e * 8; i < e * 8 + 8; ++i) {
+          const int m = w.mt * BN + c0 + i;
+          if (m >= p.M || 4 * lane >= rows) continue;
+          const float4 val = *reinterpret_cast<const float4*>(stg + i * 128 + 4 * lane);
+          const int n = n0 + 4 * lane;
+          if (split) {
+            float* dst = p.partial + ((size_t)w.s * p.M + m) * p.N + n;
+            *reinterpret_cast<float4*>(dst) = val;
+          } else if (p.y_f32) {
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)m * p.N + n) = val;
+          } else {
+            uint2 pk;
+            pk.x = pack2<true>(val.x, val.y);
+            pk.y = pack2<true>(val.z, val.w);
+            *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + (size_t)m * p.N + n) = pk;
+          }
+        }
+        named_bar_sync(1, kNumEpi * 32);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
+      if (split) {
+        // The last CTA to finish a (row tile, token tile) sums the split-K partials in order.
+        __threadfence();
+        named_bar_sync(1, kNumEpi * 32);
+        if (threadIdx.x == kEpiWarp0 * 32) {
+          const unsigned prev = atomicAdd(&p.counters[w.mt * p.n_tiles + w.nt], 1u);
+          bars->last_flag = (prev == (unsigned)(p.S - 1));
+        }
+        named_bar_sync(1, kNumEpi * 32);
+        if (bars->last_flag) {
+          __threadfence();
+          const int tcols = min(BN, p.M - w.mt * BN);
+          for (int idx = threadIdx.x - kEpiWarp0 * 32; idx < tcols * (rows / 4); idx += kNumEpi * 32) {
+            const int i = idx / (rows / 4), n = n0 + 4 * (idx % (rows / 4));
+            const int m = w.mt * BN + i;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int k = 0; k < p.S; ++k) {
+              const float4 t = __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)k * p.M + m) * p.N + n));
+              acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+            }
+            if (p.y_f32) {
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)m * p.N + n) = acc;
+            } else {
+              uint2 pk;
+              pk.x = pack2<true>(acc.x, acc.y);
+              pk.y = pack2<true>(acc.z, acc.w);
+              *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + (size_t)m * p.N + n) = pk;
+            }
+          }
+          if (threadIdx.x == kEpiWarp0 * 32) p.counters[w.mt * p.n_tiles + w.nt] = 0u;
+        }
+        named_bar_sync(1, kNumEpi * 32);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// X_p[m][j] = X[m][perm[j]] (16-bit values), eight columns per thread.
+__global__ void permute_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int M, int K,
+                               uint16_t* __restrict__ xp) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long per_row = K / 8;
+  if (i >= (long long)M * per_row) return;
+  const int m = (int)(i / per_row);
+  const int j0 = (int)(i % per_row) * 8;
+  const uint16_t* xr = x + (size_t)m * K;
+  uint16_t v[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = xr[__ldg(perm + j0 + k)];
+  uint4 o;
+  o.x = v[0] | ((uint32_t)v[1] << 16);
+  o.y = v[2] | ((uint32_t)v[3] << 16);
+  o.z = v[4] | ((uint32_t)v[5] << 16);
+  o.w = v[6] | ((uint32_t)v[7] << 16);
+  *reinterpret_cast<uint4*>(xp + (size_t)m * K + j0) = o;
+}
+
+template <int BN, int NS, bool BF16>
+cudaError_t launch_bn(const CUtensorMap& tm, const GemmKParams& p, int grid, cudaStream_t st) {
+  constexpr uint32_t smem = smem_bytes<BN, NS>();
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, NS, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  gemm_kernel<BN, NS, BF16><<<grid, kThreads, smem, st>>>(tm, p);
+  return cudaGetLastError();
+}
+
+template <bool BF16>
+cudaError_t launch_typed(int BN, const CUtensorMap& tm, const GemmKParams& p, int grid, cudaStream_t st) {
+  switch (BN) {
+    case 16: return launch_bn<16, 6, BF16>(tm, p, grid, st);
+    case 32: return launch_bn<32, 6, BF16>(tm, p, grid, st);
+    case 64: return launch_bn<64, 5, BF16>(tm, p, grid, st);
+    case 128: return launch_bn<128, 4, BF16>(tm, p, grid, st);
+    default: return launch_bn<256, 3, BF16>(tm, p, grid, st);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
+  GemmPlan g{};
+  g.BN = M >= 256 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : (M > 16 ? 32 : 16)));
+  g.m_tiles = (M + g.BN - 1) / g.BN;
+  g.n_tiles = num_tiles(N);
+  const int T = g.n_tiles * g.m_tiles;
+  const int KB = K / 64;
+  double best = 1e30;
+  g.S = 1;
+  for (int S = 1; S <= std::min(16, std::max(1, KB / 4)); ++S) {
+    const double waves = std::ceil((double)T * S / num_sms);
+    const double est = waves / S * (1.0 + 0.04 * (S - 1));
+    if (est < best - 1e-9) { best = est; g.S = S; }
+  }
+  g.grid = std::min(T * g.S, num_sms);
+  const size_t xp = ((size_t)M * K * 2 + 255) / 256 * 256;
+  g.xp_offset = 0;
+  g.partial_offset = xp;
+  size_t part = 0, cnt = 0;
+  if (g.S > 1) {
+    part = ((size_t)g.S * M * N * 4 + 255) / 256 * 256;
+    cnt = ((size_t)T * 4 + 255) / 256 * 256;
+  }
+  g.counter_offset = xp + part;
+  g.ws_bytes = xp + part + cnt;
+  return g;
+}
+
+cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* status, cudaStream_t st) {
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  uint16_t* xp = reinterpret_cast<uint16_t*>(wsb + g.xp_offset);
+  {
+    const long long work = (long long)d.M * (d.K / 8);
+    permute_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(d.x, d.perm, d.M, d.K, xp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tm;
+  const cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)d.M};
+  const cuuint64_t strides[1] = {(cuuint64_t)d.K * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)g.BN};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(&tm, d.x_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xp,
+                         dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  GemmKParams p{};
+  p.packed = reinterpret_cast<const uint8_t*>(d.packed);
+  p.codebook = reinterpret_cast<const uint4*>(d.codebook);
+  p.scale = d.scale;
+  p.offset = d.offset;
+  p.N = d.N; p.K = d.K; p.b_d = d.b_d; p.M = d.M;
+  p.n_tiles = g.n_tiles; p.m_tiles = g.m_tiles; p.S = g.S;
+  p.cb_replicas = d.b_d <= 8 ? 8 : (d.b_d == 9 ? 4 : 2);
+  p.y = d.y;
+  p.y_f32 = d.y_f32;
+  p.partial = g.S > 1 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
+  p.counters = g.S > 1 ? reinterpret_cast<unsigned*>(wsb + g.counter_offset) : nullptr;
+  p.status = status;
+  return d.x_bf16 ? launch_typed<true>(g.BN, tm, p, g.grid, st) : launch_typed<false>(g.BN, tm, p, g.grid, st);
+}
+
+}  // namespace svq

@@ -1,0 +1,46 @@
+// gemm_params.h -- parameter block and launch plan of the tensor-core GEMM.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace svq {
+
+struct GemmKParams {
+  const uint8_t* packed;
+  const uint4* codebook;
+  const uint16_t* scale;
+  const uint16_t* offset;
+  int N, K, b_d, M;
+  int n_tiles, m_tiles, S;
+  int cb_replicas;
+  void* y;
+  int y_f32;
+  float* partial;       // [S][M][N] when S > 1
+  unsigned* counters;   // [m_tiles * n_tiles]
+  int* status;          // device status word (bounded-wait timeouts)
+};
+
+struct GemmPlan {
+  int BN, m_tiles, n_tiles, S, grid;
+  size_t xp_offset, partial_offset, counter_offset, ws_bytes;
+};
+
+struct GemmMatDesc {
+  int N, K, b_d, M;
+  const void* packed;
+  const uint16_t* codebook;
+  const uint16_t* scale;
+  const uint16_t* offset;
+  const int32_t* perm;
+  const uint16_t* x;    // [M][K], fp16 or bf16 (x_bf16)
+  int x_bf16;
+  void* y;              // [M][N], fp32 (y_f32) or bf16
+  int y_f32;
+};
+
+GemmPlan plan_gemm(int N, int K, int M, int num_sms);
+cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* status, cudaStream_t st);
+
+}  // namespace svq

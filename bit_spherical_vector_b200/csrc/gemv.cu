@@ -1,0 +1,136 @@
+// gemv.cu -- launch planning for the fused SVQ decode-and-multiply for small batches (1..8 tokens per
+// pass), y = W x[perm], over a group of up to eight independent matrices in one
+// launch.
+//
+// Method ("SAGE", arXiv 2610.14745): a subvector of eight weights is
+// r * sign (.) c_idx (Figure 2 caption: signs, direction index, quantized
+// radius); it multiplies eight reordered activations x[perm[8g..8g+7]]
+// (Figure 6 caption); weights are reconstructed on demand, never stored dense
+// (Figures 1 and 5).
+//
+// B200 mapping:
+//   * a CTA of 8 warps works on one matrix, one k-slice and up to 8 row tiles;
+//     each warp owns a 128-row tile and each lane owns 4 complete rows, so a
+//     row's partial sum never leaves its thread (no shuffles in the hot loop);
+//   * packed codes stream from HBM with 16-byte coalesced loads
+//     (ld.global.nc.L1::no_allocate), one block (9 loads per lane) ahead;
+//   * the fp16 codebook sits in shared memory as 8 replicas, entry e of
+//     replica q at 16-byte slot 8e + q, and lane l reads replica l % 8: the 8
+//     lanes of each quarter-warp phase of an LDS.128 hit 8 different bank
+//     groups whatever the indices, so the random gather is conflict free;
+//   * x[perm] for the CTA's k-slice is gathered into shared memory once and
+//     read with broadcast loads;
+//   * signs are applied by XOR on fp16 sign bits; the eight products of a
+//     subvector are summed in fp16x2, then scaled by the radius and
+//     accumulated across subvectors in fp32;
+//   * split-K partials go to the workspace; the last CTA of a row chunk (found
+//     with a counter) sums them in a fixed order, so results are reproducible.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "gemv_params.h"
+#include "layout.cuh"
+#include "svq_internal.h"
+
+namespace svq {
+namespace {
+
+constexpr size_t kSmemPerCtaTwo = 110 * 1024;   // two CTAs per SM
+constexpr size_t kSmemPerCtaOne = kGemvSmemMax;
+
+size_t cta_smem(int b_d, int mt, int K, int S) {
+  const int B = K / kBlockCols;
+  const int nbmax = (B + S - 1) / S;
+  return ((size_t)16 << b_d) * 8 + (size_t)mt * nbmax * kBlockCols * 2;
+}
+
+}  // namespace
+
+bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan* plan) {
+  if (n_mats < 1 || n_mats > kGemvMaxMats || M < 1) return false;
+  const int mt = M >= 5 ? 8 : (M >= 3 ? 4 : M);
+  plan->n_mats = n_mats;
+  plan->M = M;
+  plan->mt = mt;
+  const int per_sm = mt <= 2 ? 2 : 1;
+  const size_t smem_cap = per_sm == 2 ? kSmemPerCtaTwo : kSmemPerCtaOne;
+  const double budget = (double)num_sms * per_sm;
+  double total = 0;
+  for (int i = 0; i < n_mats; ++i) total += (double)packed_bytes(mats[i].N, mats[i].K);
+  size_t off = 0;
+  int ctas = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    const GemvMatDesc& d = mats[i];
+    const int R = num_tiles(d.N), RC = (R + kGemvWarps - 1) / kGemvWarps, B = d.K / kBlockCols;
+    const double share = std::max(1.0, budget * (double)packed_bytes(d.N, d.K) / total);
+    int S = (int)std::lround(share / RC);
+    S = std::max(1, std::min(S, B));
+    while (S < B && cta_smem(d.b_d, mt, d.K, S) > smem_cap) ++S;
+    if (cta_smem(d.b_d, mt, d.K, S) > kSmemPerCtaOne) return false;
+    GemvPlanMat& pm = plan->m[i];
+    pm.S = S;
+    pm.n_rc = RC;
+    pm.ctas = S * RC;
+    pm.ws_offset = off;
+    pm.ws_bytes = 0;
+    if (S > 1) {
+      const size_t part = ((size_t)S * mt * d.N * sizeof(float) + 255) / 256 * 256;
+      const size_t cnt = ((size_t)RC * sizeof(unsigned) + 255) / 256 * 256;
+      pm.ws_bytes = part + cnt;
+    }
+    off += pm.ws_bytes;
+    ctas += pm.ctas;
+  }
+  plan->ws_total = off;
+  plan->total_ctas = ctas;
+  return true;
+}
+
+cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32, void* ws, cudaStream_t st) {
+  const int mt = plan.mt;
+  const int passes = (plan.M + mt - 1) / mt;
+  for (int p = 0; p < passes; ++p) {
+    const int m0 = p * mt, Mp = std::min(mt, plan.M - m0);
+    GemvKParams kp{};
+    kp.n_mats = plan.n_mats;
+    kp.y_f32 = y_f32;
+    size_t smem = 0;
+    int cta = 0;
+    for (int i = 0; i < plan.n_mats; ++i) {
+      const GemvMatDesc& d = mats[i];
+      const GemvPlanMat& pm = plan.m[i];
+      GemvKMat& g = kp.mats[i];
+      g.packed = reinterpret_cast<const uint8_t*>(d.packed);
+      g.codebook = reinterpret_cast<const uint4*>(d.codebook);
+      g.scale = d.scale;
+      g.offset = d.offset;
+      g.perm = d.perm;
+      g.x = d.x + (size_t)m0 * d.K;
+      g.y = reinterpret_cast<char*>(d.y) + (size_t)m0 * d.N * (y_f32 ? 4 : 2);
+      if (pm.S > 1) {
+        char* base = reinterpret_cast<char*>(ws) + pm.ws_offset;
+        g.partial = reinterpret_cast<float*>(base);
+        g.counters = reinterpret_cast<unsigned*>(base + ((size_t)pm.S * mt * d.N * sizeof(float) + 255) / 256 * 256);
+      } else {
+        g.partial = nullptr;
+        g.counters = nullptr;
+      }
+      g.N = d.N; g.K = d.K; g.b_d = d.b_d; g.S = pm.S; g.n_rc = pm.n_rc; g.cta_begin = cta; g.M = Mp;
+      cta += pm.ctas;
+      smem = std::max(smem, cta_smem(d.b_d, mt, d.K, pm.S));
+    }
+    cudaError_t e;
+    switch (mt) {
+      case 1: e = launch_gemv_mt<1>(kp, cta, smem, st); break;
+      case 2: e = launch_gemv_mt<2>(kp, cta, smem, st); break;
+      case 4: e = launch_gemv_mt<4>(kp, cta, smem, st); break;
+      default: e = launch_gemv_mt<8>(kp, cta, smem, st); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace svq

@@ -1,0 +1,167 @@
+/*
+ * svq.h -- C ABI of libsvq, the B200 (sm_100a) library for SAGE's 2-bit
+ * spherical vector quantization (SVQ) linear layer, y = W x.
+ *
+ * The method ("SAGE: Pushing 2-Bit Vector-Quantized LLMs toward Real-World
+ * Usability", arXiv 2610.14745):
+ *   - Figure 2 caption: each subvector of eight weights is stored as eight
+ *     signs, a direction index into a per-matrix codebook and a quantized
+ *     radius, 18 bits per eight weights; the 10 non-sign bits are split
+ *     between direction (b_d) and radius (b_r = 10 - b_d) per matrix (ABS).
+ *   - Figure 6 caption: the kernel multiplies each decoded subvector by eight
+ *     reordered activations (the ESG input-channel permutation).
+ *   - Figures 1 and 5 captions: weights are reconstructed on demand; no dense
+ *     copy of W is kept.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller, except where
+ *     a parameter says "host".  The library never allocates or frees memory
+ *     and never synchronises the device (svq_get_device_status excepted).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy stream) and
+ *     runs asynchronously; the return value reports argument validation and
+ *     launch errors only.
+ *   - fp16 / bf16 values are passed as 16-bit bit patterns (uint16_t).
+ *   - Shapes: K % 8 == 0 is the format's own rule.  The device layout and all
+ *     kernels additionally need K % 128 == 0 and N % 4 == 0; other shapes return
+ *     SVQ_ERR_UNSUPPORTED_SHAPE.  1 <= b_d <= 10.
+ *   - Return codes: SVQ_OK or one of the SVQ_ERR_* values below; nothing is
+ *     enqueued when an error is returned.
+ */
+#ifndef SVQ_H_
+#define SVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SVQ_API __attribute__((visibility("default")))
+#else
+#define SVQ_API
+#endif
+
+typedef struct CUstream_st* svq_stream_t; /* same type as cudaStream_t */
+
+enum svq_status {
+  SVQ_OK = 0,
+  SVQ_ERR_INVALID_ARG = 1,       /* NULL or misaligned pointer, bad enum, M out of range */
+  SVQ_ERR_UNSUPPORTED_SHAPE = 2, /* N, K or b_d outside what the kernels handle */
+  SVQ_ERR_WORKSPACE = 3,         /* workspace NULL or smaller than the *_workspace_size query */
+  SVQ_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, attribute) */
+  SVQ_ERR_TIMEOUT = 5            /* a kernel's bounded wait ran out (read by svq_get_device_status) */
+};
+
+enum svq_dtype { SVQ_F16 = 1, SVQ_BF16 = 2, SVQ_F32 = 3 };
+
+/* One SVQ matrix W[N][K].  Column j of the stored order multiplies x[perm[j]]. */
+typedef struct svq_matrix {
+  int32_t N;                      /* output features (rows of W)                            */
+  int32_t K;                      /* input features                                         */
+  int32_t b_d;                    /* direction-index bits; radius code has 10 - b_d bits    */
+  int32_t reserved;               /* must be 0                                              */
+  const void* packed;             /* device layout written by svq_repack, svq_packed_bytes  */
+  const uint16_t* codebook;       /* fp16 [1 << b_d][8], 16-byte aligned                    */
+  const uint16_t* radius_scale;   /* fp16 [N]                                               */
+  const uint16_t* radius_offset;  /* fp16 [N]                                               */
+  const int32_t* perm;            /* [K], a permutation of 0..K-1                           */
+} svq_matrix;
+
+/* Message for a status code (static string). */
+SVQ_API const char* svq_status_string(int status);
+
+/* Library version, e.g. 100 for 0.1.0. */
+SVQ_API int svq_version(void);
+
+/* Bytes of the device layout of an N x K matrix: exactly N * K * 9 / 32 (18 bits
+ * per 8 weights, Figure 2 caption), the same size as the canonical stream.
+ * Returns 0 for shapes the layout does not support. */
+SVQ_API size_t svq_packed_bytes(int N, int K);
+
+/* Bytes of the canonical stream: N * ceil(18 * (K/8) / 8). */
+SVQ_API size_t svq_canonical_bytes(int N, int K);
+
+/*
+ * svq_repack -- lossless conversion of the canonical code stream into the
+ * device layout used by every kernel (done once per matrix, offline).
+ *
+ * canonical [N][ceil(18*(K/8)/8)] bytes: row n, subvector g occupies stream bits
+ *   [18g, 18g+18) of the row, stream bit b = bit (b mod 8) of byte b/8 (LSB
+ *   first); code word bits 0..7 = signs (bit i -> element i, 1 = negative),
+ *   bits 8..8+b_d-1 = direction index, the remaining b_r bits = radius code.
+ *   (The pages give the 18-bit budget and the three fields, Figure 2 caption;
+ *   the bit order is this library's interchange reading.)
+ * packed_out: svq_packed_bytes(N, K) bytes, 16-byte aligned.
+ * The device layout groups 4 rows x 16 subvectors (144 bytes) per lane so that a
+ * warp streams 16-byte coalesced loads; it holds exactly the same bits.
+ */
+SVQ_API int svq_repack(const uint8_t* canonical, int N, int K, int b_d, void* packed_out,
+               svq_stream_t stream);
+
+/*
+ * svq_unpack_fields -- decode the device layout back into per-subvector fields
+ * (test and inspection aid).  signs [N][K/8] uint8, idx [N][K/8] uint16,
+ * code [N][K/8] uint16.  Bit-exact inverse of svq_repack.
+ */
+SVQ_API int svq_unpack_fields(const void* packed, int N, int K, int b_d, uint8_t* signs,
+                      uint16_t* idx, uint16_t* code, svq_stream_t stream);
+
+/*
+ * svq_dequantize -- export the dense weights in the stored (permuted) column
+ * order, w_out [N][K] of out_dtype SVQ_F16 or SVQ_BF16.  Per element:
+ *   r = fmaf(scale_n, code, offset_n) in fp32 (the quantized radius, Figure 2),
+ *   w = round_to_nearest_even(r * c_{idx,i}) (binary32 product, then fp16/bf16),
+ *   then the sign bit is set when the code's sign bit is 1 (a zero becomes -0).
+ * Bit-exact against the reference decoder.
+ */
+SVQ_API int svq_dequantize(const svq_matrix* W /* host struct */, int out_dtype, void* w_out,
+                   svq_stream_t stream);
+
+/*
+ * Workspace for svq_linear_gemv / svq_linear_gemv_batched: split-K partial sums
+ * and completion counters.  The counter region must be zero before the first
+ * call that uses a workspace (svq_workspace_init does that); every completed
+ * call leaves it zero again, so one workspace can serve a stream of calls.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+SVQ_API int svq_linear_gemv_workspace_size(const svq_matrix* W /* host */, int M, size_t* bytes);
+SVQ_API int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t stream);
+
+/*
+ * svq_linear_gemv -- decode-and-multiply for batch 1 to 16:
+ *   y[m][n] = sum_j W[n][j] * x[m][perm[j]],  m < M, with W decoded on the fly.
+ * x: fp16 [M][K] (natural input order; the kernel applies perm, Figure 6).
+ * y: [M][N] of y_dtype SVQ_F16 or SVQ_F32.  fp32 accumulation across
+ * subvectors; each subvector's eight products are summed in fp16x2 pairs.
+ * Error bound used by the tests: |y - y_ref| <= 1e-3 * sum_j |W[n][j]||x[m][perm[j]]|.
+ */
+SVQ_API int svq_linear_gemv(const svq_matrix* W /* host */, const uint16_t* x, int M, void* y,
+                    int y_dtype, void* workspace, size_t workspace_bytes, svq_stream_t stream);
+
+/*
+ * svq_linear_gemv_batched -- several independent layers in one launch
+ * (e.g. the seven linears of a decoder layer, or q|k|v sharing one x):
+ *   y_i = W_i x_i for i < n_mats (n_mats <= 8), each with its own M-row input.
+ * mats, x, y are HOST arrays of n_mats entries (x[i], y[i] device pointers).
+ * Workspace: the sum over i of svq_linear_gemv_workspace_size(mats[i], M)
+ * rounded up to 256 bytes each, in order (svq_linear_gemv_batched_workspace_size).
+ */
+SVQ_API int svq_linear_gemv_batched_workspace_size(const svq_matrix* mats, int n_mats, int M,
+                                           size_t* bytes);
+SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const uint16_t* const* x,
+                            int M, void* const* y, int y_dtype, void* workspace,
+                            size_t workspace_bytes, svq_stream_t stream);
+
+/*
+ * Synchronising read-and-clear of the device status word that kernels set
+ * when a bounded wait runs out (SVQ_OK or SVQ_ERR_TIMEOUT).  Tests only.
+ */
+SVQ_API int svq_get_device_status(svq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVQ_H_ */

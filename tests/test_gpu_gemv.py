@@ -1,0 +1,154 @@
+"""GPU parity of the fused decode-and-multiply GEMV against the CPU oracle.
+
+Bar: max |y - y_ref| / sum_j |W[n][j]| |x[m][perm[j]]| <= 1e-3 (fp32 accumulate
+across subvectors), on every output for sizes the oracle finishes quickly, and
+at the full decoder-layer and 8192 x 8192 sizes on every output as well (the
+fp64 oracle handles them in seconds).  Also: permutation metamorphic test,
+run-to-run bit reproducibility, fp16 outputs, the grouped launch."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.gpu_util import need_gpu, rel_err, torch, u16, x_f16
+
+import bit_spherical_vector_b200 as svq
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+
+
+def _run(W, x_bits, y_dtype=torch.float32):
+    M = x_bits.shape[0]
+    x = x_f16(x_bits)
+    y = torch.empty((M, W.N), dtype=y_dtype, device="cuda")
+    nb = svq.svq_linear_gemv_workspace_size(W, M)
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device="cuda")
+    svq.svq_workspace_init(ws)
+    svq.svq_linear_gemv(W, x, y, ws)
+    torch.cuda.synchronize()
+    return y, ws
+
+
+def test_single_layer_1024():
+    need_gpu()
+    m, x = synth.single_layer_1024()
+    W = svq.SvqWeight.from_synth(m)
+    y, _ = _run(W, x)
+    y_ref, den = oracle.linear(m, x)
+    assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
+
+
+@pytest.mark.parametrize("b_d", range(1, 11))
+@pytest.mark.parametrize("N,K", [(4, 128), (132, 256), (388, 640), (1024, 1152)])
+def test_gemv_every_split_and_ragged_tiles(N, K, b_d):
+    need_gpu()
+    m = synth.make_matrix(60, 10 * b_d + N % 7, N, K, b_d)
+    x = synth.make_x(60, 10 * b_d + N % 7, 1, K)
+    W = svq.SvqWeight.from_synth(m)
+    y, _ = _run(W, x)
+    y_ref, den = oracle.linear(m, x)
+    assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 8, 9, 16])
+def test_gemv_small_batches(M):
+    need_gpu()
+    m = synth.make_matrix(61, M, 640, 2560, 7)
+    x = synth.make_x(61, M, M, 2560)
+    W = svq.SvqWeight.from_synth(m)
+    y, _ = _run(W, x)
+    y_ref, den = oracle.linear(m, x)
+    assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
+
+
+def test_gemv_fp16_output():
+    need_gpu()
+    m = synth.make_matrix(62, 0, 512, 1024, 8)
+    x = synth.make_x(62, 0, 2, 1024)
+    W = svq.SvqWeight.from_synth(m)
+    y, _ = _run(W, x, torch.float16)
+    y_ref, den = oracle.linear(m, x)
+    # fp16 output adds one rounding of y (relative 2^-11 of |y| <= den)
+    assert rel_err(y.float().cpu().numpy(), y_ref, den) <= TOL + 2.0 ** -11
+
+
+def test_permutation_metamorphic_bit_exact():
+    """y(W, perm, x) == y(W, identity, x[perm]) bit for bit (same data order in the kernel)."""
+    need_gpu()
+    m = synth.make_matrix(63, 0, 256, 1024, 8)
+    x = synth.make_x(63, 0, 1, 1024)
+    W = svq.SvqWeight.from_synth(m)
+    mid = synth.make_matrix(63, 0, 256, 1024, 8, identity_perm=True)
+    Wid = svq.SvqWeight.from_synth(mid)
+    y1, _ = _run(W, x)
+    y2, _ = _run(Wid, np.ascontiguousarray(x[:, m.perm]))
+    assert torch.equal(y1, y2)
+
+
+def test_reproducible_and_workspace_reusable():
+    """Split-K partials are reduced in a fixed order: repeated calls on one workspace agree bit for bit,
+    and the completion counters are left at zero."""
+    need_gpu()
+    m = synth.make_matrix(64, 0, 2560, 9728, 8)
+    x = synth.make_x(64, 0, 1, 9728)
+    W = svq.SvqWeight.from_synth(m)
+    y1, ws = _run(W, x)
+    xd = x_f16(x)
+    ys = []
+    for _ in range(3):
+        y = torch.empty_like(y1)
+        svq.svq_linear_gemv(W, xd, y, ws)
+        ys.append(y)
+    torch.cuda.synchronize()
+    for y in ys:
+        assert torch.equal(y, y1)
+    y_ref, den = oracle.linear(m, x)
+    assert rel_err(y1.cpu().numpy(), y_ref, den) <= TOL
+
+
+def test_workspace_too_small_rejected():
+    need_gpu()
+    m = synth.make_matrix(65, 0, 2560, 9728, 8)
+    W = svq.SvqWeight.from_synth(m)
+    nb = svq.svq_linear_gemv_workspace_size(W, 1)
+    assert nb > 0
+    x = torch.zeros((1, 9728), dtype=torch.float16, device="cuda")
+    y = torch.empty((1, 2560), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(nb - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(svq.SvqError) as e:
+        svq.svq_linear_gemv(W, x, y, ws)
+    assert e.value.status == svq.SVQ_ERR_WORKSPACE
+
+
+def test_decoder_layer_grouped_full_size():
+    """The seven linears of a Qwen3-4B-shaped decoder layer (batch 1) in one grouped launch,
+    every output checked against the oracle."""
+    need_gpu()
+    layer = synth.qwen3_4b_layer(0)
+    Ws = [svq.SvqWeight.from_synth(m) for m, _ in layer]
+    xs = [x_f16(x) for _, x in layer]
+    ys = [torch.empty((1, m.N), dtype=torch.float32, device="cuda") for m, _ in layer]
+    nb = svq.svq_linear_gemv_batched_workspace_size(Ws, 1)
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device="cuda")
+    svq.svq_workspace_init(ws)
+    svq.svq_linear_gemv_batched(Ws, xs, ys, ws)
+    torch.cuda.synchronize()
+    for (m, x), y in zip(layer, ys):
+        y_ref, den = oracle.linear(m, x)
+        assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL, m.name
+    # the grouped launch equals the per-matrix launches
+    for (m, x), W, y in zip(layer, Ws, ys):
+        y1, _ = _run(W, x)
+        assert rel_err(y1.cpu().numpy(), y.cpu().numpy().astype(np.float64), oracle.linear(m, x)[1]) <= 1e-6
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 8, 16])
+def test_square_8192_sweep(M):
+    need_gpu()
+    m = synth.square_8192()
+    x = synth.square_8192_x(M)
+    W = svq.SvqWeight.from_synth(m)
+    y, _ = _run(W, x)
+    y_ref, den = oracle.linear(m, x)
+    assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
