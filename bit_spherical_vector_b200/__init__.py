@@ -66,6 +66,8 @@ def lib():
         "svq_linear_gemv": ([MP, P, I, P, I, P, SZ, P], I),
         "svq_linear_gemv_batched_workspace_size": ([MP, I, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemv_batched": ([MP, I, ctypes.POINTER(P), I, ctypes.POINTER(P), I, P, SZ, P], I),
+        "svq_linear_gemm_workspace_size": ([MP, I, ctypes.POINTER(SZ)], I),
+        "svq_linear_gemm": ([MP, P, I, I, P, I, P, SZ, P], I),
         "svq_get_device_status": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -196,6 +198,21 @@ def svq_linear_gemv_batched(Ws, xs, ys, ws=None, stream=None):
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().svq_linear_gemv_batched(arr, n, xp, M, yp, _dtype_code(ys[0].dtype), _ptr(ws), nb,
                                          _stream(stream)), "svq_linear_gemv_batched")
+
+
+def svq_linear_gemm_workspace_size(W: SvqWeight, M: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().svq_linear_gemm_workspace_size(ctypes.byref(W.desc), M, ctypes.byref(n)),
+           "svq_linear_gemm_workspace_size")
+    return int(n.value)
+
+
+def svq_linear_gemm(W: SvqWeight, x, y, ws, stream=None):
+    """y[M][N] = W x[M][K]^T on the tensor cores; x bf16 or fp16, y fp32 or bf16."""
+    M = x.shape[0]
+    nb = ws.numel() * ws.element_size()
+    _check(lib().svq_linear_gemm(ctypes.byref(W.desc), _ptr(x), _dtype_code(x.dtype), M, _ptr(y),
+                                 _dtype_code(y.dtype), _ptr(ws), nb, _stream(stream)), "svq_linear_gemm")
 
 
 def svq_get_device_status(stream=None) -> int:

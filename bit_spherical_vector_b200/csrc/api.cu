@@ -8,6 +8,7 @@
 
 #include "layout.cuh"
 #include "svq.h"
+#include "gemm_params.h"
 #include "svq_internal.h"
 
 namespace {
@@ -58,6 +59,18 @@ int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
   if (sms <= 0) return SVQ_ERR_CUDA;
   if (!svq::plan_gemv(descs, n_mats, M, sms, plan)) return SVQ_ERR_UNSUPPORTED_SHAPE;
   return SVQ_OK;
+}
+
+int* status_word() {
+  static int* ptr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptr[dev] = static_cast<int*>(p);
+  }
+  return ptr[dev];
 }
 
 }  // namespace
@@ -158,6 +171,38 @@ int svq_linear_gemv(const svq_matrix* W, const uint16_t* x, int M, void* y, int 
   const uint16_t* xx[1] = {x};
   if (!x || !y) return SVQ_ERR_INVALID_ARG;
   return svq_linear_gemv_batched(W, 1, xx, M, yy, y_dtype, workspace, workspace_bytes, stream);
+}
+
+int svq_linear_gemm_workspace_size(const svq_matrix* W, int M, size_t* bytes) {
+  if (!bytes) return SVQ_ERR_INVALID_ARG;
+  const int st = check_matrix(W);
+  if (st != SVQ_OK) return st;
+  if (M < 1) return SVQ_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return SVQ_ERR_CUDA;
+  *bytes = svq::plan_gemm(W->N, W->K, M, sms).ws_bytes;
+  return SVQ_OK;
+}
+
+int svq_linear_gemm(const svq_matrix* W, const uint16_t* x, int x_dtype, int M, void* y, int y_dtype,
+                    void* workspace, size_t workspace_bytes, svq_stream_t stream) {
+  const int st = check_matrix(W);
+  if (st != SVQ_OK) return st;
+  if (!x || !y || M < 1) return SVQ_ERR_INVALID_ARG;
+  if (x_dtype != SVQ_BF16 && x_dtype != SVQ_F16) return SVQ_ERR_INVALID_ARG;
+  if (y_dtype != SVQ_BF16 && y_dtype != SVQ_F32) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(y, 16)) return SVQ_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return SVQ_ERR_CUDA;
+  const svq::GemmPlan g = svq::plan_gemm(W->N, W->K, M, sms);
+  if (!workspace || workspace_bytes < g.ws_bytes || !aligned(workspace, 256)) return SVQ_ERR_WORKSPACE;
+  int* status = status_word();
+  if (!status) return SVQ_ERR_CUDA;
+  svq::GemmMatDesc d;
+  d.N = W->N; d.K = W->K; d.b_d = W->b_d; d.M = M;
+  d.packed = W->packed; d.codebook = W->codebook; d.scale = W->radius_scale; d.offset = W->radius_offset;
+  d.perm = W->perm; d.x = x; d.x_bf16 = x_dtype == SVQ_BF16; d.y = y; d.y_f32 = y_dtype == SVQ_F32;
+  return cuda_status(svq::launch_gemm(d, g, workspace, status, (cudaStream_t)stream));
 }
 
 int svq_get_device_status(svq_stream_t stream) {

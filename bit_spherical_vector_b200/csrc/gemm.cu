@@ -17,7 +17,8 @@
 //                   in TMEM (two buffers of BN columns)
 //       warps 2..5  decoders: packed codes -> 128 x 64 bf16/fp16 weight tile in
 //                   shared memory (K-major, 128-byte swizzle), codebook from
-//                   8 shared-memory replicas; each warp fills its own stages
+//                   8 shared-memory replicas; the four warps share every stage
+//                   (two of its eight subvector groups each)
 //       warps 6..9  epilogue: tcgen05.ld -> registers -> shared staging ->
 //                   coalesced stores of y (or split-K partials + fix-up)
 //   * weights are the A operand (swap-AB), so small token counts still map to
@@ -52,10 +53,6 @@ constexpr int kCbBytes = 32 * 1024;               // codebook replicas
 constexpr int kStageCols = 32;                    // epilogue columns per round
 constexpr int kStgBytes = kStageCols * 128 * 4;
 
-struct Smem {
-  // offsets (bytes from the 1024-aligned base)
-  uint32_t a, b, cb, stg, bars;
-};
 
 template <int BN, int NS>
 __host__ __device__ constexpr uint32_t smem_bytes() {
@@ -112,10 +109,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return r;
 }
 
-// Decode one 64-column stage of one 128-row tile into the swizzled A tile.
+// Decode decoder warp dw's share of one 64-column stage of one 128-row tile
+// into the swizzled A tile: subvector groups jj = 2*dw, 2*dw+1 of the stage,
+// all 128 rows (4 per lane).  The four decoder warps together fill the stage.
 template <bool BF16>
 __device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int kb, uint8_t* a_tile,
-                                             const uint8_t* cbs, int lane) {
+                                             const uint8_t* cbs, int lane, int dw) {
   const int L = tile_lanes(p.N, nt);
   if (lane >= L) return;
   const int b = kb >> 1, h = kb & 1;
@@ -141,6 +140,7 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int k
   }
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
+    if ((jj >> 1) != dw) continue;
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       if (hh != h) continue;
@@ -196,7 +196,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&bars->full_a[s], 1);
+      mbar_init(&bars->full_a[s], kNumDec);
       mbar_init(&bars->full_b[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
@@ -283,21 +283,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       mbar_wait(&bars->drain, 0);
     }
   } else if (warp < kEpiWarp0) {
-    // ---------------- decoders
+    // ---------------- decoders: all four warps fill every stage together, so each
+    // waits on every phase of every barrier in order (a warp that skipped
+    // phases could alias an mbarrier parity).
     const int d = warp - kDecWarp0;
     int it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-        if (it % kNumDec != d) continue;
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         int good = 1;
         if (it >= NS && lane == 0) good = wait_bar(&bars->empty[s], ph ^ 1, p, bars) ? 1 : 0;
         good = __shfl_sync(0xFFFFFFFFu, good, 0);
         if (!good) { ok = false; break; }
-        decode_stage<BF16>(p, w.nt, kb, a_st + s * kATileBytes, cbs, lane);
+        decode_stage<BF16>(p, w.nt, kb, a_st + s * kATileBytes, cbs, lane, d);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->full_a[s]);

@@ -40,10 +40,12 @@ namespace {
 constexpr size_t kSmemPerCtaTwo = 110 * 1024;   // two CTAs per SM
 constexpr size_t kSmemPerCtaOne = kGemvSmemMax;
 
+// codebook replicas + x slice + cross-warp reduction buffer
 size_t cta_smem(int b_d, int mt, int K, int S) {
   const int B = K / kBlockCols;
   const int nbmax = (B + S - 1) / S;
-  return ((size_t)16 << b_d) * 8 + (size_t)mt * nbmax * kBlockCols * 2;
+  return ((size_t)16 << b_d) * 8 + (size_t)mt * nbmax * kBlockCols * 2 +
+         (size_t)kGemvWarps * mt * kTileRows * sizeof(float);
 }
 
 }  // namespace
@@ -56,28 +58,44 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
   plan->mt = mt;
   const int per_sm = mt <= 2 ? 2 : 1;
   const size_t smem_cap = per_sm == 2 ? kSmemPerCtaTwo : kSmemPerCtaOne;
-  const double budget = (double)num_sms * per_sm;
-  double total = 0;
-  for (int i = 0; i < n_mats; ++i) total += (double)packed_bytes(mats[i].N, mats[i].K);
+  const int slots = num_sms * per_sm;
+  // One CTA per (128-row tile, k-slice).  Start with one slice per tile (at the
+  // smallest count shared memory allows), then repeatedly split the matrix whose
+  // CTAs carry the most blocks while the grid still fits in one wave.
+  int S[kGemvMaxMats], R[kGemvMaxMats], B[kGemvMaxMats];
+  int total = 0;
+  for (int i = 0; i < n_mats; ++i) {
+    R[i] = num_tiles(mats[i].N);
+    B[i] = mats[i].K / kBlockCols;
+    S[i] = 1;
+    while (S[i] < B[i] && cta_smem(mats[i].b_d, mt, mats[i].K, S[i]) > smem_cap) ++S[i];
+    if (cta_smem(mats[i].b_d, mt, mats[i].K, S[i]) > kSmemPerCtaOne) return false;
+    total += R[i] * S[i];
+  }
+  for (;;) {
+    int best = -1;
+    double worst = 0;
+    for (int i = 0; i < n_mats; ++i) {
+      const double per_cta = (double)B[i] / S[i];
+      if (S[i] < B[i] && per_cta > worst) { worst = per_cta; best = i; }
+    }
+    if (best < 0 || total + R[best] > slots) break;
+    ++S[best];
+    total += R[best];
+  }
   size_t off = 0;
   int ctas = 0;
   for (int i = 0; i < n_mats; ++i) {
     const GemvMatDesc& d = mats[i];
-    const int R = num_tiles(d.N), RC = (R + kGemvWarps - 1) / kGemvWarps, B = d.K / kBlockCols;
-    const double share = std::max(1.0, budget * (double)packed_bytes(d.N, d.K) / total);
-    int S = (int)std::lround(share / RC);
-    S = std::max(1, std::min(S, B));
-    while (S < B && cta_smem(d.b_d, mt, d.K, S) > smem_cap) ++S;
-    if (cta_smem(d.b_d, mt, d.K, S) > kSmemPerCtaOne) return false;
     GemvPlanMat& pm = plan->m[i];
-    pm.S = S;
-    pm.n_rc = RC;
-    pm.ctas = S * RC;
+    pm.S = S[i];
+    pm.n_rc = R[i];
+    pm.ctas = S[i] * R[i];
     pm.ws_offset = off;
     pm.ws_bytes = 0;
-    if (S > 1) {
-      const size_t part = ((size_t)S * mt * d.N * sizeof(float) + 255) / 256 * 256;
-      const size_t cnt = ((size_t)RC * sizeof(unsigned) + 255) / 256 * 256;
+    if (S[i] > 1) {
+      const size_t part = ((size_t)S[i] * mt * d.N * sizeof(float) + 255) / 256 * 256;
+      const size_t cnt = ((size_t)R[i] * sizeof(unsigned) + 255) / 256 * 256;
       pm.ws_bytes = part + cnt;
     }
     off += pm.ws_bytes;

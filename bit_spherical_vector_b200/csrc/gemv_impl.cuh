@@ -10,22 +10,23 @@
 // (Figures 1 and 5).
 //
 // B200 mapping:
-//   * a CTA of 8 warps works on one matrix, one k-slice and up to 8 row tiles;
-//     each warp owns a 128-row tile and each lane owns 4 complete rows, so a
-//     row's partial sum never leaves its thread (no shuffles in the hot loop);
+//   * a CTA of 8 warps works on one 128-row tile of one matrix and one k-slice;
+//     the warps split the slice's blocks, each lane owns 4 complete rows, so a
+//     row's partial sum never leaves its thread in the hot loop; the 8 warps'
+//     sums are combined once in shared memory;
 //   * packed codes stream from HBM with 16-byte coalesced loads
 //     (ld.global.nc.L1::no_allocate), one block (9 loads per lane) ahead;
 //   * the fp16 codebook sits in shared memory as 8 replicas, entry e of
 //     replica q at 16-byte slot 8e + q, and lane l reads replica l % 8: the 8
 //     lanes of each quarter-warp phase of an LDS.128 hit 8 different bank
 //     groups whatever the indices, so the random gather is conflict free;
-//   * x[perm] for the CTA's k-slice is gathered into shared memory once and
-//     read with broadcast loads;
+//   * each warp gathers its columns of x[perm] into shared memory (eight
+//     independent gathers in flight per lane) and reads them with broadcast loads;
 //   * signs are applied by XOR on fp16 sign bits; the eight products of a
 //     subvector are summed in fp16x2, then scaled by the radius and
 //     accumulated across subvectors in fp32;
-//   * split-K partials go to the workspace; the last CTA of a row chunk (found
-//     with a counter) sums them in a fixed order, so results are reproducible.
+//   * split-K partials go to the workspace; the last CTA of a tile (found with a
+//     counter) sums them in slice order, so results are reproducible.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -64,13 +65,11 @@ __device__ __forceinline__ void load_block(uint4 (&d)[kChunks], const uint8_t* b
   for (int c = 0; c < kChunks; ++c) d[c] = ldg_stream(blk + ((size_t)c * L + lane) * 16);
 }
 
-template <int BD, int MT>
+template <int MT>
 __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const unsigned char* xb,
-                                              int xstride_bytes, const unsigned char* cbq, const float (&scp)[4], const float (&ofp)[4],
-                                              float (&acc)[4][MT]) {
-  constexpr int BR = 10 - BD;
-  constexpr uint32_t IDX7 = ((1u << BD) - 1u) << 7;
-  constexpr uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
+                                              int xstride_bytes, const unsigned char* cbs, uint32_t q16,
+                                              uint32_t IDX7, uint32_t CODEM, const float2 (&scp)[2],
+                                              const float2 (&ofp)[2], float2 (&acc)[2][MT]) {
   uint32_t w[kWords];
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
@@ -82,6 +81,8 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
 #pragma unroll
     for (int m = 0; m < MT; ++m) xv[m] = lds128(xb, m * xstride_bytes + 16 * j);
     const uint32_t S = w[j];
+    float vf[4];
+    float dsum[4][MT];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int v = 4 * j + r;
@@ -101,140 +102,186 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
         ia = shl<7>(pw) & IDX7;
         vb = shl<13>(pw) & CODEM;
       }
-      uint4 cw = lds128(cbq, ia);
-      const float vf = __uint_as_float(vb | 0x3F800000u);     // 1 + code * 2^-BR
+      // replica offset q16 (bits 4..6) and the index (bits 7..) do not overlap: OR, not add
+      uint4 cw = lds128(cbs, ia | q16);
+      vf[r] = __uint_as_float(vb | 0x3F800000u);     // 1 + code * 2^-BR
       cw.x ^= (S << (4 * r + 0)) & 0x80008000u;
       cw.y ^= (S << (4 * r + 1)) & 0x80008000u;
       cw.z ^= (S << (4 * r + 2)) & 0x80008000u;
       cw.w ^= (S << (4 * r + 3)) & 0x80008000u;
-      const float rr = fmaf(scp[r], vf, ofp[r]);
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
         __half2 p = __hmul2(as_h2(cw.x), as_h2(xv[m].x));
         p = __hfma2(as_h2(cw.y), as_h2(xv[m].y), p);
         p = __hfma2(as_h2(cw.z), as_h2(xv[m].z), p);
         p = __hfma2(as_h2(cw.w), as_h2(xv[m].w), p);
-        const float dsum = __low2float(p) + __high2float(p);
-        acc[r][m] = fmaf(rr, dsum, acc[r][m]);
+        dsum[r][m] = __half2float(__hadd(__low2half(p), __high2half(p)));
       }
+    }
+    // radius r = scp * v + ofp and accumulation, two rows per packed fp32x2 FMA
+    const float2 r01 = __ffma2_rn(scp[0], make_float2(vf[0], vf[1]), ofp[0]);
+    const float2 r23 = __ffma2_rn(scp[1], make_float2(vf[2], vf[3]), ofp[1]);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      acc[0][m] = __ffma2_rn(r01, make_float2(dsum[0][m], dsum[1][m]), acc[0][m]);
+      acc[1][m] = __ffma2_rn(r23, make_float2(dsum[2][m], dsum[3][m]), acc[1][m]);
     }
   }
 }
 
-template <int BD, int MT>
+// One CTA = one 128-row tile of one matrix and one k-slice; its 8 warps split
+// the k-slice's blocks and their partial sums are combined in shared memory.
+template <int MT>
 __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char* smem, int y_f32) {
-  constexpr int BR = 10 - BD;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = g.N, K = g.K, B = K / kBlockCols;
-  const int s = c % g.S, rc = c / g.S;
-  const int b0 = (int)(((long long)B * s) / g.S), b1 = (int)(((long long)B * (s + 1)) / g.S);
-  const int nb = b1 - b0, ncols = nb * kBlockCols;
-  const int t = rc * kGemvWarps + warp;
-  const int L = (t < num_tiles(N)) ? tile_lanes(N, t) : 0;
+  const int BD = g.b_d, BR = 10 - BD;
+  const uint32_t IDX7 = ((1u << BD) - 1u) << 7;
+  const uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
+  const int N = g.N, K = g.K, B = K / kBlockCols, S = g.S, M = g.M;
+  const int t = c / S, s = c - t * S;
+  const int kb0 = (int)(((long long)B * s) / S), kb1 = (int)(((long long)B * (s + 1)) / S);
+  const int nbk = kb1 - kb0;
+  const int wb0 = kb0 + (nbk * warp) / kGemvWarps, wb1 = kb0 + (nbk * (warp + 1)) / kGemvWarps;
+  const int nb = wb1 - wb0;
+  const int L = tile_lanes(N, t);
   const bool on = lane < L;
   const int row0 = t * kTileRows + 4 * lane;
 
   uint4* cbs = reinterpret_cast<uint4*>(smem);
-  unsigned char* xs = smem + ((size_t)16 << BD) * 8;
+  unsigned char* xs = smem + ((size_t)16 << BD) * 8;                 // [MT][nbk*128] fp16
+  const int xstride = nbk * kBlockCols * 2;
+  float* red = reinterpret_cast<float*>(xs + (size_t)MT * xstride);  // [8 warps][MT][128]
 
-  const uint8_t* tile_base = g.packed + (on ? tile_offset(K, t) : 0);
+  const uint8_t* tile_base = g.packed + tile_offset(K, t);
   const size_t blk_bytes = (size_t)L * kLaneBlockBytes;
-
   uint4 d0[kChunks], d1[kChunks];
-  if (on && nb > 0) load_block(d0, tile_base + (size_t)b0 * blk_bytes, L, lane);
+  if (on && nb > 0) load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane);
 
-  // Codebook replicas: entry e, replica q -> 16-byte slot 8e + q.
-  for (int i = threadIdx.x; i < (8 << BD); i += blockDim.x) cbs[i] = __ldg(g.codebook + (i >> 3));
-  // x[perm] for this k-slice, token-major, zero for tokens >= M.
-  const __half* xh = reinterpret_cast<const __half*>(g.x);
-  __half* xsh = reinterpret_cast<__half*>(xs);
-  for (int i = threadIdx.x; i < MT * ncols; i += blockDim.x) {
-    const int m = i / ncols, j = i - m * ncols;
-    __half v = __ushort_as_half(0);
-    if (m < g.M) v = xh[(size_t)m * K + __ldg(g.perm + (size_t)b0 * kBlockCols + j)];
-    xsh[i] = v;
+  // Codebook replicas: entry e, replica q -> 16-byte slot 8e + q (one load per entry).
+  for (int e = threadIdx.x; e < (1 << BD); e += blockDim.x) {
+    const uint4 v = __ldg(g.codebook + e);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cbs[8 * e + q] = v;
+  }
+  // This warp's columns of x[perm] (8 independent gathers in flight per lane).
+  {
+    const __half* xh = reinterpret_cast<const __half*>(g.x);
+    __half* xsh = reinterpret_cast<__half*>(xs);
+    const int jc0 = (wb0 - kb0) * kBlockCols, ncw = nb * kBlockCols;
+    const int32_t* pp = g.perm + (size_t)kb0 * kBlockCols + jc0;
+    for (int j0 = lane; j0 < ncw; j0 += 32 * 8) {
+      int pj[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pj[u] = (j0 + 32 * u < ncw) ? __ldg(pp + j0 + 32 * u) : 0;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        __half hv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) hv[u] = (m < M) ? xh[(size_t)m * K + pj[u]] : __ushort_as_half(0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (j0 + 32 * u < ncw) xsh[(size_t)m * (xstride / 2) + jc0 + j0 + 32 * u] = hv[u];
+      }
+    }
   }
   // Radius r = offset + scale * code, written as r = scp * v + ofp with v = 1 + code * 2^-BR.
-  float scp[4], ofp[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    float sc = 0.f, of = 0.f;
+  float2 scp[2], ofp[2];
+  {
+    float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
     if (on) {
-      sc = __half2float(__ushort_as_half(g.scale[row0 + r]));
-      of = __half2float(__ushort_as_half(g.offset[row0 + r]));
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        sc[r] = __half2float(__ushort_as_half(g.scale[row0 + r]));
+        of[r] = __half2float(__ushort_as_half(g.offset[row0 + r]));
+      }
     }
-    if (BR > 0) { scp[r] = sc * (float)(1 << BR); ofp[r] = of - scp[r]; }
-    else { scp[r] = 0.f; ofp[r] = of; }
+    float sp[4], op[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (BR > 0) { sp[r] = sc[r] * (float)(1 << BR); op[r] = of[r] - sp[r]; }
+      else { sp[r] = 0.f; op[r] = of[r]; }
+    }
+    scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
+    ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
   }
   __syncthreads();
 
-  float acc[4][MT];
+  float2 acc[2][MT];
 #pragma unroll
-  for (int r = 0; r < 4; ++r)
+  for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
+    for (int m = 0; m < MT; ++m) acc[h][m] = make_float2(0.f, 0.f);
 
-  const unsigned char* cbq = reinterpret_cast<const unsigned char*>(cbs) + (lane & 7) * 16;
-  const unsigned char* xbase = xs;
-  const int xstride = ncols * 2;
+  const unsigned char* cbb = reinterpret_cast<const unsigned char*>(cbs);
+  const uint32_t q16 = (uint32_t)(lane & 7) * 16;
+  const unsigned char* xw = xs + (size_t)(wb0 - kb0) * kBlockCols * 2;
   if (on) {
-    int b = 0;
-    for (; b + 1 < nb; b += 2) {
-      load_block(d1, tile_base + (size_t)(b0 + b + 1) * blk_bytes, L, lane);
-      process_block<BD, MT>(d0, xbase + b * kBlockCols * 2, xstride, cbq, scp, ofp, acc);
-      if (b + 2 < nb) load_block(d0, tile_base + (size_t)(b0 + b + 2) * blk_bytes, L, lane);
-      process_block<BD, MT>(d1, xbase + (b + 1) * kBlockCols * 2, xstride, cbq, scp, ofp, acc);
+    for (int b = 0; b < nb; ++b) {
+      if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane);
+      process_block<MT>(d0, xw + b * kBlockCols * 2, xstride, cbb, q16, IDX7, CODEM, scp, ofp, acc);
+#pragma unroll
+      for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     }
-    if (b < nb) process_block<BD, MT>(d0, xbase + b * kBlockCols * 2, xstride, cbq, scp, ofp, acc);
   }
 
-  const int M = g.M;
-  if (g.S == 1) {
-    if (on) {
+  // Combine the 8 warps' partial sums of the tile's 128 rows (fixed order).
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (m >= M) break;
+  for (int m = 0; m < MT; ++m) {
+    float* rr = red + ((size_t)warp * MT + m) * kTileRows + 4 * lane;
+    *reinterpret_cast<float4*>(rr) = make_float4(acc[0][m].x, acc[0][m].y, acc[1][m].x, acc[1][m].y);
+  }
+  __syncthreads();
+  const int rows = L * 4;
+  const int nout = rows * M;
+  if (S == 1) {
+    for (int i = threadIdx.x; i < nout; i += blockDim.x) {
+      const int om = i / rows, on_i = i - om * rows;
+      float outv = 0.f;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const size_t o = (size_t)m * N + row0 + r;
-          if (y_f32) reinterpret_cast<float*>(g.y)[o] = acc[r][m];
-          else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(acc[r][m]);
-        }
-      }
+      for (int w8 = 0; w8 < kGemvWarps; ++w8) outv += red[((size_t)w8 * MT + om) * kTileRows + on_i];
+      const size_t o = (size_t)om * N + t * kTileRows + on_i;
+      if (y_f32) reinterpret_cast<float*>(g.y)[o] = outv;
+      else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(outv);
     }
     return;
   }
 
-  // Split-K: write partials, then the last CTA of this row chunk reduces them.
-  if (on) {
+  // Split-K: write this k-slice's partial, then the last CTA of the tile sums the
+  // S partials in slice order.
+  for (int i = threadIdx.x; i < nout; i += blockDim.x) {
+    const int om = i / rows, on_i = i - om * rows;
+    float outv = 0.f;
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      if (m >= M) break;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) g.partial[((size_t)s * M + m) * N + row0 + r] = acc[r][m];
-    }
+    for (int w8 = 0; w8 < kGemvWarps; ++w8) outv += red[((size_t)w8 * MT + om) * kTileRows + on_i];
+    g.partial[((size_t)s * M + om) * N + t * kTileRows + on_i] = outv;
   }
   __threadfence();
   __syncthreads();
   __shared__ int s_last;
   if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(&g.counters[rc], 1u);
-    s_last = (prev == (unsigned)(g.S - 1));
+    const unsigned prev = atomicAdd(&g.counters[t], 1u);
+    s_last = (prev == (unsigned)(S - 1));
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const int rbeg = rc * kGemvWarps * kTileRows;
-  const int rows = min(N - rbeg, kGemvWarps * kTileRows);
-  for (int i = threadIdx.x; i < rows * M; i += blockDim.x) {
-    const int m = i / rows, n = rbeg + (i - m * rows);
+  for (int i = threadIdx.x; i < nout; i += blockDim.x) {
+    const int om = i / rows, n = t * kTileRows + (i - om * rows);
     float sum = 0.f;
-    for (int k = 0; k < g.S; ++k) sum += __ldcg(g.partial + ((size_t)k * M + m) * N + n);
-    const size_t o = (size_t)m * N + n;
+    int k = 0;
+    for (; k + 8 <= S; k += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(g.partial + ((size_t)(k + u) * M + om) * N + n);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[u];
+    }
+    for (; k < S; ++k) sum += __ldcg(g.partial + ((size_t)k * M + om) * N + n);
+    const size_t o = (size_t)om * N + n;
     if (y_f32) reinterpret_cast<float*>(g.y)[o] = sum;
     else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(sum);
   }
-  if (threadIdx.x == 0) g.counters[rc] = 0u;
+  if (threadIdx.x == 0) g.counters[t] = 0u;
 }
 
 template <int MT>
@@ -245,18 +292,7 @@ gemv_kernel(const __grid_constant__ GemvKParams P) {
   while (mi + 1 < P.n_mats && (int)blockIdx.x >= P.mats[mi + 1].cta_begin) ++mi;
   const GemvKMat& g = P.mats[mi];
   const int c = (int)blockIdx.x - g.cta_begin;
-  switch (g.b_d) {
-    case 1: gemv_cta<1, MT>(g, c, smem, P.y_f32); break;
-    case 2: gemv_cta<2, MT>(g, c, smem, P.y_f32); break;
-    case 3: gemv_cta<3, MT>(g, c, smem, P.y_f32); break;
-    case 4: gemv_cta<4, MT>(g, c, smem, P.y_f32); break;
-    case 5: gemv_cta<5, MT>(g, c, smem, P.y_f32); break;
-    case 6: gemv_cta<6, MT>(g, c, smem, P.y_f32); break;
-    case 7: gemv_cta<7, MT>(g, c, smem, P.y_f32); break;
-    case 8: gemv_cta<8, MT>(g, c, smem, P.y_f32); break;
-    case 9: gemv_cta<9, MT>(g, c, smem, P.y_f32); break;
-    default: gemv_cta<10, MT>(g, c, smem, P.y_f32); break;
-  }
+  gemv_cta<MT>(g, c, smem, P.y_f32);
 }
 
 }  // namespace

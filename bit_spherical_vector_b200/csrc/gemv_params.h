@@ -19,7 +19,7 @@ struct GemvKMat {
   const uint16_t* x;      // fp16 [M][K]
   void* y;                // [M][N]
   float* partial;         // [S][M][N]
-  unsigned* counters;     // [n_rc]
+  unsigned* counters;     // [n_rc] (one per 128-row tile)
   int N, K, b_d, S, n_rc, cta_begin, M;
 };
 

@@ -9,9 +9,11 @@
 namespace svq {
 namespace sm100 {
 
-// Upper bound on mbarrier polls before a wait gives up (well above any
-// legitimate wait: each poll suspends for up to ~0.5 us).
-constexpr uint32_t kWaitPolls = 1u << 22;
+// Upper bound on mbarrier polls before a wait gives up.  Each poll suspends
+// for at most kPollSuspendNs, so a wait ends within about 2 s -- far above any
+// legitimate wait in these kernels (microseconds), far below a hung GPU.
+constexpr uint32_t kWaitPolls = 1u << 21;
+constexpr uint32_t kPollSuspendNs = 1000;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -44,7 +46,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kPollSuspendNs)
       : "memory");
   return ok != 0;
 }

@@ -155,6 +155,25 @@ SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const ui
                             size_t workspace_bytes, svq_stream_t stream);
 
 /*
+ * svq_linear_gemm -- prefill / batched layer on the tensor cores (tcgen05):
+ *   y[m][n] = sum_j W[n][j] * x[m][perm[j]],  any M >= 1.
+ * The pages' prefill kernel is a 64-row GEMM loop that accumulates mma products
+ * (Figure 6(b) caption); here weight tiles are decoded from the codes into
+ * shared memory as bf16 (x_dtype SVQ_BF16) or fp16 (x_dtype SVQ_F16) -- the
+ * weights are the same rounded values svq_dequantize exports -- and multiplied
+ * with fp32 accumulation in tensor memory.  x: [M][K] of x_dtype (natural input
+ * order).  y: [M][N] of y_dtype SVQ_F32 or SVQ_BF16.
+ * Workspace (svq_linear_gemm_workspace_size): the permuted activations
+ * x[:, perm] plus split-K partials and counters; as for the GEMV the counter
+ * region must be zero before the first use (svq_workspace_init) and is left
+ * zero by every completed call.  Error bound used by the tests:
+ * |y - y_ref| <= 1e-2 * sum_j |W[n][j]||x[m][perm[j]]|.
+ */
+SVQ_API int svq_linear_gemm_workspace_size(const svq_matrix* W /* host */, int M, size_t* bytes);
+SVQ_API int svq_linear_gemm(const svq_matrix* W /* host */, const uint16_t* x, int x_dtype, int M, void* y,
+                            int y_dtype, void* workspace, size_t workspace_bytes, svq_stream_t stream);
+
+/*
  * Synchronising read-and-clear of the device status word that kernels set
  * when a bounded wait runs out (SVQ_OK or SVQ_ERR_TIMEOUT).  Tests only.
  */
