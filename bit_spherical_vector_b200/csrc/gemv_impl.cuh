@@ -157,44 +157,57 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   uint4 d0[kChunks], d1[kChunks];
   if (on && nb > 0) load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane);
 
-  // Codebook replicas: entry e, replica q -> 16-byte slot 8e + q (one load per entry).
-  for (int e = threadIdx.x; e < (1 << BD); e += blockDim.x) {
-    const uint4 v = __ldg(g.codebook + e);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) cbs[8 * e + q] = v;
+  // Codebook replicas: entry e, replica q -> 16-byte slot 8e + q.  Thread i fills
+  // slot i with an asynchronous global->shared copy (consecutive slots per warp:
+  // no bank conflicts; the eight copies of one entry share a load request).
+  {
+    const uint32_t cb_s = (uint32_t)__cvta_generic_to_shared(cbs);
+    for (int i = threadIdx.x; i < (8 << BD); i += blockDim.x)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(cb_s + 16u * i), "l"(g.codebook + (i >> 3))
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
-  // This warp's columns of x[perm] (8 independent gathers in flight per lane).
+  // Radius parameters of this lane's rows (weights: independent of earlier kernels).
+  float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
+  if (on) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      sc[r] = __half2float(__ushort_as_half(g.scale[row0 + r]));
+      of[r] = __half2float(__ushort_as_half(g.offset[row0 + r]));
+    }
+  }
+  // Everything above reads weights only; x may be written by the previous kernel
+  // in the stream (programmatic dependent launch): wait for it here.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // This warp's columns of x[perm]: up to 16 gathers per lane in flight at once
+  // (all perm loads, then all x loads), i.e. two dependent round trips.
   {
     const __half* xh = reinterpret_cast<const __half*>(g.x);
     __half* xsh = reinterpret_cast<__half*>(xs);
     const int jc0 = (wb0 - kb0) * kBlockCols, ncw = nb * kBlockCols;
     const int32_t* pp = g.perm + (size_t)kb0 * kBlockCols + jc0;
-    for (int j0 = lane; j0 < ncw; j0 += 32 * 8) {
-      int pj[8];
+    constexpr int U = MT == 1 ? 16 : 8;
+    for (int j0 = lane; j0 < ncw; j0 += 32 * U) {
+      int pj[U];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) pj[u] = (j0 + 32 * u < ncw) ? __ldg(pp + j0 + 32 * u) : 0;
+      for (int u = 0; u < U; ++u) pj[u] = (j0 + 32 * u < ncw) ? __ldg(pp + j0 + 32 * u) : 0;
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        __half hv[8];
+        __half hv[U];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) hv[u] = (m < M) ? xh[(size_t)m * K + pj[u]] : __ushort_as_half(0);
+        for (int u = 0; u < U; ++u) hv[u] = (m < M) ? xh[(size_t)m * K + pj[u]] : __ushort_as_half(0);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < U; ++u)
           if (j0 + 32 * u < ncw) xsh[(size_t)m * (xstride / 2) + jc0 + j0 + 32 * u] = hv[u];
       }
     }
   }
+  // Let the next kernel in the stream start its own weight-only prologue as this
+  // grid's CTAs retire.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Radius r = offset + scale * code, written as r = scp * v + ofp with v = 1 + code * 2^-BR.
   float2 scp[2], ofp[2];
   {
-    float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
-    if (on) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        sc[r] = __half2float(__ushort_as_half(g.scale[row0 + r]));
-        of[r] = __half2float(__ushort_as_half(g.offset[row0 + r]));
-      }
-    }
     float sp[4], op[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -204,6 +217,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
     scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
     ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
   float2 acc[2][MT];
@@ -309,7 +323,21 @@ cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStre
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
   }
-  gemv_kernel<MT><<<grid, kGemvWarps * 32, smem, st>>>(p);
+  // Programmatic dependent launch: the kernel's weight-only prologue may overlap
+  // the tail of the previous kernel in the stream (it waits for that kernel
+  // before reading x).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kGemvWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
