@@ -66,6 +66,7 @@ def lib():
         "svq_linear_gemv": ([MP, P, I, P, I, P, SZ, P], I),
         "svq_linear_gemv_batched_workspace_size": ([MP, I, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemv_batched": ([MP, I, ctypes.POINTER(P), I, ctypes.POINTER(P), I, P, SZ, P], I),
+        "svq_linear_gemv_noalloc": ([MP, P, I, P, I, P], I),
         "svq_linear_gemm_workspace_size": ([MP, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemm": ([MP, P, I, I, P, I, P, SZ, P], I),
         "svq_get_device_status": ([P], I),
@@ -198,6 +199,13 @@ def svq_linear_gemv_batched(Ws, xs, ys, ws=None, stream=None):
     nb = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib().svq_linear_gemv_batched(arr, n, xp, M, yp, _dtype_code(ys[0].dtype), _ptr(ws), nb,
                                          _stream(stream)), "svq_linear_gemv_batched")
+
+
+def svq_linear_gemv_noalloc(W: SvqWeight, x, y, stream=None):
+    """svq_linear_gemv with the library's fixed internal scratch (no workspace argument)."""
+    M = x.shape[0]
+    _check(lib().svq_linear_gemv_noalloc(ctypes.byref(W.desc), _ptr(x), M, _ptr(y), _dtype_code(y.dtype),
+                                         _stream(stream)), "svq_linear_gemv_noalloc")
 
 
 def svq_linear_gemm_workspace_size(W: SvqWeight, M: int) -> int:

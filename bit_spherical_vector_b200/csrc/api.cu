@@ -61,6 +61,30 @@ int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
   return SVQ_OK;
 }
 
+// Scratch for svq_linear_gemv_noalloc: split-K partial sums and completion
+// counters of one call.  Every GPU that loads the library holds these bytes
+// until the process exits.
+constexpr size_t kNoAllocScratchBytes = 4u << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch for the current device, looked up (and
+// the scratch zero-filled on `stream`) on the first call per device.  In host
+// code the array's name is only a host-side stand-in; kernels must be given the
+// address returned by cudaGetSymbolAddress.
+void* noalloc_scratch(cudaStream_t stream) {
+  static void* ptr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
+    // Completion counters must start at zero; every completed call leaves them zero.
+    if (cudaMemsetAsync(p, 0, kNoAllocScratchBytes, stream) != cudaSuccess) return nullptr;
+    ptr[dev] = p;
+  }
+  return ptr[dev];
+}
+
 int* status_word() {
   static int* ptr[64] = {nullptr};
   int dev = 0;
@@ -171,6 +195,23 @@ int svq_linear_gemv(const svq_matrix* W, const uint16_t* x, int M, void* y, int 
   const uint16_t* xx[1] = {x};
   if (!x || !y) return SVQ_ERR_INVALID_ARG;
   return svq_linear_gemv_batched(W, 1, xx, M, yy, y_dtype, workspace, workspace_bytes, stream);
+}
+
+int svq_linear_gemv_noalloc(const svq_matrix* W, const uint16_t* x, int M, void* y, int y_dtype,
+                            svq_stream_t stream) {
+  if (!x || !y) return SVQ_ERR_INVALID_ARG;
+  if (y_dtype != SVQ_F16 && y_dtype != SVQ_F32) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(x, 2) || !aligned(y, y_dtype == SVQ_F32 ? 4 : 2)) return SVQ_ERR_INVALID_ARG;
+  svq::GemvPlan plan;
+  svq::GemvMatDesc descs[1];
+  const uint16_t* xx[1] = {x};
+  void* yy[1] = {y};
+  const int st = plan_group(W, 1, M, &plan, descs, xx, yy);
+  if (st != SVQ_OK) return st;
+  if (plan.ws_total > kNoAllocScratchBytes) return SVQ_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch((cudaStream_t)stream);
+  if (!scratch) return SVQ_ERR_CUDA;
+  return cuda_status(svq::launch_gemv(descs, plan, y_dtype == SVQ_F32, scratch, (cudaStream_t)stream));
 }
 
 int svq_linear_gemm_workspace_size(const svq_matrix* W, int M, size_t* bytes) {

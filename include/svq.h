@@ -155,6 +155,30 @@ SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const ui
                             size_t workspace_bytes, svq_stream_t stream);
 
 /*
+ * svq_linear_gemv_noalloc -- svq_linear_gemv for callers that cannot allocate
+ * device memory.  The paper has no counterpart; this is a deployment aid.  Some
+ * callers have no allocator to get a workspace from: a plugin that is handed
+ * only a stream, code that runs after its host has frozen its memory pools, or
+ * a real-time loop where a cudaMalloc could stall.  This entry point takes the
+ * same inputs and outputs as svq_linear_gemv (x fp16 [M][K], y [M][N] of
+ * SVQ_F16 or SVQ_F32, M 1..16) but keeps its split-K scratch in a fixed 4 MiB
+ * array inside the library, which every GPU that loads the library holds
+ * until the process exits.  It allocates nothing and calls no allocating
+ * routine.
+ *   - A call whose scratch need (svq_linear_gemv_workspace_size) exceeds
+ *     4 MiB returns SVQ_ERR_WORKSPACE and enqueues nothing.
+ *   - The first call on a device looks up the array's device address and
+ *     zero-fills it on `stream`; make that first call before any stream
+ *     capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other threads) race and give wrong results; serialise them.
+ *   - The array keeps the last call's contents; the counters that must start
+ *     at zero are zeroed at set-up and left zero by every completed call.
+ */
+SVQ_API int svq_linear_gemv_noalloc(const svq_matrix* W /* host */, const uint16_t* x, int M, void* y,
+                                    int y_dtype, svq_stream_t stream);
+
+/*
  * svq_linear_gemm -- prefill / batched layer on the tensor cores (tcgen05):
  *   y[m][n] = sum_j W[n][j] * x[m][perm[j]],  any M >= 1.
  * The pages' prefill kernel is a 64-row GEMM loop that accumulates mma products

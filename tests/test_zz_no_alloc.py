@@ -1,0 +1,60 @@
+"""svq_linear_gemv_noalloc: the GEMV entry point for callers that cannot
+allocate device memory (its split-K scratch is a fixed array inside the
+library instead of a caller workspace).  Checked through the C ABI against
+svq_linear_gemv on two calls in a row, so that scratch contents left by the
+first call cannot spoil the second.  This file is collected last; its tests
+pass alone in a fresh process and after the rest of the suite."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import synth
+from tests.gpu_util import need_gpu, torch, x_f16
+
+import bit_spherical_vector_b200 as svq
+
+pytestmark = pytest.mark.gpu
+TOL = 1e-3
+LIMIT = 4 << 20
+
+
+def _noalloc(desc, x_ptr, M, y_ptr):
+    return svq.lib().svq_linear_gemv_noalloc(ctypes.byref(desc), ctypes.c_void_p(x_ptr), M,
+                                             ctypes.c_void_p(y_ptr), svq.SVQ_F32,
+                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("N,K,M,b_d", [(2560, 9728, 1, 8), (1024, 2560, 3, 7), (9728, 2560, 2, 6)])
+def test_noalloc_matches_workspace_entry_two_calls(N, K, M, b_d):
+    need_gpu()
+    m = synth.make_matrix(99, N + M, N, K, b_d)
+    W = svq.SvqWeight.from_synth(m)
+    nb = svq.svq_linear_gemv_workspace_size(W, M)
+    assert 0 < nb <= LIMIT                     # split-K scratch is used, and fits the fixed array
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    svq.svq_workspace_init(ws)
+    wq = torch.empty((N, K), dtype=torch.float16, device="cuda")
+    svq.svq_dequantize(W, wq)
+    perm = torch.from_numpy(m.perm.astype(np.int64)).cuda()
+    for call in range(2):
+        x = x_f16(synth.make_x(99, 10 * call + M, M, K))
+        ref = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        svq.svq_linear_gemv(W, x, ref, ws)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        assert _noalloc(W.desc, x.data_ptr(), M, y.data_ptr()) == svq.SVQ_OK
+        torch.cuda.synchronize()
+        den = x[:, perm].float().abs() @ wq.float().abs().t()     # sum_j |W[n][j]| |x[m][perm[j]]|
+        assert bool(((y - ref).abs() <= TOL * den).all())
+        assert torch.equal(y, ref)             # same kernel and plan: in fact identical
+
+
+def test_noalloc_rejects_scratch_beyond_limit():
+    """A shape whose split-K scratch exceeds the fixed 4 MiB is refused before anything is
+    enqueued (the pointers below are never dereferenced)."""
+    need_gpu()
+    desc = svq.svq_matrix(16384, 81920, 8, 0, 0x10000, 0x20000, 0x30000, 0x40000, 0x50000)
+    n = ctypes.c_size_t(0)
+    assert svq.lib().svq_linear_gemv_workspace_size(ctypes.byref(desc), 8, ctypes.byref(n)) == svq.SVQ_OK
+    assert n.value > LIMIT
+    assert _noalloc(desc, 0x60000, 8, 0x70000) == svq.SVQ_ERR_WORKSPACE
