@@ -337,6 +337,148 @@ def run_gpu(args, world, rank, local):
     return 0
 
 
+# --------------------------------------------------------------------------- secondary workloads
+def _time_graph(fn, reps, stream):
+    """Capture fn() once in a CUDA graph, replay `reps` times; return microseconds per replay."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def run_sweep(args):
+    """8192 x 8192 (7,3) matrix, M = 1..16 tokens: GEMV and tensor-core GEMM, 20 rotated copies (378 MB)."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    stream = torch.cuda.Stream()
+    copies = 20
+    base = synth.square_8192()
+    Ws = []
+    for c in range(copies):
+        m = synth.make_matrix(2, 100 + c, 8192, 8192, 7) if c else base
+        Ws.append(svq.SvqWeight.from_synth(m))
+    torch.cuda.synchronize()
+    packed = 8192 * 8192 * 9 // 32
+    for M in (1, 2, 4, 8, 16):
+        x = torch.from_numpy(synth.square_8192_x(M).view(np.int16)).cuda().view(torch.float16)
+        y = torch.empty((M, 8192), dtype=torch.float32, device="cuda")
+        nbv = svq.svq_linear_gemv_workspace_size(Ws[0], M)
+        wsv = torch.empty(max(nbv, 256), dtype=torch.uint8, device="cuda")
+        nbg = svq.svq_linear_gemm_workspace_size(Ws[0], M)
+        wsg = torch.empty(max(nbg, 256), dtype=torch.uint8, device="cuda")
+        with torch.cuda.stream(stream):
+            svq.svq_workspace_init(wsv)
+            svq.svq_workspace_init(wsg)
+
+        def gemv():
+            for W in Ws:
+                svq.svq_linear_gemv(W, x, y, wsv)
+
+        def gemm():
+            for W in Ws:
+                svq.svq_linear_gemm(W, x, y, wsg)
+        tv = _time_graph(gemv, 20, stream) / copies
+        tg = _time_graph(gemm, 20, stream) / copies
+        print(json.dumps({"workload": "sweep 8192x8192 (7,3)", "M": M, "gemv_us": round(tv, 3),
+                          "gemv_GBps": round(packed / tv / 1e3, 1), "gemm_us": round(tg, 3),
+                          "gemm_GBps": round(packed / tg / 1e3, 1), "faster": "gemv" if tv <= tg else "gemm",
+                          "tokens_per_s_best": round(M / min(tv, tg) * 1e6, 1)}), flush=True)
+
+
+def run_prefill(args):
+    """Qwen3-4B gate/up (2560->9728) and down (9728->2560), (8,2), M = 512 and 2048, bf16."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    stream = torch.cuda.Stream()
+    peak, kind = read_peaks()
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tpeak = float(json.load(f)["bf16_tflops"])
+    except Exception:
+        tpeak = 1590.0
+    for which, m in enumerate(synth.prefill_mats()):
+        W = svq.SvqWeight.from_synth(m)
+        wq = torch.empty((m.N, m.K), dtype=torch.bfloat16, device="cuda")
+        svq.svq_dequantize(W, wq)
+        for M in (512, 2048):
+            x = torch.from_numpy(synth.prefill_x(M, m.K, which).view(np.int16)).cuda().view(torch.bfloat16)
+            y = torch.empty((M, m.N), dtype=torch.float32, device="cuda")
+            nb = svq.svq_linear_gemm_workspace_size(W, M)
+            ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+            with torch.cuda.stream(stream):
+                svq.svq_workspace_init(ws)
+            t = _time_graph(lambda: svq.svq_linear_gemm(W, x, y, ws), 20, stream)
+            xp = x[:, torch.from_numpy(m.perm.astype(np.int64)).cuda()].contiguous()
+            yc = torch.empty((M, m.N), dtype=torch.bfloat16, device="cuda")
+            tc = _time_graph(lambda: torch.matmul(xp, wq.t(), out=yc), 20, stream)
+            flop = 2.0 * M * m.N * m.K
+            print(json.dumps({"workload": f"prefill {m.K}->{m.N} (8,2) bf16", "M": M, "svq_gemm_us": round(t, 2),
+                              "svq_TFLOPs": round(flop / t / 1e6, 1),
+                              "svq_frac_of_bf16_peak": round(flop / t / 1e6 / tpeak, 3),
+                              "cublas_dense_bf16_us": round(tc, 2), "cublas_TFLOPs": round(flop / tc / 1e6, 1),
+                              "peak_bf16_TFLOPs": tpeak, "note": "svq time includes the x[:,perm] pass"}),
+                  flush=True)
+
+
+def run_moe(args):
+    """Qwen3-30B-A3B-shaped MoE FFN (hidden 2048, 128 experts, inter 768, top-8), T = 1 and 16."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    stream = torch.cuda.Stream()
+    experts = synth.moe_experts()
+    gu, down = [], []
+    for g, u, d in experts:
+        gu += [svq.SvqWeight.from_synth(g), svq.SvqWeight.from_synth(u)]
+        down.append(svq.SvqWeight.from_synth(d))
+    gu_tab, dn_tab = svq.descriptor_table(gu), svq.descriptor_table(down)
+    per_mat = 768 * 2048 * 9 // 32
+    for T in (1, 16):
+        ids, w = synth.moe_routing(T)
+        k = ids.shape[1]
+        e = torch.from_numpy(ids.astype(np.int64)).cuda().reshape(-1)
+        tok = torch.arange(T, device="cuda").repeat_interleave(k)
+        pair = torch.arange(T * k, device="cuda")
+        items1 = svq.item_table(torch.stack([2 * e, 2 * e + 1], 1).reshape(-1), tok.repeat_interleave(2),
+                                torch.stack([2 * pair, 2 * pair + 1], 1).reshape(-1), torch.ones(2 * T * k, device="cuda"))
+        items2 = svq.item_table(e, pair, tok, torch.from_numpy(w.reshape(-1)).cuda())
+        x = torch.from_numpy(synth.moe_x(T).view(np.int16)).cuda().view(torch.float16)
+        y1 = torch.empty((2 * T * k, 768), dtype=torch.float32, device="cuda")
+        out = torch.empty((T, 2048), dtype=torch.float32, device="cuda")
+        ws1 = torch.empty(svq.svq_moe_grouped_gemv_workspace_size(len(gu), 2 * T * k, 768, False), dtype=torch.uint8,
+                          device="cuda")
+        ws2 = torch.empty(svq.svq_moe_grouped_gemv_workspace_size(len(down), T * k, 2048, True), dtype=torch.uint8,
+                          device="cuda")
+
+        def ffn():
+            svq.svq_moe_grouped_gemv(gu_tab, len(gu), 768, 2048, 8, items1, 2 * T * k, T, x, svq.SVQ_X_F16, y1,
+                                     2 * T * k, False, ws1)
+            svq.svq_moe_grouped_gemv(dn_tab, len(down), 2048, 768, 8, items2, T * k, T, y1.view(T * k, 1536),
+                                     svq.SVQ_X_SWIGLU_F32, out, T, True, ws2)
+        t = _time_graph(ffn, 50, stream)
+        touched = len(set(ids.reshape(-1).tolist()))
+        nbytes = touched * 3 * per_mat
+        print(json.dumps({"workload": "moe ffn qwen3-30b-a3b shapes", "T": T, "us": round(t, 2),
+                          "tokens_per_s": round(T / t * 1e6, 1), "experts_touched": touched,
+                          "GBps_distinct_packed": round(nbytes / t / 1e3, 1),
+                          "note": "L2-warm: the same routed experts every replay"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -344,7 +486,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=1400)
     ap.add_argument("--impl", default="svq", choices=["svq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="layer", choices=["layer", "sweep", "prefill", "moe"],
+                    help="layer = the headline line; the others print one JSON line per configuration")
     args = ap.parse_args()
+    if args.workload != "layer":
+        return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe}[args.workload](args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_init() if args.impl == "svq" else (int(os.environ.get("WORLD_SIZE", "1")),

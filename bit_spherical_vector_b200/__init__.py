@@ -69,6 +69,8 @@ def lib():
         "svq_linear_gemv_noalloc": ([MP, P, I, P, I, P], I),
         "svq_linear_gemm_workspace_size": ([MP, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemm": ([MP, P, I, I, P, I, P, SZ, P], I),
+        "svq_moe_grouped_gemv_workspace_size": ([I, I, I, I, ctypes.POINTER(SZ)], I),
+        "svq_moe_grouped_gemv": ([P, I, I, I, I, P, I, I, P, I, P, I, I, P, SZ, P], I),
         "svq_get_device_status": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -221,6 +223,46 @@ def svq_linear_gemm(W: SvqWeight, x, y, ws, stream=None):
     nb = ws.numel() * ws.element_size()
     _check(lib().svq_linear_gemm(ctypes.byref(W.desc), _ptr(x), _dtype_code(x.dtype), M, _ptr(y),
                                  _dtype_code(y.dtype), _ptr(ws), nb, _stream(stream)), "svq_linear_gemm")
+
+
+class svq_group_item(ctypes.Structure):
+    _fields_ = [("matrix", ctypes.c_int32), ("x_row", ctypes.c_int32), ("out_row", ctypes.c_int32),
+                ("out_scale", ctypes.c_float)]
+
+
+SVQ_X_F16, SVQ_X_SWIGLU_F32 = 0, 1
+
+
+def descriptor_table(Ws, device="cuda"):
+    """Device array of svq_matrix descriptors (the layout the MoE kernel reads)."""
+    import numpy as np
+    import torch
+    arr = (svq_matrix * len(Ws))(*[w.desc for w in Ws])
+    raw = np.frombuffer(bytes(arr), dtype=np.uint8).copy()
+    return torch.from_numpy(raw).to(device)
+
+
+def item_table(matrix, x_row, out_row, out_scale):
+    """Device array of svq_group_item from four equal-length device tensors (int32, int32, int32, float32)."""
+    import torch
+    t = torch.stack([matrix.to(torch.int32), x_row.to(torch.int32), out_row.to(torch.int32),
+                     out_scale.to(torch.float32).view(torch.int32)], dim=1).contiguous()
+    return t
+
+
+def svq_moe_grouped_gemv_workspace_size(n_mats: int, n_items: int, N: int, accumulate: bool) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().svq_moe_grouped_gemv_workspace_size(n_mats, n_items, N, int(accumulate), ctypes.byref(n)),
+           "svq_moe_grouped_gemv_workspace_size")
+    return int(n.value)
+
+
+def svq_moe_grouped_gemv(mats_dev, n_mats, N, K, max_b_d, items_dev, n_items, max_items_per_matrix, x, x_mode,
+                         y, n_out_rows, accumulate, ws, stream=None):
+    _check(lib().svq_moe_grouped_gemv(_ptr(mats_dev), n_mats, N, K, max_b_d, _ptr(items_dev), n_items,
+                                      max_items_per_matrix, _ptr(x), x_mode, _ptr(y), n_out_rows, int(accumulate),
+                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "svq_moe_grouped_gemv")
 
 
 def svq_get_device_status(stream=None) -> int:

@@ -9,6 +9,7 @@
 #include "layout.cuh"
 #include "svq.h"
 #include "gemm_params.h"
+#include "moe_params.h"
 #include "svq_internal.h"
 
 namespace {
@@ -244,6 +245,43 @@ int svq_linear_gemm(const svq_matrix* W, const uint16_t* x, int x_dtype, int M, 
   d.packed = W->packed; d.codebook = W->codebook; d.scale = W->radius_scale; d.offset = W->radius_offset;
   d.perm = W->perm; d.x = x; d.x_bf16 = x_dtype == SVQ_BF16; d.y = y; d.y_f32 = y_dtype == SVQ_F32;
   return cuda_status(svq::launch_gemm(d, g, workspace, status, (cudaStream_t)stream));
+}
+
+int svq_moe_grouped_gemv_workspace_size(int n_mats, int n_items, int N, int accumulate, size_t* bytes) {
+  if (!bytes || n_mats < 1 || n_items < 0 || N < 1) return SVQ_ERR_INVALID_ARG;
+  *bytes = svq::moe_workspace_layout(n_mats, n_items, N, accumulate ? 1 : 0).total;
+  return SVQ_OK;
+}
+
+int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int max_b_d, const svq_group_item* items,
+                         int n_items, int max_items_per_matrix, const void* x, int x_mode, float* y,
+                         int n_out_rows, int accumulate, void* workspace, size_t workspace_bytes,
+                         svq_stream_t stream) {
+  if (!mats || !items || !x || !y || n_mats < 1 || n_items < 1 || n_out_rows < 1) return SVQ_ERR_INVALID_ARG;
+  if (max_b_d < 1 || max_b_d > 10 || !svq::layout_supported(N, K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (n_mats > 16384 || max_items_per_matrix < 1) return SVQ_ERR_INVALID_ARG;
+  if (x_mode != SVQ_X_F16 && x_mode != SVQ_X_SWIGLU_F32) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(mats, 8) || !aligned(items, 4) || !aligned(y, 4) || !aligned(x, x_mode == SVQ_X_F16 ? 2 : 4))
+    return SVQ_ERR_INVALID_ARG;
+  const int mt = max_items_per_matrix == 1 ? 1 : (max_items_per_matrix == 2 ? 2 : 4);
+  if (svq::moe_smem_bytes(max_b_d, K, mt) > 220 * 1024) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  const svq::MoeWorkspace w = svq::moe_workspace_layout(n_mats, n_items, N, accumulate ? 1 : 0);
+  if (!workspace || workspace_bytes < w.total || !aligned(workspace, 256)) return SVQ_ERR_WORKSPACE;
+  const int sms = num_sms();
+  int* status = status_word();
+  if (sms <= 0 || !status) return SVQ_ERR_CUDA;
+  char* b = reinterpret_cast<char*>(workspace);
+  svq::MoeKParams p;
+  p.mats = mats; p.n_mats = n_mats; p.N = N; p.K = K; p.max_b_d = max_b_d;
+  p.items = items; p.n_items = n_items; p.x = x; p.x_mode = x_mode; p.y = y; p.accumulate = accumulate ? 1 : 0;
+  p.offsets = reinterpret_cast<int*>(b + w.offsets);
+  p.cursor = reinterpret_cast<int*>(b + w.cursor);
+  p.sorted = reinterpret_cast<int*>(b + w.sorted);
+  p.active = reinterpret_cast<int*>(b + w.active);
+  p.n_active = reinterpret_cast<int*>(b + w.n_active);
+  p.item_out = accumulate ? reinterpret_cast<float*>(b + w.item_out) : nullptr;
+  p.status = status;
+  return cuda_status(svq::launch_moe(p, mt, n_out_rows, sms, (cudaStream_t)stream));
 }
 
 int svq_get_device_status(svq_stream_t stream) {

@@ -37,16 +37,16 @@
 namespace svq {
 namespace {
 
-constexpr size_t kSmemPerCtaTwo = 110 * 1024;   // two CTAs per SM
-constexpr size_t kSmemPerCtaOne = kGemvSmemMax;
-
-// codebook replicas + x slice + cross-warp reduction buffer
+// codebook replicas (at most 32 KB) + x slice + cross-warp reduction buffer
 size_t cta_smem(int b_d, int mt, int K, int S) {
+  const int R = b_d <= 8 ? 8 : (b_d == 9 ? 4 : 2);
   const int B = K / kBlockCols;
   const int nbmax = (B + S - 1) / S;
-  return ((size_t)16 << b_d) * 8 + (size_t)mt * nbmax * kBlockCols * 2 +
+  return ((size_t)16 * R << b_d) + (size_t)mt * nbmax * kBlockCols * 2 +
          (size_t)kGemvWarps * mt * kTileRows * sizeof(float);
 }
+
+size_t up256(size_t b) { return (b + 255) / 256 * 256; }
 
 }  // namespace
 
@@ -56,12 +56,14 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
   plan->n_mats = n_mats;
   plan->M = M;
   plan->mt = mt;
-  const int per_sm = mt <= 2 ? 2 : 1;
-  const size_t smem_cap = per_sm == 2 ? kSmemPerCtaTwo : kSmemPerCtaOne;
+  // 4 CTAs (16 warps) per SM for 1-2 tokens per pass, 2 for wider passes
+  // (register-limited); shared memory per CTA is capped accordingly.
+  const int per_sm = mt <= 2 ? 4 : 2;
+  const size_t smem_cap = (227 * 1024) / per_sm - 1024;
   const int slots = num_sms * per_sm;
-  // One CTA per (128-row tile, k-slice).  Start with one slice per tile (at the
-  // smallest count shared memory allows), then repeatedly split the matrix whose
-  // CTAs carry the most blocks while the grid still fits in one wave.
+  // One CTA per (128-row tile, k-slice).  Start with the fewest slices shared
+  // memory allows, then repeatedly split the matrix whose CTAs carry the most
+  // blocks while the grid still fits in one wave.
   int S[kGemvMaxMats], R[kGemvMaxMats], B[kGemvMaxMats];
   int total = 0;
   for (int i = 0; i < n_mats; ++i) {
@@ -69,7 +71,7 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
     B[i] = mats[i].K / kBlockCols;
     S[i] = 1;
     while (S[i] < B[i] && cta_smem(mats[i].b_d, mt, mats[i].K, S[i]) > smem_cap) ++S[i];
-    if (cta_smem(mats[i].b_d, mt, mats[i].K, S[i]) > kSmemPerCtaOne) return false;
+    if (cta_smem(mats[i].b_d, mt, mats[i].K, S[i]) > smem_cap) return false;
     total += R[i] * S[i];
   }
   for (;;) {
@@ -92,12 +94,9 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
     pm.n_rc = R[i];
     pm.ctas = S[i] * R[i];
     pm.ws_offset = off;
-    pm.ws_bytes = 0;
-    if (S[i] > 1) {
-      const size_t part = ((size_t)S[i] * mt * d.N * sizeof(float) + 255) / 256 * 256;
-      const size_t cnt = ((size_t)R[i] * sizeof(unsigned) + 255) / 256 * 256;
-      pm.ws_bytes = part + cnt;
-    }
+    pm.xp_bytes = up256((size_t)mt * d.K * 2);
+    pm.part_bytes = S[i] > 1 ? up256((size_t)S[i] * mt * d.N * sizeof(float)) : 0;
+    pm.ws_bytes = pm.xp_bytes + pm.part_bytes + (S[i] > 1 ? up256((size_t)R[i] * sizeof(unsigned)) : 0);
     off += pm.ws_bytes;
     ctas += pm.ctas;
   }
@@ -111,26 +110,36 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
   const int passes = (plan.M + mt - 1) / mt;
   for (int p = 0; p < passes; ++p) {
     const int m0 = p * mt, Mp = std::min(mt, plan.M - m0);
+    GatherParams gp{};
+    gp.n_mats = plan.n_mats;
     GemvKParams kp{};
     kp.n_mats = plan.n_mats;
     kp.y_f32 = y_f32;
     size_t smem = 0;
-    int cta = 0;
+    int cta = 0, gcta = 0;
     for (int i = 0; i < plan.n_mats; ++i) {
       const GemvMatDesc& d = mats[i];
       const GemvPlanMat& pm = plan.m[i];
+      char* base = reinterpret_cast<char*>(ws) + pm.ws_offset;
+      uint16_t* xp = reinterpret_cast<uint16_t*>(base);
+      GatherMat& gm = gp.mats[i];
+      gm.x = d.x + (size_t)m0 * d.K;
+      gm.perm = d.perm;
+      gm.xp = xp;
+      gm.K = d.K;
+      gm.M = Mp;
+      gm.cta_begin = gcta;
+      gcta += (int)(((long long)Mp * d.K + 2047) / 2048);
       GemvKMat& g = kp.mats[i];
       g.packed = reinterpret_cast<const uint8_t*>(d.packed);
       g.codebook = reinterpret_cast<const uint4*>(d.codebook);
       g.scale = d.scale;
       g.offset = d.offset;
-      g.perm = d.perm;
-      g.x = d.x + (size_t)m0 * d.K;
+      g.xp = xp;
       g.y = reinterpret_cast<char*>(d.y) + (size_t)m0 * d.N * (y_f32 ? 4 : 2);
       if (pm.S > 1) {
-        char* base = reinterpret_cast<char*>(ws) + pm.ws_offset;
-        g.partial = reinterpret_cast<float*>(base);
-        g.counters = reinterpret_cast<unsigned*>(base + ((size_t)pm.S * mt * d.N * sizeof(float) + 255) / 256 * 256);
+        g.partial = reinterpret_cast<float*>(base + pm.xp_bytes);
+        g.counters = reinterpret_cast<unsigned*>(base + pm.xp_bytes + pm.part_bytes);
       } else {
         g.partial = nullptr;
         g.counters = nullptr;
@@ -139,7 +148,8 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
       cta += pm.ctas;
       smem = std::max(smem, cta_smem(d.b_d, mt, d.K, pm.S));
     }
-    cudaError_t e;
+    cudaError_t e = launch_gather(gp, gcta, st);
+    if (e != cudaSuccess) return e;
     switch (mt) {
       case 1: e = launch_gemv_mt<1>(kp, cta, smem, st); break;
       case 2: e = launch_gemv_mt<2>(kp, cta, smem, st); break;

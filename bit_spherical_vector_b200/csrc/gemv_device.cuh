@@ -1,0 +1,167 @@
+#pragma once
+// gemv_device.cuh -- device-side building blocks of the fused SVQ
+// decode-and-multiply (shared by the grouped GEMV and the MoE kernels):
+// cache-policy loads, lane-block loads and the per-block decode + dot product.
+//
+// A lane owns 4 rows x 16 subvectors of a block (layout.cuh).  For each
+// subvector: idx and radius code come out of the payload word with one shift
+// and one mask each; the fp16 codeword is gathered from the lane's replica of
+// the shared-memory codebook (conflict free); the subvector's sign bits are
+// XORed onto the fp16 sign bits (the shifted sign word puts each pair's two
+// signs on bits 15 and 31); 8 products are summed in fp16x2 and the radius
+// r = offset + scale * code ("SAGE", arXiv 2610.14745, Figure 2 caption: signs,
+// direction index, quantized radius) scales the sum in fp32.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "layout.cuh"
+
+namespace svq {
+namespace {
+
+// L2 cache policies: packed codes are read once per call (evict first), while a
+// matrix's small reused tables -- codebook, permutation, radius parameters and
+// the activations -- should stay resident across calls (evict last).  Without
+// this a stream of layers evicts every table and each CTA's prologue pays HBM
+// latency twice (permutation, then x).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ int ldg_keep_i32(const int32_t* p, uint64_t pol) {
+  int v;
+  asm("ld.global.nc.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(v) : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ uint16_t ldg_keep_u16(const uint16_t* p, uint64_t pol) {
+  uint16_t v;
+  asm("ld.global.nc.L2::cache_hint.b16 %0, [%1], %2;" : "=h"(v) : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(const unsigned char* base, uint32_t byte_off) {
+  return *reinterpret_cast<const uint4*>(base + byte_off);
+}
+
+template <int k>
+__device__ __forceinline__ uint32_t shl(uint32_t x) {
+  if constexpr (k >= 0) return x << k; else return x >> (-k);
+}
+
+__device__ __forceinline__ __half2 as_h2(uint32_t u) {
+  return *reinterpret_cast<const __half2*>(&u);
+}
+
+__device__ __forceinline__ void load_block(uint4 (&d)[kChunks], const uint8_t* blk, int L, int lane,
+                                           uint64_t pol) {
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) d[c] = ldg_stream(blk + ((size_t)c * L + lane) * 16, pol);
+}
+
+// Shared-memory codebook with R replicas (R = 8, 4 or 2): entry e of replica q
+// sits in 16-byte slot e*R + q, lane l reads replica l % R.  With R = 8 the 8
+// lanes of an LDS.128 phase always hit 8 different bank groups; R is lowered
+// for 512- and 1024-entry codebooks to keep the table at 32 KB (two lanes of
+// a phase may then share a bank group).  The payload's index field is moved
+// to bit l0 = 4 + log2(R) (byte offset e * 16R) with one shift.
+struct CbShift {
+  uint32_t l0, r1, r2, mask;
+};
+
+__device__ __forceinline__ int cb_replicas(int b_d) { return b_d <= 8 ? 8 : (b_d == 9 ? 4 : 2); }
+
+__device__ __forceinline__ CbShift cb_shift(int b_d) {
+  const int R = cb_replicas(b_d);
+  const uint32_t l0 = 4u + (R == 8 ? 3u : (R == 4 ? 2u : 1u));
+  CbShift c;
+  c.l0 = l0;
+  c.r1 = 10u - l0;
+  c.r2 = 20u - l0;
+  c.mask = ((1u << b_d) - 1u) << l0;
+  return c;
+}
+
+template <int MT>
+__device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const unsigned char* xb,
+                                              int xstride_bytes, const unsigned char* cbs, uint32_t q16,
+                                              const CbShift& cs, uint32_t CODEM, const float2 (&scp)[2],
+                                              const float2 (&ofp)[2], float2 (&acc)[2][MT]) {
+  uint32_t w[kWords];
+#pragma unroll
+  for (int c = 0; c < kChunks; ++c) {
+    w[4 * c] = d[c].x; w[4 * c + 1] = d[c].y; w[4 * c + 2] = d[c].z; w[4 * c + 3] = d[c].w;
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    uint4 xv[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) xv[m] = lds128(xb, m * xstride_bytes + 16 * j);
+    const uint32_t S = w[j];
+    float vf[4];
+    float dsum[4][MT];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int v = 4 * j + r;
+      uint32_t ia, vb;
+      if (v < 60) {
+        const uint32_t pw = w[16 + v / 3];
+        switch (v % 3) {
+          case 0: ia = (pw << cs.l0) & cs.mask; vb = shl<13>(pw) & CODEM; break;
+          case 1: ia = (pw >> cs.r1) & cs.mask; vb = shl<3>(pw) & CODEM; break;
+          default: ia = (pw >> cs.r2) & cs.mask; vb = shl<-7>(pw) & CODEM; break;
+        }
+      } else {
+        const int a = v - 60;
+        const uint32_t pw = ((w[16 + 5 * a] >> 30) << 8) | ((w[17 + 5 * a] >> 30) << 6) |
+                            ((w[18 + 5 * a] >> 30) << 4) | ((w[19 + 5 * a] >> 30) << 2) |
+                            (w[20 + 5 * a] >> 30);
+        ia = (pw << cs.l0) & cs.mask;
+        vb = shl<13>(pw) & CODEM;
+      }
+      // replica offset q16 (below bit l0) and the scaled index do not overlap: OR, not add
+      uint4 cw = lds128(cbs, ia | q16);
+      vf[r] = __uint_as_float(vb | 0x3F800000u);     // 1 + code * 2^-BR
+      cw.x ^= (S << (4 * r + 0)) & 0x80008000u;
+      cw.y ^= (S << (4 * r + 1)) & 0x80008000u;
+      cw.z ^= (S << (4 * r + 2)) & 0x80008000u;
+      cw.w ^= (S << (4 * r + 3)) & 0x80008000u;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        __half2 p = __hmul2(as_h2(cw.x), as_h2(xv[m].x));
+        p = __hfma2(as_h2(cw.y), as_h2(xv[m].y), p);
+        p = __hfma2(as_h2(cw.z), as_h2(xv[m].z), p);
+        p = __hfma2(as_h2(cw.w), as_h2(xv[m].w), p);
+        dsum[r][m] = __half2float(__hadd(__low2half(p), __high2half(p)));
+      }
+    }
+    // radius r = scp * v + ofp and accumulation, two rows per packed fp32x2 FMA
+    const float2 r01 = __ffma2_rn(scp[0], make_float2(vf[0], vf[1]), ofp[0]);
+    const float2 r23 = __ffma2_rn(scp[1], make_float2(vf[2], vf[3]), ofp[1]);
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      acc[0][m] = __ffma2_rn(r01, make_float2(dsum[0][m], dsum[1][m]), acc[0][m]);
+      acc[1][m] = __ffma2_rn(r23, make_float2(dsum[2][m], dsum[3][m]), acc[1][m]);
+    }
+  }
+}
+
+}  // namespace
+}  // namespace svq

@@ -10,9 +10,9 @@
 // (Figures 1 and 5).
 //
 // B200 mapping:
-//   * a CTA of 8 warps works on one 128-row tile of one matrix and one k-slice;
+//   * a CTA of 4 warps works on one 128-row tile of one matrix and one k-slice;
 //     the warps split the slice's blocks, each lane owns 4 complete rows, so a
-//     row's partial sum never leaves its thread in the hot loop; the 8 warps'
+//     row's partial sum never leaves its thread in the hot loop; the warps'
 //     sums are combined once in shared memory;
 //   * packed codes stream from HBM with 16-byte coalesced loads
 //     (ld.global.nc.L1::no_allocate), one block (9 loads per lane) ahead;
@@ -20,8 +20,9 @@
 //     replica q at 16-byte slot 8e + q, and lane l reads replica l % 8: the 8
 //     lanes of each quarter-warp phase of an LDS.128 hit 8 different bank
 //     groups whatever the indices, so the random gather is conflict free;
-//   * each warp gathers its columns of x[perm] into shared memory (eight
-//     independent gathers in flight per lane) and reads them with broadcast loads;
+//   * x[perm] is gathered once per matrix by gather.cu; each warp copies its
+//     columns of it into shared memory (16-byte asynchronous copies) and reads
+//     them with broadcast loads;
 //   * signs are applied by XOR on fp16 sign bits; the eight products of a
 //     subvector are summed in fp16x2, then scaled by the radius and
 //     accumulated across subvectors in fp32;
@@ -36,106 +37,19 @@
 #include "layout.cuh"
 #include "svq_internal.h"
 #include "gemv_params.h"
+#include "gemv_device.cuh"
 
 namespace svq {
 namespace {
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ uint4 lds128(const unsigned char* base, uint32_t byte_off) {
-  return *reinterpret_cast<const uint4*>(base + byte_off);
-}
-
-template <int k>
-__device__ __forceinline__ uint32_t shl(uint32_t x) {
-  if constexpr (k >= 0) return x << k; else return x >> (-k);
-}
-
-__device__ __forceinline__ __half2 as_h2(uint32_t u) {
-  return *reinterpret_cast<const __half2*>(&u);
-}
-
-__device__ __forceinline__ void load_block(uint4 (&d)[kChunks], const uint8_t* blk, int L, int lane) {
-#pragma unroll
-  for (int c = 0; c < kChunks; ++c) d[c] = ldg_stream(blk + ((size_t)c * L + lane) * 16);
-}
-
-template <int MT>
-__device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const unsigned char* xb,
-                                              int xstride_bytes, const unsigned char* cbs, uint32_t q16,
-                                              uint32_t IDX7, uint32_t CODEM, const float2 (&scp)[2],
-                                              const float2 (&ofp)[2], float2 (&acc)[2][MT]) {
-  uint32_t w[kWords];
-#pragma unroll
-  for (int c = 0; c < kChunks; ++c) {
-    w[4 * c] = d[c].x; w[4 * c + 1] = d[c].y; w[4 * c + 2] = d[c].z; w[4 * c + 3] = d[c].w;
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    uint4 xv[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) xv[m] = lds128(xb, m * xstride_bytes + 16 * j);
-    const uint32_t S = w[j];
-    float vf[4];
-    float dsum[4][MT];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int v = 4 * j + r;
-      uint32_t ia, vb;
-      if (v < 60) {
-        const uint32_t pw = w[16 + v / 3];
-        switch (v % 3) {
-          case 0: ia = shl<7>(pw) & IDX7; vb = shl<13>(pw) & CODEM; break;
-          case 1: ia = shl<-3>(pw) & IDX7; vb = shl<3>(pw) & CODEM; break;
-          default: ia = shl<-13>(pw) & IDX7; vb = shl<-7>(pw) & CODEM; break;
-        }
-      } else {
-        const int a = v - 60;
-        const uint32_t pw = ((w[16 + 5 * a] >> 30) << 8) | ((w[17 + 5 * a] >> 30) << 6) |
-                            ((w[18 + 5 * a] >> 30) << 4) | ((w[19 + 5 * a] >> 30) << 2) |
-                            (w[20 + 5 * a] >> 30);
-        ia = shl<7>(pw) & IDX7;
-        vb = shl<13>(pw) & CODEM;
-      }
-      // replica offset q16 (bits 4..6) and the index (bits 7..) do not overlap: OR, not add
-      uint4 cw = lds128(cbs, ia | q16);
-      vf[r] = __uint_as_float(vb | 0x3F800000u);     // 1 + code * 2^-BR
-      cw.x ^= (S << (4 * r + 0)) & 0x80008000u;
-      cw.y ^= (S << (4 * r + 1)) & 0x80008000u;
-      cw.z ^= (S << (4 * r + 2)) & 0x80008000u;
-      cw.w ^= (S << (4 * r + 3)) & 0x80008000u;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        __half2 p = __hmul2(as_h2(cw.x), as_h2(xv[m].x));
-        p = __hfma2(as_h2(cw.y), as_h2(xv[m].y), p);
-        p = __hfma2(as_h2(cw.z), as_h2(xv[m].z), p);
-        p = __hfma2(as_h2(cw.w), as_h2(xv[m].w), p);
-        dsum[r][m] = __half2float(__hadd(__low2half(p), __high2half(p)));
-      }
-    }
-    // radius r = scp * v + ofp and accumulation, two rows per packed fp32x2 FMA
-    const float2 r01 = __ffma2_rn(scp[0], make_float2(vf[0], vf[1]), ofp[0]);
-    const float2 r23 = __ffma2_rn(scp[1], make_float2(vf[2], vf[3]), ofp[1]);
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      acc[0][m] = __ffma2_rn(r01, make_float2(dsum[0][m], dsum[1][m]), acc[0][m]);
-      acc[1][m] = __ffma2_rn(r23, make_float2(dsum[2][m], dsum[3][m]), acc[1][m]);
-    }
-  }
-}
-
-// One CTA = one 128-row tile of one matrix and one k-slice; its 8 warps split
-// the k-slice's blocks and their partial sums are combined in shared memory.
+// One CTA = one 128-row tile of one matrix and one k-slice; its warps split the
+// k-slice's blocks and their partial sums are combined in shared memory.
 template <int MT>
 __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char* smem, int y_f32) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BD = g.b_d, BR = 10 - BD;
-  const uint32_t IDX7 = ((1u << BD) - 1u) << 7;
+  const int R = cb_replicas(BD);
+  const CbShift cs = cb_shift(BD);
   const uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
   const int N = g.N, K = g.K, B = K / kBlockCols, S = g.S, M = g.M;
   const int t = c / S, s = c - t * S;
@@ -148,59 +62,55 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   const int row0 = t * kTileRows + 4 * lane;
 
   uint4* cbs = reinterpret_cast<uint4*>(smem);
-  unsigned char* xs = smem + ((size_t)16 << BD) * 8;                 // [MT][nbk*128] fp16
+  unsigned char* xs = smem + ((size_t)16 * R << BD);                  // [MT][nbk*128] fp16
   const int xstride = nbk * kBlockCols * 2;
-  float* red = reinterpret_cast<float*>(xs + (size_t)MT * xstride);  // [8 warps][MT][128]
+  float* red = reinterpret_cast<float*>(xs + (size_t)MT * xstride);  // [warps][MT][128]
 
   const uint8_t* tile_base = g.packed + tile_offset(K, t);
   const size_t blk_bytes = (size_t)L * kLaneBlockBytes;
+  const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
   uint4 d0[kChunks], d1[kChunks];
-  if (on && nb > 0) load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane);
+  if (on && nb > 0) load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane, pol_stream);
 
-  // Codebook replicas: entry e, replica q -> 16-byte slot 8e + q.  Thread i fills
-  // slot i with an asynchronous global->shared copy (consecutive slots per warp:
-  // no bank conflicts; the eight copies of one entry share a load request).
-  {
-    const uint32_t cb_s = (uint32_t)__cvta_generic_to_shared(cbs);
-    for (int i = threadIdx.x; i < (8 << BD); i += blockDim.x)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(cb_s + 16u * i), "l"(g.codebook + (i >> 3))
-                   : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  }
+  // Codebook replicas: thread i fills slot i (entry i / R, replica i % R) with an
+  // asynchronous global->shared copy; a warp covers consecutive slots.
+  const uint32_t cb_s = (uint32_t)__cvta_generic_to_shared(cbs);
+  for (int i = threadIdx.x; i < (R << BD); i += blockDim.x)
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(cb_s + 16u * i),
+                 "l"(g.codebook + i / R), "l"(pol_keep)
+                 : "memory");
   // Radius parameters of this lane's rows (weights: independent of earlier kernels).
   float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
   if (on) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      sc[r] = __half2float(__ushort_as_half(g.scale[row0 + r]));
-      of[r] = __half2float(__ushort_as_half(g.offset[row0 + r]));
+      sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.scale + row0 + r, pol_keep)));
+      of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + row0 + r, pol_keep)));
     }
   }
-  // Everything above reads weights only; x may be written by the previous kernel
-  // in the stream (programmatic dependent launch): wait for it here.
+  // Everything above reads weights only.  The permuted activations come from
+  // the gather kernel just before this one (programmatic dependent launch):
+  // wait for it here.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // This warp's columns of x[perm]: up to 16 gathers per lane in flight at once
-  // (all perm loads, then all x loads), i.e. two dependent round trips.
+  // This warp's columns of x[perm] (contiguous in the gathered copy): 16-byte
+  // asynchronous copies; rows beyond M are zero.
   {
-    const __half* xh = reinterpret_cast<const __half*>(g.x);
-    __half* xsh = reinterpret_cast<__half*>(xs);
     const int jc0 = (wb0 - kb0) * kBlockCols, ncw = nb * kBlockCols;
-    const int32_t* pp = g.perm + (size_t)kb0 * kBlockCols + jc0;
-    constexpr int U = MT == 1 ? 16 : 8;
-    for (int j0 = lane; j0 < ncw; j0 += 32 * U) {
-      int pj[U];
+    const uint32_t xs_s = (uint32_t)__cvta_generic_to_shared(xs);
 #pragma unroll
-      for (int u = 0; u < U; ++u) pj[u] = (j0 + 32 * u < ncw) ? __ldg(pp + j0 + 32 * u) : 0;
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        __half hv[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) hv[u] = (m < M) ? xh[(size_t)m * K + pj[u]] : __ushort_as_half(0);
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (j0 + 32 * u < ncw) xsh[(size_t)m * (xstride / 2) + jc0 + j0 + 32 * u] = hv[u];
+    for (int m = 0; m < MT; ++m) {
+      for (int j = lane * 8; j < ncw; j += 32 * 8) {
+        const uint32_t dst = xs_s + (uint32_t)(m * xstride + (jc0 + j) * 2);
+        if (m < M) {
+          asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
+                       "l"(g.xp + (size_t)m * K + (size_t)kb0 * kBlockCols + jc0 + j), "l"(pol_keep)
+                       : "memory");
+        } else {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+        }
       }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
   // Let the next kernel in the stream start its own weight-only prologue as this
   // grid's CTAs retire.
@@ -227,18 +137,18 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
     for (int m = 0; m < MT; ++m) acc[h][m] = make_float2(0.f, 0.f);
 
   const unsigned char* cbb = reinterpret_cast<const unsigned char*>(cbs);
-  const uint32_t q16 = (uint32_t)(lane & 7) * 16;
+  const uint32_t q16 = (uint32_t)(lane % R) * 16;
   const unsigned char* xw = xs + (size_t)(wb0 - kb0) * kBlockCols * 2;
   if (on) {
     for (int b = 0; b < nb; ++b) {
-      if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane);
-      process_block<MT>(d0, xw + b * kBlockCols * 2, xstride, cbb, q16, IDX7, CODEM, scp, ofp, acc);
+      if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
+      process_block<MT>(d0, xw + b * kBlockCols * 2, xstride, cbb, q16, cs, CODEM, scp, ofp, acc);
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     }
   }
 
-  // Combine the 8 warps' partial sums of the tile's 128 rows (fixed order).
+  // Combine the warps' partial sums of the tile's 128 rows (fixed order).
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
     float* rr = red + ((size_t)warp * MT + m) * kTileRows + 4 * lane;
@@ -299,7 +209,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 }
 
 template <int MT>
-__global__ void __launch_bounds__(kGemvWarps * 32, MT <= 2 ? 2 : 1)
+__global__ void __launch_bounds__(kGemvWarps * 32, MT <= 2 ? 4 : 2)
 gemv_kernel(const __grid_constant__ GemvKParams P) {
   extern __shared__ __align__(1024) unsigned char smem[];
   int mi = 0;

@@ -1,0 +1,295 @@
+// moe.cu -- grouped SVQ GEMV over a device-side list of (matrix, token) items,
+// for mixture-of-experts layers whose routing is produced on the GPU.
+//
+// Method ("SAGE", arXiv 2610.14745): each expert matrix is an SVQ matrix
+// (Figure 2 caption) applied with its own ESG permutation (Figure 6 caption);
+// the pages evaluate an MoE model (Qwen3-30B-A3B, abstract) but describe no
+// MoE kernel.  Design here:
+//   1. route_kernel (one CTA): counts the items of every matrix, builds the list
+//      of touched matrices and groups the item indices by matrix -- all on the
+//      device, no host round trip;
+//   2. moe_kernel (persistent): one work unit = (touched matrix, 128-row tile);
+//      the unit decodes its weights once and applies them to all of that
+//      matrix's items (up to MT tokens per pass), 8 warps splitting K, partial
+//      sums combined in shared memory; the input row of an item is either fp16
+//      x or, for a down projection, fp16(silu(gate) * up) computed on the fly
+//      from an fp32 [gate | up] row;
+//   3. combine_kernel (when accumulating): y[r] = sum of the items with
+//      out_row r, in item order (deterministic).
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "gemv_device.cuh"
+#include "layout.cuh"
+#include "moe_params.h"
+#include "svq.h"
+
+namespace svq {
+namespace {
+
+constexpr int kMoeWarps = 8;
+constexpr int kRouteThreads = 1024;
+
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(MoeKParams p) {
+  extern __shared__ int sh[];                   // [n_mats] counts, then scan scratch
+  int* cnt = sh;
+  __shared__ int s_warp[kRouteThreads / 32];
+  __shared__ int s_total;
+  for (int i = threadIdx.x; i < p.n_mats; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.n_items; i += blockDim.x) {
+    const int m = p.items[i].matrix;
+    if (m >= 0 && m < p.n_mats) atomicAdd(&cnt[m], 1);
+    else atomicExch(p.status, SVQ_ERR_INVALID_ARG);
+  }
+  __syncthreads();
+  // Exclusive scans of the counts (item offsets) and of the touched flags
+  // (active list), in chunks of blockDim.x matrices.
+  int base_items = 0, base_active = 0;
+  for (int c0 = 0; c0 < p.n_mats; c0 += blockDim.x) {
+    const int m = c0 + threadIdx.x;
+    const int v = m < p.n_mats ? cnt[m] : 0;
+    const int f = v > 0 ? 1 : 0;
+    // pack (items, active) into one 64-bit scan value
+    long long x = ((long long)v << 20) | f;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+      if (lane >= o) x += y;
+    }
+    __shared__ long long s_w[kRouteThreads / 32];
+    if (lane == 31) s_w[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      long long w = lane < (int)(blockDim.x / 32) ? s_w[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < (int)(blockDim.x / 32)) s_w[lane] = w;
+    }
+    __syncthreads();
+    const long long incl = x + (wid > 0 ? s_w[wid - 1] : 0);
+    const long long excl = incl - (((long long)v << 20) | f);
+    if (m < p.n_mats) {
+      p.offsets[m] = base_items + (int)(excl >> 20);
+      p.cursor[m] = 0;
+      if (f) p.active[base_active + (int)(excl & 0xFFFFF)] = m;
+    }
+    const long long tot = s_w[blockDim.x / 32 - 1];
+    __syncthreads();
+    base_items += (int)(tot >> 20);
+    base_active += (int)(tot & 0xFFFFF);
+  }
+  if (threadIdx.x == 0) {
+    p.offsets[p.n_mats] = base_items;
+    *p.n_active = base_active;
+    s_total = base_items;
+  }
+  (void)s_warp;
+  __syncthreads();
+  // Group item indices by matrix (order inside a matrix does not affect any
+  // result: every item is computed on its own).
+  for (int i = threadIdx.x; i < p.n_items; i += blockDim.x) {
+    const int m = p.items[i].matrix;
+    if (m < 0 || m >= p.n_mats) continue;
+    const int slot = atomicAdd(&p.cursor[m], 1);
+    p.sorted[p.offsets[m] + slot] = i;
+  }
+}
+
+template <int MT>
+__device__ void moe_unit(const MoeKParams& p, const svq_matrix& W, int m, int t, unsigned char* smem,
+                         int& cb_matrix) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = p.N, K = p.K, B = K / kBlockCols;
+  const int BD = W.b_d, BR = 10 - BD;
+  const int RR = cb_replicas(BD);
+  const CbShift cs = cb_shift(BD);
+  const uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
+  const int wb0 = (B * warp) / kMoeWarps, wb1 = (B * (warp + 1)) / kMoeWarps, nb = wb1 - wb0;
+  const int L = tile_lanes(N, t);
+  const bool on = lane < L;
+  const int row0 = t * kTileRows + 4 * lane;
+  uint4* cbs = reinterpret_cast<uint4*>(smem);
+  unsigned char* xs = smem + (size_t)32 * 1024;                  // [MT][K] fp16 after the codebook
+  const int xstride = K * 2;
+  float* red = reinterpret_cast<float*>(xs + (size_t)MT * xstride);   // [8][MT][128]
+  const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
+  const uint8_t* packed = reinterpret_cast<const uint8_t*>(W.packed);
+  const uint8_t* tile_base = packed + tile_offset(K, t);
+  const size_t blk_bytes = (size_t)L * kLaneBlockBytes;
+
+  __syncthreads();                                  // previous unit done with shared memory
+  if (cb_matrix != m) {
+    const uint4* cb = reinterpret_cast<const uint4*>(W.codebook);
+    for (int i = threadIdx.x; i < (RR << BD); i += blockDim.x) cbs[i] = __ldg(cb + i / RR);
+    cb_matrix = m;
+  }
+  float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
+  if (on) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(W.radius_scale + row0 + r, pol_keep)));
+      of[r] = __half2float(__ushort_as_half(ldg_keep_u16(W.radius_offset + row0 + r, pol_keep)));
+    }
+  }
+  float2 scp[2], ofp[2];
+  {
+    float sp[4], op[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (BR > 0) { sp[r] = sc[r] * (float)(1 << BR); op[r] = of[r] - sp[r]; }
+      else { sp[r] = 0.f; op[r] = of[r]; }
+    }
+    scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
+    ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
+  }
+  const int i0 = p.offsets[m], ni = p.offsets[m + 1] - i0;
+  for (int c0 = 0; c0 < ni; c0 += MT) {
+    const int nc = min(MT, ni - c0);
+    if (c0 > 0) __syncthreads();                    // previous chunk done with x and red
+    // x[perm] rows of this chunk's items (or fp16(silu(g) * u) for x_mode 1).
+    for (int e = threadIdx.x; e < MT * K; e += blockDim.x) {
+      const int c = e / K, j = e - c * K;
+      __half v = __ushort_as_half(0);
+      if (c < nc) {
+        const svq_group_item it = p.items[p.sorted[i0 + c0 + c]];
+        const int pj = ldg_keep_i32(W.perm + j, pol_keep);
+        if (p.x_mode == 0) {
+          v = __ushort_as_half(reinterpret_cast<const uint16_t*>(p.x)[(size_t)it.x_row * K + pj]);
+        } else {
+          const float* xr = reinterpret_cast<const float*>(p.x) + (size_t)it.x_row * 2 * K;
+          const float gv = xr[pj], uv = xr[K + pj];
+          v = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
+        }
+      }
+      reinterpret_cast<__half*>(xs)[(size_t)c * K + j] = v;
+    }
+    __syncthreads();
+    float2 acc[2][MT];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int q = 0; q < MT; ++q) acc[h][q] = make_float2(0.f, 0.f);
+    const unsigned char* cbb = reinterpret_cast<const unsigned char*>(cbs);
+    const uint32_t q16 = (uint32_t)(lane % RR) * 16;
+    if (on && nb > 0) {
+      uint4 d0[kChunks], d1[kChunks];
+      load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane, pol_stream);
+      for (int b = 0; b < nb; ++b) {
+        if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
+        process_block<MT>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, xstride, cbb, q16, cs, CODEM, scp, ofp,
+                          acc);
+#pragma unroll
+        for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < MT; ++q) {
+      float* rr = red + ((size_t)warp * MT + q) * kTileRows + 4 * lane;
+      *reinterpret_cast<float4*>(rr) = make_float4(acc[0][q].x, acc[0][q].y, acc[1][q].x, acc[1][q].y);
+    }
+    __syncthreads();
+    const int rows = L * 4;
+    for (int e = threadIdx.x; e < rows * nc; e += blockDim.x) {
+      const int c = e / rows, nl = e - c * rows;
+      float v = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < kMoeWarps; ++w8) v += red[((size_t)w8 * MT + c) * kTileRows + nl];
+      const int item = p.sorted[i0 + c0 + c];
+      const svq_group_item it = p.items[item];
+      const int n = t * kTileRows + nl;
+      v *= it.out_scale;
+      if (p.accumulate) p.item_out[(size_t)item * N + n] = v;
+      else p.y[(size_t)it.out_row * N + n] = v;
+    }
+  }
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_constant__ MoeKParams p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int R = num_tiles(p.N);
+  const int units = *p.n_active * R;
+  int cb_matrix = -1;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int a = u / R, t = u - a * R;
+    const int m = p.active[a];
+    const svq_matrix W = p.mats[m];
+    moe_unit<MT>(p, W, m, t, smem, cb_matrix);
+  }
+}
+
+// y[r][n] = sum over items i with out_row r (ascending i) of item_out[i][n].
+__global__ void combine_kernel(const MoeKParams p, int n_out_rows) {
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)n_out_rows * p.N) return;
+  const int r = (int)(e / p.N), n = (int)(e - (long long)r * p.N);
+  float s = 0.f;
+  bool any = false;
+  for (int i = 0; i < p.n_items; ++i) {
+    if (p.items[i].out_row == r) {
+      s += p.item_out[(size_t)i * p.N + n];
+      any = true;
+    }
+  }
+  if (any) p.y[(size_t)r * p.N + n] = s;
+}
+
+template <int MT>
+cudaError_t launch_moe_mt(const MoeKParams& p, int grid, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(moe_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  moe_kernel<MT><<<grid, kMoeWarps * 32, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t moe_smem_bytes(int max_b_d, int K, int mt) {
+  (void)max_b_d;                                   // replicas keep every codebook within 32 KB
+  return (size_t)32 * 1024 + (size_t)mt * K * 2 + (size_t)kMoeWarps * mt * kTileRows * 4;
+}
+
+MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate) {
+  MoeWorkspace w;
+  auto up = [](size_t b) { return (b + 255) / 256 * 256; };
+  size_t off = 0;
+  w.offsets = off; off += up((size_t)(n_mats + 1) * 4);
+  w.cursor = off; off += up((size_t)n_mats * 4);
+  w.sorted = off; off += up((size_t)n_items * 4);
+  w.active = off; off += up((size_t)n_mats * 4);
+  w.n_active = off; off += 256;
+  w.item_out = off; off += accumulate ? up((size_t)n_items * N * 4) : 0;
+  w.total = off;
+  return w;
+}
+
+cudaError_t launch_moe(MoeKParams p, int mt, int n_out_rows, int num_sms, cudaStream_t st) {
+  const size_t route_smem = (size_t)p.n_mats * 4;
+  cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_smem);
+  if (e != cudaSuccess) return e;
+  route_kernel<<<1, kRouteThreads, route_smem, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t smem = moe_smem_bytes(p.max_b_d, p.K, mt);
+  switch (mt) {
+    case 1: e = launch_moe_mt<1>(p, num_sms, smem, st); break;
+    case 2: e = launch_moe_mt<2>(p, num_sms, smem, st); break;
+    default: e = launch_moe_mt<4>(p, num_sms, smem, st); break;
+  }
+  if (e != cudaSuccess) return e;
+  if (p.accumulate) {
+    const long long work = (long long)n_out_rows * p.N;
+    combine_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(p, n_out_rows);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace svq

@@ -17,7 +17,7 @@ cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint
 
 // ---------------------------------------------------------------- GEMV
 constexpr int kGemvMaxMats = 8;
-constexpr int kGemvWarps = 8;            // warps per CTA; they split the k-slice of one 128-row tile
+constexpr int kGemvWarps = 4;            // warps per CTA; they split the k-slice of one 128-row tile
 constexpr int kGemvMaxTokens = 8;        // tokens per pass (more are split into passes)
 
 struct GemvMatDesc {                      // host-side description of one matrix of a launch
@@ -35,7 +35,8 @@ struct GemvPlanMat {
   int S;                                 // k-splits
   int n_rc;                              // 128-row tiles (one CTA per tile and k-slice)
   int ctas;                              // S * n_rc
-  size_t ws_offset;                      // partials then counters, 256-byte aligned
+  size_t ws_offset;                      // gathered x, partials, counters; 256-byte aligned
+  size_t xp_bytes, part_bytes;
   size_t ws_bytes;
 };
 

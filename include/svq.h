@@ -198,6 +198,44 @@ SVQ_API int svq_linear_gemm(const svq_matrix* W /* host */, const uint16_t* x, i
                             int y_dtype, void* workspace, size_t workspace_bytes, svq_stream_t stream);
 
 /*
+ * svq_moe_grouped_gemv -- many SVQ matrices applied to many rows in one call,
+ * driven by a DEVICE-side item list (mixture-of-experts layers, whose routing
+ * is produced on the GPU).  The pages evaluate SVQ on an MoE model
+ * (Qwen3-30B-A3B, abstract) without describing an MoE kernel; each expert
+ * matrix is an SVQ matrix as in Figure 2 with its own permutation (Figure 6).
+ *
+ *   for every item i:  v_i = out_scale_i * W[matrix_i] * in(x_row_i)
+ *   accumulate == 0:   y[out_row_i] = v_i          (out rows must be distinct)
+ *   accumulate == 1:   y[r] = sum of v_i over the items with out_row == r, in
+ *                      item order (rows with no item are left untouched)
+ * in(row): x_mode SVQ_X_F16 -> x is fp16 [*][K], in(row) = x[row];
+ *          x_mode SVQ_X_SWIGLU_F32 -> x is fp32 [*][2K] holding [gate | up],
+ *          in(row) = fp16(silu(gate) * up) computed per element in fp32.
+ * mats: DEVICE array of n_mats descriptors (same layout as svq_matrix), every
+ *   one N x K with b_d <= max_b_d; the host cannot read them, so the caller
+ *   guarantees them (the host checks N, K, max_b_d and the pointers it sees).
+ * items: DEVICE array of n_items.  Each touched matrix is decoded once per call
+ *   and applied to all of its items (up to max_items_per_matrix, a bound the
+ *   caller guarantees; it selects how many rows share one decode pass).
+ * y: fp32 [n_out_rows][N].  Workspace: svq_moe_grouped_gemv_workspace_size.
+ * Tolerance used by the tests: as svq_linear_gemv (1e-3 of sum |W| |in|).
+ */
+typedef struct svq_group_item {
+  int32_t matrix;    /* index into mats                         */
+  int32_t x_row;     /* input row                               */
+  int32_t out_row;   /* output row of y                         */
+  float out_scale;   /* multiplies W * in before it is written  */
+} svq_group_item;
+
+enum svq_x_mode { SVQ_X_F16 = 0, SVQ_X_SWIGLU_F32 = 1 };
+
+SVQ_API int svq_moe_grouped_gemv_workspace_size(int n_mats, int n_items, int N, int accumulate, size_t* bytes);
+SVQ_API int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int max_b_d,
+                                 const svq_group_item* items, int n_items, int max_items_per_matrix,
+                                 const void* x, int x_mode, float* y, int n_out_rows, int accumulate,
+                                 void* workspace, size_t workspace_bytes, svq_stream_t stream);
+
+/*
  * Synchronising read-and-clear of the device status word that kernels set
  * when a bounded wait runs out (SVQ_OK or SVQ_ERR_TIMEOUT).  Tests only.
  */
