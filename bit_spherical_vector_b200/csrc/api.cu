@@ -65,7 +65,7 @@ int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
 // Scratch for svq_linear_gemv_noalloc: split-K partial sums and completion
 // counters of one call.  Every GPU that loads the library holds these bytes
 // until the process exits.
-constexpr size_t kNoAllocScratchBytes = 4u << 20;
+constexpr size_t kNoAllocScratchBytes = 1u << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch for the current device, looked up (and

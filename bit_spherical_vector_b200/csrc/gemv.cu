@@ -18,8 +18,8 @@
 //     replica q at 16-byte slot 8e + q, and lane l reads replica l % 8: the 8
 //     lanes of each quarter-warp phase of an LDS.128 hit 8 different bank
 //     groups whatever the indices, so the random gather is conflict free;
-//   * x[perm] for the CTA's k-slice is gathered into shared memory once and
-//     read with broadcast loads;
+//   * each warp gathers x[perm] for its blocks itself, one block ahead of the
+//     decode, into two small shared-memory slots read with broadcast loads;
 //   * signs are applied by XOR on fp16 sign bits; the eight products of a
 //     subvector are summed in fp16x2, then scaled by the radius and
 //     accumulated across subvectors in fp32;
@@ -37,12 +37,12 @@
 namespace svq {
 namespace {
 
-// codebook replicas (at most 32 KB) + x slice + cross-warp reduction buffer
+// codebook replicas (at most 32 KB) + two x slots per warp + cross-warp reduction buffer
 size_t cta_smem(int b_d, int mt, int K, int S) {
+  (void)K;
+  (void)S;
   const int R = b_d <= 8 ? 8 : (b_d == 9 ? 4 : 2);
-  const int B = K / kBlockCols;
-  const int nbmax = (B + S - 1) / S;
-  return ((size_t)16 * R << b_d) + (size_t)mt * nbmax * kBlockCols * 2 +
+  return ((size_t)16 * R << b_d) + (size_t)kGemvWarps * 2 * mt * kBlockCols * 2 +
          (size_t)kGemvWarps * mt * kTileRows * sizeof(float);
 }
 
@@ -94,7 +94,7 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
     pm.n_rc = R[i];
     pm.ctas = S[i] * R[i];
     pm.ws_offset = off;
-    pm.xp_bytes = up256((size_t)mt * d.K * 2);
+    pm.xp_bytes = 0;
     pm.part_bytes = S[i] > 1 ? up256((size_t)S[i] * mt * d.N * sizeof(float)) : 0;
     pm.ws_bytes = pm.xp_bytes + pm.part_bytes + (S[i] > 1 ? up256((size_t)R[i] * sizeof(unsigned)) : 0);
     off += pm.ws_bytes;
@@ -110,32 +110,22 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
   const int passes = (plan.M + mt - 1) / mt;
   for (int p = 0; p < passes; ++p) {
     const int m0 = p * mt, Mp = std::min(mt, plan.M - m0);
-    GatherParams gp{};
-    gp.n_mats = plan.n_mats;
     GemvKParams kp{};
     kp.n_mats = plan.n_mats;
     kp.y_f32 = y_f32;
     size_t smem = 0;
-    int cta = 0, gcta = 0;
+    int cta = 0;
     for (int i = 0; i < plan.n_mats; ++i) {
       const GemvMatDesc& d = mats[i];
       const GemvPlanMat& pm = plan.m[i];
       char* base = reinterpret_cast<char*>(ws) + pm.ws_offset;
-      uint16_t* xp = reinterpret_cast<uint16_t*>(base);
-      GatherMat& gm = gp.mats[i];
-      gm.x = d.x + (size_t)m0 * d.K;
-      gm.perm = d.perm;
-      gm.xp = xp;
-      gm.K = d.K;
-      gm.M = Mp;
-      gm.cta_begin = gcta;
-      gcta += (int)(((long long)Mp * d.K + 2047) / 2048);
       GemvKMat& g = kp.mats[i];
       g.packed = reinterpret_cast<const uint8_t*>(d.packed);
       g.codebook = reinterpret_cast<const uint4*>(d.codebook);
       g.scale = d.scale;
       g.offset = d.offset;
-      g.xp = xp;
+      g.perm = d.perm;
+      g.x = d.x + (size_t)m0 * d.K;
       g.y = reinterpret_cast<char*>(d.y) + (size_t)m0 * d.N * (y_f32 ? 4 : 2);
       if (pm.S > 1) {
         g.partial = reinterpret_cast<float*>(base + pm.xp_bytes);
@@ -148,8 +138,7 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
       cta += pm.ctas;
       smem = std::max(smem, cta_smem(d.b_d, mt, d.K, pm.S));
     }
-    cudaError_t e = launch_gather(gp, gcta, st);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
     switch (mt) {
       case 1: e = launch_gemv_mt<1>(kp, cta, smem, st); break;
       case 2: e = launch_gemv_mt<2>(kp, cta, smem, st); break;

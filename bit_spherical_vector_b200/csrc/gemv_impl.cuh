@@ -20,9 +20,10 @@
 //     replica q at 16-byte slot 8e + q, and lane l reads replica l % 8: the 8
 //     lanes of each quarter-warp phase of an LDS.128 hit 8 different bank
 //     groups whatever the indices, so the random gather is conflict free;
-//   * x[perm] is gathered once per matrix by gather.cu; each warp copies its
-//     columns of it into shared memory (16-byte asynchronous copies) and reads
-//     them with broadcast loads;
+//   * each warp gathers x[perm] for its blocks itself, software-pipelined: the
+//     permutation of block b+2 and the activations of block b+1 are loaded
+//     while block b is decoded, into the other of two small shared-memory
+//     slots that the lanes read with broadcast loads;
 //   * signs are applied by XOR on fp16 sign bits; the eight products of a
 //     subvector are summed in fp16x2, then scaled by the radius and
 //     accumulated across subvectors in fp32;
@@ -62,9 +63,11 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   const int row0 = t * kTileRows + 4 * lane;
 
   uint4* cbs = reinterpret_cast<uint4*>(smem);
-  unsigned char* xs = smem + ((size_t)16 * R << BD);                  // [MT][nbk*128] fp16
-  const int xstride = nbk * kBlockCols * 2;
-  float* red = reinterpret_cast<float*>(xs + (size_t)MT * xstride);  // [warps][MT][128]
+  // Per warp: two x slots (double buffer) of MT rows x 128 columns fp16.
+  unsigned char* xs = smem + ((size_t)16 * R << BD) + (size_t)warp * 2 * MT * kBlockCols * 2;
+  constexpr int kXSlot = MT * kBlockCols * 2;          // bytes per slot
+  float* red = reinterpret_cast<float*>(smem + ((size_t)16 * R << BD) +
+                                        (size_t)kGemvWarps * 2 * kXSlot);   // [warps][MT][128]
 
   const uint8_t* tile_base = g.packed + tile_offset(K, t);
   const size_t blk_bytes = (size_t)L * kLaneBlockBytes;
@@ -79,7 +82,9 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
     asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(cb_s + 16u * i),
                  "l"(g.codebook + i / R), "l"(pol_keep)
                  : "memory");
-  // Radius parameters of this lane's rows (weights: independent of earlier kernels).
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  // Radius parameters of this lane's rows and the permutation of the warp's
+  // first two blocks (all weights: independent of earlier kernels).
   float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
   if (on) {
 #pragma unroll
@@ -88,30 +93,30 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + row0 + r, pol_keep)));
     }
   }
-  // Everything above reads weights only.  The permuted activations come from
-  // the gather kernel just before this one (programmatic dependent launch):
-  // wait for it here.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // This warp's columns of x[perm] (contiguous in the gathered copy): 16-byte
-  // asynchronous copies; rows beyond M are zero.
-  {
-    const int jc0 = (wb0 - kb0) * kBlockCols, ncw = nb * kBlockCols;
-    const uint32_t xs_s = (uint32_t)__cvta_generic_to_shared(xs);
+  // x[perm] pipeline: lane l owns columns l, l+32, l+64, l+96 of a block.  The
+  // permutation of block b+2 and the activations of block b+1 are loaded while
+  // block b is decoded; the activations land in the other x slot.
+  const int32_t* pw = g.perm + (size_t)wb0 * kBlockCols + lane;
+  const uint16_t* xg = g.x;
+  int pj_a[4], pj_b[4];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      for (int j = lane * 8; j < ncw; j += 32 * 8) {
-        const uint32_t dst = xs_s + (uint32_t)(m * xstride + (jc0 + j) * 2);
-        if (m < M) {
-          asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
-                       "l"(g.xp + (size_t)m * K + (size_t)kb0 * kBlockCols + jc0 + j), "l"(pol_keep)
-                       : "memory");
-        } else {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
-        }
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int u = 0; u < 4; ++u) {
+    pj_a[u] = nb > 0 ? ldg_keep_i32(pw + 32 * u, pol_keep) : 0;
+    pj_b[u] = nb > 1 ? ldg_keep_i32(pw + kBlockCols + 32 * u, pol_keep) : 0;
   }
+  // The activations may be written by the previous kernel in the stream
+  // (programmatic dependent launch): wait for it before reading x.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  uint16_t hx[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int u = 0; u < 4; ++u) hx[m][u] = (m < M && nb > 0) ? ldg_keep_u16(xg + (size_t)m * K + pj_a[u], pol_keep) : 0;
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      reinterpret_cast<uint16_t*>(xs + m * kBlockCols * 2)[lane + 32 * u] = hx[m][u];
   // Let the next kernel in the stream start its own weight-only prologue as this
   // grid's CTAs retire.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -138,13 +143,32 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 
   const unsigned char* cbb = reinterpret_cast<const unsigned char*>(cbs);
   const uint32_t q16 = (uint32_t)(lane % R) * 16;
-  const unsigned char* xw = xs + (size_t)(wb0 - kb0) * kBlockCols * 2;
-  if (on) {
-    for (int b = 0; b < nb; ++b) {
+  for (int b = 0; b < nb; ++b) {
+    // activations of block b+1 (permutation already loaded), permutation of block b+2
+    if (b + 1 < nb) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) hx[m][u] = m < M ? ldg_keep_u16(xg + (size_t)m * K + pj_b[u], pol_keep) : 0;
+      if (b + 2 < nb) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) pj_b[u] = ldg_keep_i32(pw + (size_t)(b + 2) * kBlockCols + 32 * u, pol_keep);
+      }
+    }
+    if (on) {
       if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
-      process_block<MT>(d0, xw + b * kBlockCols * 2, xstride, cbb, q16, cs, CODEM, scp, ofp, acc);
+      process_block<MT>(d0, xs + (b & 1) * kXSlot, kBlockCols * 2, cbb, q16, cs, CODEM, scp, ofp, acc);
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
+    }
+    if (b + 1 < nb) {
+      __syncwarp();                                   // all lanes done reading the slot about to be reused
+      unsigned char* nx = xs + ((b + 1) & 1) * kXSlot;
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) reinterpret_cast<uint16_t*>(nx + m * kBlockCols * 2)[lane + 32 * u] = hx[m][u];
+      __syncwarp();
     }
   }
 

@@ -15,7 +15,8 @@ struct GemvKMat {
   const uint4* codebook;
   const uint16_t* scale;
   const uint16_t* offset;
-  const uint16_t* xp;     // x[:, perm], fp16 [M][K] (written by the gather kernel)
+  const int32_t* perm;    // [K]
+  const uint16_t* x;      // fp16 [M][K], natural input order
   void* y;                // [M][N]
   float* partial;         // [S][M][N]
   unsigned* counters;     // [n_rc] (one per 128-row tile)
@@ -28,20 +29,7 @@ struct GemvKParams {
   int y_f32;
 };
 
-struct GatherMat {
-  const uint16_t* x;      // fp16 [M][K]
-  const int32_t* perm;    // [K]
-  uint16_t* xp;           // fp16 [M][K] out
-  int K, M, cta_begin;
-};
-
-struct GatherParams {
-  GatherMat mats[kGemvMaxMats];
-  int n_mats;
-};
-
 constexpr size_t kGemvSmemMax = 220 * 1024;
-cudaError_t launch_gather(const GatherParams& p, int grid, cudaStream_t st);
 
 template <int MT>
 cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStream_t st);

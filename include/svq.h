@@ -161,12 +161,13 @@ SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const ui
  * only a stream, code that runs after its host has frozen its memory pools, or
  * a real-time loop where a cudaMalloc could stall.  This entry point takes the
  * same inputs and outputs as svq_linear_gemv (x fp16 [M][K], y [M][N] of
- * SVQ_F16 or SVQ_F32, M 1..16) but keeps its split-K scratch in a fixed 4 MiB
+ * SVQ_F16 or SVQ_F32, M 1..16) but keeps its split-K scratch in a fixed 1 MiB
  * array inside the library, which every GPU that loads the library holds
  * until the process exits.  It allocates nothing and calls no allocating
  * routine.
  *   - A call whose scratch need (svq_linear_gemv_workspace_size) exceeds
- *     4 MiB returns SVQ_ERR_WORKSPACE and enqueues nothing.
+ *     1 MiB returns SVQ_ERR_WORKSPACE and enqueues nothing (e.g. M = 5..8 on a
+ *     2560 x 9728 matrix; split such a call into passes of at most 4 rows).
  *   - The first call on a device looks up the array's device address and
  *     zero-fills it on `stream`; make that first call before any stream
  *     capture.

@@ -16,7 +16,7 @@ import bit_spherical_vector_b200 as svq
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-3
-LIMIT = 4 << 20
+LIMIT = 1 << 20
 
 
 def _noalloc(desc, x_ptr, M, y_ptr):
@@ -50,10 +50,10 @@ def test_noalloc_matches_workspace_entry_two_calls(N, K, M, b_d):
 
 
 def test_noalloc_rejects_scratch_beyond_limit():
-    """A shape whose split-K scratch exceeds the fixed 4 MiB is refused before anything is
-    enqueued (the pointers below are never dereferenced)."""
+    """A shape whose split-K scratch exceeds the fixed 1 MiB (2560 x 9728, 8 rows) is refused
+    before anything is enqueued (the pointers below are never dereferenced)."""
     need_gpu()
-    desc = svq.svq_matrix(16384, 81920, 8, 0, 0x10000, 0x20000, 0x30000, 0x40000, 0x50000)
+    desc = svq.svq_matrix(2560, 9728, 8, 0, 0x10000, 0x20000, 0x30000, 0x40000, 0x50000)
     n = ctypes.c_size_t(0)
     assert svq.lib().svq_linear_gemv_workspace_size(ctypes.byref(desc), 8, ctypes.byref(n)) == svq.SVQ_OK
     assert n.value > LIMIT
