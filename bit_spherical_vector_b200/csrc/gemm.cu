@@ -9,18 +9,21 @@
 //
 //   * pass 1 (permute kernel): X_p[m][j] = X[m][perm[j]] into the workspace, so
 //     activation tiles become plain 2-D boxes for TMA;
-//   * pass 2 (this kernel, persistent, one CTA per SM, 10 warps):
-//       warp 0      TMA producer: X_p tiles [BN tokens x 64 k], 128-byte swizzle
+//   * pass 2 (this kernel, persistent, one CTA per SM, 14 warps):
+//       warp 0      TMA producer: X_p tiles [BN tokens x 64 k], 128-byte swizzle,
+//                   and bulk copies of the matching packed-code blocks
 //       warp 1      TMEM allocator and the single MMA-issuing thread:
 //                   tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
 //                   N = BN tokens, K = 16 per instruction, fp32 accumulators
 //                   in TMEM (two buffers of BN columns)
-//       warps 2..5  decoders: packed codes -> 128 x 64 bf16/fp16 weight tile in
-//                   shared memory (K-major, 128-byte swizzle), codebook from
-//                   8 shared-memory replicas; the four warps share every stage
-//                   (two of its eight subvector groups each)
-//       warps 6..9  epilogue: tcgen05.ld -> registers -> shared staging ->
-//                   coalesced stores of y (or split-K partials + fix-up)
+//       warps 2..9  decoders: packed codes (bulk-copied into shared memory by
+//                   the producer) -> 128 x 64 bf16/fp16 weight tile in shared
+//                   memory (K-major, 128-byte swizzle), codebook from
+//                   shared-memory replicas; the eight warps share every stage
+//                   (one of its eight subvector groups each)
+//       warps 10..13 epilogue: tcgen05.ld -> registers -> shared staging ->
+//                   coalesced stores of y (or of split-K partials)
+//   * pass 3 (split K only): y = sum of the partials in slice order.
 //   * weights are the A operand (swap-AB), so small token counts still map to
 //     the 128-row MMA; work units are (token tile, k-split, row tile).
 // Weight rows are placed in the A tile in the order rho = lane + 32 * r (lane
@@ -45,10 +48,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
-constexpr int kDecWarp0 = 2, kNumDec = 4;
-constexpr int kEpiWarp0 = 6, kNumEpi = 4;
+constexpr int kDecWarp0 = 2, kNumDec = 8;
+constexpr int kEpiWarp0 = kDecWarp0 + kNumDec, kNumEpi = 4;
+constexpr int kThreads = (kEpiWarp0 + kNumEpi) * 32;
 constexpr int kATileBytes = 128 * 128;           // 128 rows x 64 k x 2 bytes
+constexpr int kPTileBytes = 32 * kLaneBlockBytes; // packed codes of one 128-row x 128-column block
 constexpr int kCbBytes = 32 * 1024;               // codebook replicas
 constexpr int kStageCols = 32;                    // epilogue columns per round
 constexpr int kStgBytes = kStageCols * 128 * 4;
@@ -56,14 +60,14 @@ constexpr int kStgBytes = kStageCols * 128 * 4;
 
 template <int BN, int NS>
 __host__ __device__ constexpr uint32_t smem_bytes() {
-  return NS * kATileBytes + NS * BN * 128 + kCbBytes + kStgBytes + 1024 /* barriers */ + 1024 /* align */;
+  return NS * kATileBytes + NS * BN * 128 + NS * kPTileBytes + kCbBytes + kStgBytes + 1024 /* barriers */ +
+         1024 /* align */;
 }
 
 struct Bars {
   uint64_t full_a[8], full_b[8], empty[8], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort_flag;
-  int last_flag;
   int epi_ok;
 };
 
@@ -110,21 +114,25 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 // Decode decoder warp dw's share of one 64-column stage of one 128-row tile
-// into the swizzled A tile: subvector groups jj = 2*dw, 2*dw+1 of the stage,
-// all 128 rows (4 per lane).  The four decoder warps together fill the stage.
+// into the swizzled A tile: subvector group j = 8 * (kb & 1) + dw of the
+// packed block, all 128 rows (4 per lane).  The eight decoder warps together
+// fill the stage.  Every decoder warp runs the same instructions (the group is
+// a runtime value and the code words are read from the shared-memory copy of
+// the packed block by computed address), so the warps share instruction-cache
+// lines.
 template <bool BF16>
-__device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int kb, uint8_t* a_tile,
-                                             const uint8_t* cbs, int lane, int dw) {
+__device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int kb, const uint8_t* pk,
+                                             uint8_t* a_tile, const uint8_t* cbs, int lane, int dw) {
   const int L = tile_lanes(p.N, nt);
   if (lane >= L) return;
-  const int b = kb >> 1, h = kb & 1;
-  const uint8_t* blk = p.packed + tile_offset(p.K, nt) + (size_t)b * L * kLaneBlockBytes;
-  uint32_t w[kWords];
-#pragma unroll
-  for (int c = 0; c < kChunks; ++c) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(blk + ((size_t)c * L + lane) * 16));
-    w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-  }
+  const int j = 8 * (kb & 1) + dw;                     // subvector group within the packed block
+  // word wi of this lane's lane-block: chunk wi / 4 at ((wi / 4) * L + lane) * 16, word wi % 4
+  const uint8_t* lb = pk + lane * 16;
+  const int cstride = L * 16;
+  auto word = [&](int wi) -> uint32_t {
+    return *reinterpret_cast<const uint32_t*>(lb + (wi >> 2) * cstride + (wi & 3) * 4);
+  };
+  const uint32_t S = word(j);
   const int bd = p.b_d;
   const uint32_t imask = (1u << bd) - 1u;
   const uint32_t cmask = (1u << (10 - bd)) - 1u;
@@ -132,50 +140,38 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int k
   const uint8_t* cbq = cbs + (lane & (rep - 1)) * 16;
   const int cb_stride = rep * 16;                      // bytes per codebook entry (all replicas)
   const int n0 = nt * kTileRows + 4 * lane;
-  float sc[4], of[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    sc[r] = __half2float(__ushort_as_half(p.scale[n0 + r]));
-    of[r] = __half2float(__ushort_as_half(p.offset[n0 + r]));
-  }
+    const int v = 4 * j + r;
+    uint32_t pay;
+    if (j < 15) {
+      const int wi = 16 + v / 3;
+      pay = word(wi) >> (10 * (v - 3 * (wi - 16)));
+    } else {
+      // payloads 60..63 live in the top two bits of five payload words each
+      pay = 0;
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
-    if ((jj >> 1) != dw) continue;
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      if (hh != h) continue;
-      const int j = 8 * hh + jj;
-      const uint32_t S = w[j];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int v = 4 * j + r;
-        uint32_t pay;
-        if (v < 60) {
-          pay = w[16 + v / 3] >> (10 * (v % 3));
-        } else {
-          const int a = v - 60;
-          pay = ((w[16 + 5 * a] >> 30) << 8) | ((w[17 + 5 * a] >> 30) << 6) | ((w[18 + 5 * a] >> 30) << 4) |
-                ((w[19 + 5 * a] >> 30) << 2) | (w[20 + 5 * a] >> 30);
-        }
-        const uint32_t id = pay & imask;
-        const uint32_t code = (pay >> bd) & cmask;
-        const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
-        const float rad = __fmaf_rn(sc[r], (float)code, of[r]);
-        const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
-        uint32_t o4[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const __half2 hv = *reinterpret_cast<const __half2*>(&c4[q]);
-          const float lo = __fmul_rn(rad, __low2float(hv));
-          const float hi = __fmul_rn(rad, __high2float(hv));
-          o4[q] = pack2<BF16>(lo, hi) ^ ((S << (4 * r + q)) & 0x80008000u);
-        }
-        const int rho = lane + 32 * r;                   // A-tile row of weight row n0 + r
-        const int kc = jj;                               // 16-byte chunk within the 128-byte row
-        uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-      }
+      for (int i = 0; i < 5; ++i) pay |= (word(16 + 5 * r + i) >> 30) << (8 - 2 * i);
     }
+    const uint32_t id = pay & imask;
+    const uint32_t code = (pay >> bd) & cmask;
+    const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
+    const float sc = __half2float(__ushort_as_half(p.scale[n0 + r]));
+    const float of = __half2float(__ushort_as_half(p.offset[n0 + r]));
+    const float rad = __fmaf_rn(sc, (float)code, of);
+    const float2 rr = make_float2(rad, rad);
+    const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
+    uint32_t o4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 cf = __half22float2(*reinterpret_cast<const __half2*>(&c4[q]));
+      const float2 pr = __fmul2_rn(rr, cf);                 // binary32 products r * c
+      o4[q] = pack2<BF16>(pr.x, pr.y) ^ ((S << (4 * r + q)) & 0x80008000u);
+    }
+    const int rho = lane + 32 * r;                       // A-tile row of weight row n0 + r
+    const int kc = dw;                                   // 16-byte chunk within the 128-byte row
+    uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
   }
 }
 
@@ -186,7 +182,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* a_st = base;
   uint8_t* b_st = a_st + NS * kATileBytes;
-  uint8_t* cbs = b_st + NS * BN * 128;
+  uint8_t* p_st = b_st + NS * BN * 128;             // packed codes per stage
+  uint8_t* cbs = p_st + NS * kPTileBytes;
   float* stg = reinterpret_cast<float*>(cbs + kCbBytes);
   Bars* bars = reinterpret_cast<Bars*>(reinterpret_cast<uint8_t*>(stg) + kStgBytes);
 
@@ -206,7 +203,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
-    bars->last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
@@ -238,8 +234,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           const int s = it % NS;
           const uint32_t ph = (it / NS) & 1;
           if (it >= NS && !wait_bar(&bars->empty[s], ph ^ 1, p, bars)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars->full_b[s], BN * 128);
+          // activations (TMA tile) and the packed codes of this stage's 128-column block
+          const int L = tile_lanes(p.N, w.nt);
+          const uint32_t pbytes = (uint32_t)L * kLaneBlockBytes;
+          mbar_arrive_expect_tx(&bars->full_b[s], BN * 128 + pbytes);
           tma_load_2d(b_st + s * BN * 128, &tmap_x, &bars->full_b[s], kb * 64, w.mt * BN);
+          bulk_load(p_st + s * kPTileBytes, p.packed + tile_offset(p.K, w.nt) + (size_t)(kb >> 1) * pbytes, pbytes,
+                    &bars->full_b[s]);
         }
       }
       if (!ok) {
@@ -295,10 +296,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
         int good = 1;
-        if (it >= NS && lane == 0) good = wait_bar(&bars->empty[s], ph ^ 1, p, bars) ? 1 : 0;
+        if (lane == 0) {
+          if (it >= NS) good = wait_bar(&bars->empty[s], ph ^ 1, p, bars) ? 1 : 0;
+          if (good) good = wait_bar(&bars->full_b[s], ph, p, bars) ? 1 : 0;      // packed codes landed
+        }
         good = __shfl_sync(0xFFFFFFFFu, good, 0);
         if (!good) { ok = false; break; }
-        decode_stage<BF16>(p, w.nt, kb, a_st + s * kATileBytes, cbs, lane, d);
+        decode_stage<BF16>(p, w.nt, kb, p_st + s * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->full_a[s]);
@@ -350,39 +354,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
-      if (split) {
-        // The last CTA to finish a (row tile, token tile) sums the split-K partials in order.
-        __threadfence();
-        named_bar_sync(1, kNumEpi * 32);
-        if (threadIdx.x == kEpiWarp0 * 32) {
-          const unsigned prev = atomicAdd(&p.counters[w.mt * p.n_tiles + w.nt], 1u);
-          bars->last_flag = (prev == (unsigned)(p.S - 1));
-        }
-        named_bar_sync(1, kNumEpi * 32);
-        if (bars->last_flag) {
-          __threadfence();
-          const int tcols = min(BN, p.M - w.mt * BN);
-          for (int idx = threadIdx.x - kEpiWarp0 * 32; idx < tcols * (rows / 4); idx += kNumEpi * 32) {
-            const int i = idx / (rows / 4), n = n0 + 4 * (idx % (rows / 4));
-            const int m = w.mt * BN + i;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k < p.S; ++k) {
-              const float4 t = __ldcg(reinterpret_cast<const float4*>(p.partial + ((size_t)k * p.M + m) * p.N + n));
-              acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
-            }
-            if (p.y_f32) {
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)m * p.N + n) = acc;
-            } else {
-              uint2 pk;
-              pk.x = pack2<true>(acc.x, acc.y);
-              pk.y = pack2<true>(acc.z, acc.w);
-              *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + (size_t)m * p.N + n) = pk;
-            }
-          }
-          if (threadIdx.x == kEpiWarp0 * 32) p.counters[w.mt * p.n_tiles + w.nt] = 0u;
-        }
-        named_bar_sync(1, kNumEpi * 32);
-      }
     }
   }
 
@@ -412,6 +383,30 @@ __global__ void permute_kernel(const uint16_t* __restrict__ x, const int32_t* __
   o.z = v[4] | ((uint32_t)v[5] << 16);
   o.w = v[6] | ((uint32_t)v[7] << 16);
   *reinterpret_cast<uint4*>(xp + (size_t)m * K + j0) = o;
+}
+
+// Split-K reduction: y[m][n] = sum over slices s = 0..S-1 of partial[s][m][n]
+// (in slice order, so the result does not depend on scheduling), four outputs
+// per thread.  Separate from the GEMM so that all SMs share it.
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int S, long long MN, void* __restrict__ y,
+                                     int y_f32) {
+  const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = q; i < MN / 4; i += stride) {
+    float4 acc = __ldcs(reinterpret_cast<const float4*>(partial) + i);
+    for (int k = 1; k < S; ++k) {
+      const float4 t = __ldcs(reinterpret_cast<const float4*>(partial + (size_t)k * MN) + i);
+      acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+    }
+    if (y_f32) {
+      reinterpret_cast<float4*>(y)[i] = acc;
+    } else {
+      uint2 pk;
+      pk.x = pack2<true>(acc.x, acc.y);
+      pk.y = pack2<true>(acc.z, acc.w);
+      reinterpret_cast<uint2*>(y)[i] = pk;
+    }
+  }
 }
 
 template <int BN, int NS, bool BF16>
@@ -461,24 +456,23 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   g.n_tiles = num_tiles(N);
   const int T = g.n_tiles * g.m_tiles;
   const int KB = K / 64;
-  double best = 1e30;
+  // Split K only when the output tiles alone cannot fill the GPU: split-K
+  // partials cost S * M * N * 8 bytes of traffic and a reduction pass.
   g.S = 1;
-  for (int S = 1; S <= std::min(16, std::max(1, KB / 4)); ++S) {
-    const double waves = std::ceil((double)T * S / num_sms);
-    const double est = waves / S * (1.0 + 0.04 * (S - 1));
-    if (est < best - 1e-9) { best = est; g.S = S; }
+  if (T * 5 < num_sms * 4) {
+    double best = 1e30;
+    for (int S = 1; S <= std::min(16, std::max(1, KB / 8)); ++S) {
+      const double waves = std::ceil((double)T * S / num_sms);
+      const double est = waves / S * (1.0 + 0.04 * (S - 1));
+      if (est < best - 1e-9) { best = est; g.S = S; }
+    }
   }
   g.grid = std::min(T * g.S, num_sms);
   const size_t xp = ((size_t)M * K * 2 + 255) / 256 * 256;
   g.xp_offset = 0;
   g.partial_offset = xp;
-  size_t part = 0, cnt = 0;
-  if (g.S > 1) {
-    part = ((size_t)g.S * M * N * 4 + 255) / 256 * 256;
-    cnt = ((size_t)T * 4 + 255) / 256 * 256;
-  }
-  g.counter_offset = xp + part;
-  g.ws_bytes = xp + part + cnt;
+  const size_t part = g.S > 1 ? ((size_t)g.S * M * N * 4 + 255) / 256 * 256 : 0;
+  g.ws_bytes = xp + part;
   return g;
 }
 
@@ -513,9 +507,13 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.y = d.y;
   p.y_f32 = d.y_f32;
   p.partial = g.S > 1 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
-  p.counters = g.S > 1 ? reinterpret_cast<unsigned*>(wsb + g.counter_offset) : nullptr;
   p.status = status;
-  return d.x_bf16 ? launch_typed<true>(g.BN, tm, p, g.grid, st) : launch_typed<false>(g.BN, tm, p, g.grid, st);
+  cudaError_t e = d.x_bf16 ? launch_typed<true>(g.BN, tm, p, g.grid, st) : launch_typed<false>(g.BN, tm, p, g.grid, st);
+  if (e != cudaSuccess || g.S == 1) return e;
+  const long long mn = (long long)d.M * d.N;
+  const long long blocks = std::min<long long>((mn / 4 + 255) / 256, 148LL * 8);
+  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.partial, g.S, mn, d.y, d.y_f32);
+  return cudaGetLastError();
 }
 
 }  // namespace svq

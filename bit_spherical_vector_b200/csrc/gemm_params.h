@@ -18,13 +18,12 @@ struct GemmKParams {
   void* y;
   int y_f32;
   float* partial;       // [S][M][N] when S > 1
-  unsigned* counters;   // [m_tiles * n_tiles]
   int* status;          // device status word (bounded-wait timeouts)
 };
 
 struct GemmPlan {
   int BN, m_tiles, n_tiles, S, grid;
-  size_t xp_offset, partial_offset, counter_offset, ws_bytes;
+  size_t xp_offset, partial_offset, ws_bytes;
 };
 
 struct GemmMatDesc {

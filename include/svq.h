@@ -189,9 +189,9 @@ SVQ_API int svq_linear_gemv_noalloc(const svq_matrix* W /* host */, const uint16
  * with fp32 accumulation in tensor memory.  x: [M][K] of x_dtype (natural input
  * order).  y: [M][N] of y_dtype SVQ_F32 or SVQ_BF16.
  * Workspace (svq_linear_gemm_workspace_size): the permuted activations
- * x[:, perm] plus split-K partials and counters; as for the GEMV the counter
- * region must be zero before the first use (svq_workspace_init) and is left
- * zero by every completed call.  Error bound used by the tests:
+ * x[:, perm] plus, when K is split across CTAs, the fp32 partial sums (summed
+ * by a second kernel in split order); it carries no state between calls and
+ * needs no initialisation.  Error bound used by the tests:
  * |y - y_ref| <= 1e-2 * sum_j |W[n][j]||x[m][perm[j]]|.
  */
 SVQ_API int svq_linear_gemm_workspace_size(const svq_matrix* W /* host */, int M, size_t* bytes);
