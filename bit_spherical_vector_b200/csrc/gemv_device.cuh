@@ -78,18 +78,18 @@ __device__ __forceinline__ void load_block(uint4 (&d)[kChunks], const uint8_t* b
 
 // Shared-memory codebook with R replicas (R = 8, 4 or 2): entry e of replica q
 // sits in 16-byte slot e*R + q, lane l reads replica l % R.  With R = 8 the 8
-// lanes of an LDS.128 phase always hit 8 different bank groups; R is lowered
-// for 512- and 1024-entry codebooks to keep the table at 32 KB (two lanes of
-// a phase may then share a bank group).  The payload's index field is moved
-// to bit l0 = 4 + log2(R) (byte offset e * 16R) with one shift.
+// lanes of an LDS.128 phase always hit 8 different bank groups; cb_replicas
+// lowers R for 512- and 1024-entry codebooks to keep the table at 32 KB (two
+// lanes of a phase may then share a bank group); callers with more shared
+// memory to spare pass their own R.  The payload's index field is moved to bit
+// l0 = 4 + log2(R) (byte offset e * 16R) with one shift.
 struct CbShift {
   uint32_t l0, r1, r2, mask;
 };
 
 __device__ __forceinline__ int cb_replicas(int b_d) { return b_d <= 8 ? 8 : (b_d == 9 ? 4 : 2); }
 
-__device__ __forceinline__ CbShift cb_shift(int b_d) {
-  const int R = cb_replicas(b_d);
+__device__ __forceinline__ CbShift cb_shift(int b_d, int R) {
   const uint32_t l0 = 4u + (R == 8 ? 3u : (R == 4 ? 2u : 1u));
   CbShift c;
   c.l0 = l0;
@@ -98,6 +98,8 @@ __device__ __forceinline__ CbShift cb_shift(int b_d) {
   c.mask = ((1u << b_d) - 1u) << l0;
   return c;
 }
+
+__device__ __forceinline__ CbShift cb_shift(int b_d) { return cb_shift(b_d, cb_replicas(b_d)); }
 
 template <int MT>
 __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const unsigned char* xb,

@@ -10,16 +10,21 @@
 // (Figures 1 and 5).
 //
 // B200 mapping:
-//   * a CTA of 4 warps works on one 128-row tile of one matrix and one k-slice;
-//     the warps split the slice's blocks, each lane owns 4 complete rows, so a
-//     row's partial sum never leaves its thread in the hot loop; the warps'
-//     sums are combined once in shared memory;
+//   * one CTA per SM; each matrix of the group gets SMs in proportion to its
+//     blocks, and each CTA a contiguous range of the matrix's blocks (128-row
+//     tile x 128 columns, in storage order, crossing tile boundaries), so all
+//     SMs stream about the same number of bytes;
+//   * the warps of a CTA split its range contiguously again; each lane owns 4
+//     complete rows of the current tile, so a row's partial sum never leaves
+//     its thread in the hot loop;
 //   * packed codes stream from HBM with 16-byte coalesced loads
-//     (ld.global.nc.L1::no_allocate), one block (9 loads per lane) ahead;
-//   * the fp16 codebook sits in shared memory as 8 replicas, entry e of
-//     replica q at 16-byte slot 8e + q, and lane l reads replica l % 8: the 8
-//     lanes of each quarter-warp phase of an LDS.128 hit 8 different bank
-//     groups whatever the indices, so the random gather is conflict free;
+//     (ld.global.nc.L1::no_allocate, L2 evict-first), one block (9 loads per
+//     lane) ahead of the decode;
+//   * the fp16 codebook sits in shared memory as 8 replicas (4 for 1024
+//     entries), entry e of replica q at 16-byte slot 8e + q, and lane l reads
+//     replica l % 8: the 8 lanes of each quarter-warp phase of an LDS.128 hit 8
+//     different bank groups whatever the indices, so the random gather is
+//     conflict free;
 //   * each warp gathers x[perm] for its blocks itself, software-pipelined: the
 //     permutation of block b+2 and the activations of block b+1 are loaded
 //     while block b is decoded, into the other of two small shared-memory
@@ -27,8 +32,12 @@
 //   * signs are applied by XOR on fp16 sign bits; the eight products of a
 //     subvector are summed in fp16x2, then scaled by the radius and
 //     accumulated across subvectors in fp32;
-//   * split-K partials go to the workspace; the last CTA of a tile (found with a
-//     counter) sums them in slice order, so results are reproducible.
+//   * when a warp's range leaves a tile it parks that tile's sums in shared
+//     memory; the last warp of the CTA to leave the tile (a shared-memory
+//     counter) adds the parked sums in range order, so tiles complete while
+//     other warps still decode; a tile shared by several CTAs goes through the
+//     workspace, where the last CTA to finish it (a global counter) adds the
+//     slots in CTA order, so results are reproducible.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -43,37 +52,163 @@
 namespace svq {
 namespace {
 
-// One CTA = one 128-row tile of one matrix and one k-slice; its warps split the
-// k-slice's blocks and their partial sums are combined in shared memory.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Called by a whole warp after it parked its sums of tile t.  The last warp of
+// the CTA to do so adds the parked sums of every warp range touching t in range
+// order (rb: the CTA's W + 1 range boundaries, then each range's first tile); a tile that lies wholly in the
+// CTA's range (c0 == c1) goes to y, a tile shared by CTAs c0..c1 to its
+// workspace slot (k = c - c0), and the last CTA to deposit a slot adds all slots
+// in CTA order.  Kept out of line: it
+// runs once or twice per warp, and inlining it would cost the hot loop registers.
+template <int MT>
+__device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, const float* red, int* tcnt,
+                                             const int* rb, int ta, int c0, int c1, int npw, int y_f32,
+                                             int lane) {
+  constexpr int W = gemv_warps(MT);
+  const int N = g.N, B = g.K / kBlockCols, M = g.M;
+  const int tq0 = t * B, tq1 = tq0 + B;               // blocks of tile t
+  __threadfence_block();
+  __syncwarp();
+  // ranges r_lo..r_hi (consecutive) touch tile t; empty ranges (only when the
+  // CTA has fewer blocks than warps) touch nothing
+  int r_lo = W, r_hi = -1, touching = 0;
+#pragma unroll
+  for (int r = 0; r < W; ++r) {
+    const bool tr = rb[r] < rb[r + 1] && rb[r] < tq1 && rb[r + 1] > tq0;
+    touching += tr ? 1 : 0;
+    if (tr) { r_lo = min(r_lo, r); r_hi = r; }
+  }
+  int last = 0;
+  if (lane == 0) last = atomicAdd(&tcnt[t - ta], 1) == touching - 1;
+  if (!__shfl_sync(0xFFFFFFFFu, last, 0)) return;
+  __threadfence_block();
+  float4 v[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) v[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r = r_lo; r <= r_hi; ++r) {
+    if (rb[r] == rb[r + 1]) continue;
+    const float* src = red + ((size_t)r * npw + (t - rb[W + 1 + r])) * MT * kTileRows + 4 * lane;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const float4 u = *reinterpret_cast<const float4*>(src + m * kTileRows);
+      v[m].x += u.x; v[m].y += u.y; v[m].z += u.z; v[m].w += u.w;
+    }
+  }
+  auto write_y = [&]() {
+    const int n0 = t * kTileRows + 4 * lane;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m >= M) break;
+      const float vv[4] = {v[m].x, v[m].y, v[m].z, v[m].w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const size_t o = (size_t)m * N + n0 + r;
+        if (y_f32) reinterpret_cast<float*>(g.y)[o] = vv[r];
+        else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(vv[r]);
+      }
+    }
+  };
+  const bool in_tile = lane < tile_lanes(N, t);
+  if (c0 == c1) {                                      // the tile lies wholly in this CTA's range
+    if (in_tile) write_y();
+    return;
+  }
+  float* slots = g.partial + (size_t)t * g.kmax * MT * kTileRows + 4 * lane;
+  if (in_tile) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+      *reinterpret_cast<float4*>(slots + ((size_t)(c - c0) * MT + m) * kTileRows) = v[m];
+  }
+  // Hand-off: the counter increment has acquire-release semantics at GPU scope,
+  // so this warp's slot stores (ordered before it by __syncwarp) are visible to
+  // the CTA that sees the final count, and that CTA sees every earlier slot.
+  __syncwarp();
+  int glast = 0;
+  if (lane == 0) glast = atom_add_acq_rel_gpu(&g.counters[t], 1u) == (unsigned)(c1 - c0);
+  if (!__shfl_sync(0xFFFFFFFFu, glast, 0)) return;
+  __syncwarp();                                        // the other lanes read after lane 0's acquire
+#pragma unroll
+  for (int m = 0; m < MT; ++m) v[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (in_tile) {
+    for (int k = 0; k <= c1 - c0; ++k) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const float4 u = __ldcg(reinterpret_cast<const float4*>(slots + ((size_t)k * MT + m) * kTileRows));
+        v[m].x += u.x; v[m].y += u.y; v[m].z += u.z; v[m].w += u.w;
+      }
+    }
+    write_y();
+  }
+  if (lane == 0) g.counters[t] = 0u;
+}
+
+// One CTA = one contiguous range of one matrix's blocks.
 template <int MT>
 __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char* smem, int y_f32) {
+  constexpr int W = gemv_warps(MT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BD = g.b_d, BR = 10 - BD;
-  const int R = cb_replicas(BD);
-  const CbShift cs = cb_shift(BD);
+  const int R = gemv_cb_replicas(BD);
+  const CbShift cs = cb_shift(BD, R);
   const uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
-  const int N = g.N, K = g.K, B = K / kBlockCols, S = g.S, M = g.M;
-  const int t = c / S, s = c - t * S;
-  const int kb0 = (int)(((long long)B * s) / S), kb1 = (int)(((long long)B * (s + 1)) / S);
-  const int nbk = kb1 - kb0;
-  const int wb0 = kb0 + (nbk * warp) / kGemvWarps, wb1 = kb0 + (nbk * (warp + 1)) / kGemvWarps;
-  const int nb = wb1 - wb0;
-  const int L = tile_lanes(N, t);
-  const bool on = lane < L;
-  const int row0 = t * kTileRows + 4 * lane;
+  const int N = g.N, K = g.K, B = K / kBlockCols, M = g.M, npw = g.npw;
+  const long long T = (long long)num_tiles(N) * B, G = g.ctas;
+  // this CTA's blocks [qa, qb) and this warp's blocks [wq0, wq0 + nb)
+  const int qa = (int)(c * T / G), qb = (int)((c + 1) * T / G);
+  const int n = qb - qa;
+  // Warp ranges: range r covers [qa + n*r/W, qa + n*(r+1)/W).  Warp w takes range
+  // wr = (w % 4) * (W / 4) + w / 4, so the warps of one SM sub-partition (w, w+4,
+  // ...) hold consecutive ranges and each sub-partition issues a quarter of the
+  // CTA's blocks (ranges of 2 and 3 blocks would otherwise pile up on one).
+  auto range_begin = [&](int r) -> int { return qa + (int)((long long)n * r / W); };
+  const int wr = (warp & 3) * (W / 4) + (warp >> 2);
+  const int wq0 = range_begin(wr);
+  const int nb = range_begin(wr + 1) - wq0;
+  const int ta = qa / B, tb = (qb - 1) / B;
+
+  // The CTA's last tile is shared with the next CTA when the range ends inside
+  // it; warps whose range reaches into it walk their range backwards, so that
+  // tile's sums are complete early and its cross-CTA hand-off overlaps the rest
+  // of the decode instead of trailing it.
+  const bool first_shared = (long long)ta * B < qa, last_shared = (long long)(tb + 1) * B > qb;
+  const bool rev = nb > 0 && last_shared && (wq0 + nb - 1) / B == tb && !(first_shared && wq0 / B == ta);
+  auto q_of = [&](int b) -> int { return rev ? wq0 + nb - 1 - b : wq0 + b; };
+  const int t_first = nb > 0 ? wq0 / B : 0;           // piece p of the range holds tile t_first + p
 
   uint4* cbs = reinterpret_cast<uint4*>(smem);
   // Per warp: two x slots (double buffer) of MT rows x 128 columns fp16.
-  unsigned char* xs = smem + ((size_t)16 * R << BD) + (size_t)warp * 2 * MT * kBlockCols * 2;
-  constexpr int kXSlot = MT * kBlockCols * 2;          // bytes per slot
-  float* red = reinterpret_cast<float*>(smem + ((size_t)16 * R << BD) +
-                                        (size_t)kGemvWarps * 2 * kXSlot);   // [warps][MT][128]
+  constexpr int kXSlot = MT * kBlockCols * 2;          // bytes per x slot
+  unsigned char* xs = smem + ((size_t)16 * R << BD) + (size_t)warp * 2 * kXSlot;
+  // [W][npw][MT][128]: each warp range's sums for each tile it touches, then the
+  // W + 1 range boundaries and the W ranges' first tiles (36 ints), then one
+  // completion counter per tile of the range
+  float* red = reinterpret_cast<float*>(smem + ((size_t)16 * R << BD) + (size_t)W * 2 * kXSlot);
+  int* rbt = reinterpret_cast<int*>(red + (size_t)W * npw * MT * kTileRows);
+  int* tcnt = rbt + 36;
+  for (int i = threadIdx.x; i <= tb - ta; i += blockDim.x) tcnt[i] = 0;
+  if (threadIdx.x <= W) rbt[threadIdx.x] = range_begin(threadIdx.x);
+  if (threadIdx.x < W) rbt[W + 1 + threadIdx.x] = range_begin(threadIdx.x) / B;   // first tile of range
+  // CTAs sharing the first and the last tile of the range (interior tiles are whole)
+  auto cta_of = [&](long long q) -> int { return (int)(((q + 1) * G - 1) / T); };
+  const int c0a = cta_of((long long)ta * B), c1a = cta_of((long long)(ta + 1) * B - 1);
+  const int c0b = cta_of((long long)tb * B), c1b = cta_of((long long)(tb + 1) * B - 1);
 
-  const uint8_t* tile_base = g.packed + tile_offset(K, t);
-  const size_t blk_bytes = (size_t)L * kLaneBlockBytes;
   const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
+  auto block_ptr = [&](int q, int L) -> const uint8_t* {
+    const int t = q / B, kb = q - t * B;
+    return g.packed + tile_offset(K, t) + (size_t)kb * L * kLaneBlockBytes;
+  };
+  auto perm_ptr = [&](int q) -> const int32_t* { return g.perm + (size_t)(q % B) * kBlockCols + lane; };
+
+  int t_cur = nb > 0 ? q_of(0) / B : 0;
+  int L_cur = tile_lanes(N, t_cur);
   uint4 d0[kChunks], d1[kChunks];
-  if (on && nb > 0) load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane, pol_stream);
+  if (nb > 0 && lane < L_cur) load_block(d0, block_ptr(q_of(0), L_cur), L_cur, lane, pol_stream);
 
   // Codebook replicas: thread i fills slot i (entry i / R, replica i % R) with an
   // asynchronous global->shared copy; a warp covers consecutive slots.
@@ -83,26 +218,29 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
                  "l"(g.codebook + i / R), "l"(pol_keep)
                  : "memory");
   asm volatile("cp.async.commit_group;" ::: "memory");
-  // Radius parameters of this lane's rows and the permutation of the warp's
-  // first two blocks (all weights: independent of earlier kernels).
+  // Radius parameters of this lane's rows of the first tile and the permutation
+  // of the warp's first two blocks (all weights: independent of earlier kernels).
   float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
-  if (on) {
+  if (nb > 0 && lane < L_cur) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.scale + row0 + r, pol_keep)));
-      of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + row0 + r, pol_keep)));
+      sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.scale + t_cur * kTileRows + 4 * lane + r, pol_keep)));
+      of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + t_cur * kTileRows + 4 * lane + r, pol_keep)));
     }
   }
   // x[perm] pipeline: lane l owns columns l, l+32, l+64, l+96 of a block.  The
   // permutation of block b+2 and the activations of block b+1 are loaded while
   // block b is decoded; the activations land in the other x slot.
-  const int32_t* pw = g.perm + (size_t)wb0 * kBlockCols + lane;
   const uint16_t* xg = g.x;
   int pj_a[4], pj_b[4];
+  {
+    const int32_t* pa = perm_ptr(nb > 0 ? q_of(0) : 0);
+    const int32_t* pb = perm_ptr(nb > 1 ? q_of(1) : 0);
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    pj_a[u] = nb > 0 ? ldg_keep_i32(pw + 32 * u, pol_keep) : 0;
-    pj_b[u] = nb > 1 ? ldg_keep_i32(pw + kBlockCols + 32 * u, pol_keep) : 0;
+    for (int u = 0; u < 4; ++u) {
+      pj_a[u] = nb > 0 ? ldg_keep_i32(pa + 32 * u, pol_keep) : 0;
+      pj_b[u] = nb > 1 ? ldg_keep_i32(pb + 32 * u, pol_keep) : 0;
+    }
   }
   // The activations may be written by the previous kernel in the stream
   // (programmatic dependent launch): wait for it before reading x.
@@ -122,16 +260,17 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Radius r = offset + scale * code, written as r = scp * v + ofp with v = 1 + code * 2^-BR.
   float2 scp[2], ofp[2];
-  {
+  auto radius_pairs = [&](const float (&s4)[4], const float (&o4)[4]) {
     float sp[4], op[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      if (BR > 0) { sp[r] = sc[r] * (float)(1 << BR); op[r] = of[r] - sp[r]; }
-      else { sp[r] = 0.f; op[r] = of[r]; }
+      if (BR > 0) { sp[r] = s4[r] * (float)(1 << BR); op[r] = o4[r] - sp[r]; }
+      else { sp[r] = 0.f; op[r] = o4[r]; }
     }
     scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
     ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
-  }
+  };
+  radius_pairs(sc, of);
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
@@ -151,15 +290,48 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 #pragma unroll
         for (int u = 0; u < 4; ++u) hx[m][u] = m < M ? ldg_keep_u16(xg + (size_t)m * K + pj_b[u], pol_keep) : 0;
       if (b + 2 < nb) {
+        const int32_t* pn = perm_ptr(q_of(b + 2));
 #pragma unroll
-        for (int u = 0; u < 4; ++u) pj_b[u] = ldg_keep_i32(pw + (size_t)(b + 2) * kBlockCols + 32 * u, pol_keep);
+        for (int u = 0; u < 4; ++u) pj_b[u] = ldg_keep_i32(pn + 32 * u, pol_keep);
       }
     }
-    if (on) {
-      if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
-      process_block<MT>(d0, xs + (b & 1) * kXSlot, kBlockCols * 2, cbb, q16, cs, CODEM, scp, ofp, acc);
+    // packed codes of block b+1, and the radius parameters of its tile if it is a new one
+    int t_next = t_cur, L_next = L_cur;
+    if (b + 1 < nb) {
+      const int qn = q_of(b + 1);
+      t_next = qn / B;
+      L_next = tile_lanes(N, t_next);
+      if (lane < L_next) {
+        load_block(d1, block_ptr(qn, L_next), L_next, lane, pol_stream);
+        if (t_next != t_cur) {
 #pragma unroll
-      for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
+          for (int r = 0; r < 4; ++r) {
+            sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.scale + t_next * kTileRows + 4 * lane + r, pol_keep)));
+            of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + t_next * kTileRows + 4 * lane + r, pol_keep)));
+          }
+        }
+      }
+    }
+    if (lane < L_cur) process_block<MT>(d0, xs + (b & 1) * kXSlot, kBlockCols * 2, cbb, q16, cs, CODEM, scp, ofp, acc);
+#pragma unroll
+    for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
+    if (b + 1 == nb || t_next != t_cur) {
+      // the warp leaves tile t_cur: park its sums (lanes beyond the tile park zeros)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        float* rr = red + (((size_t)wr * npw + (t_cur - t_first)) * MT + m) * kTileRows + 4 * lane;
+        *reinterpret_cast<float4*>(rr) = make_float4(acc[0][m].x, acc[0][m].y, acc[1][m].x, acc[1][m].y);
+        acc[0][m] = make_float2(0.f, 0.f);
+        acc[1][m] = make_float2(0.f, 0.f);
+      }
+      const int c0 = t_cur == ta ? c0a : (t_cur == tb ? c0b : c);
+      const int c1 = t_cur == ta ? c1a : (t_cur == tb ? c1b : c);
+      tile_piece_done<MT>(g, c, t_cur, red, tcnt, rbt, ta, c0, c1, npw, y_f32, lane);
+      if (b + 1 < nb) {
+        t_cur = t_next;
+        L_cur = L_next;
+        radius_pairs(sc, of);
+      }
     }
     if (b + 1 < nb) {
       __syncwarp();                                   // all lanes done reading the slot about to be reused
@@ -171,69 +343,10 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       __syncwarp();
     }
   }
-
-  // Combine the warps' partial sums of the tile's 128 rows (fixed order).
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    float* rr = red + ((size_t)warp * MT + m) * kTileRows + 4 * lane;
-    *reinterpret_cast<float4*>(rr) = make_float4(acc[0][m].x, acc[0][m].y, acc[1][m].x, acc[1][m].y);
-  }
-  __syncthreads();
-  const int rows = L * 4;
-  const int nout = rows * M;
-  if (S == 1) {
-    for (int i = threadIdx.x; i < nout; i += blockDim.x) {
-      const int om = i / rows, on_i = i - om * rows;
-      float outv = 0.f;
-#pragma unroll
-      for (int w8 = 0; w8 < kGemvWarps; ++w8) outv += red[((size_t)w8 * MT + om) * kTileRows + on_i];
-      const size_t o = (size_t)om * N + t * kTileRows + on_i;
-      if (y_f32) reinterpret_cast<float*>(g.y)[o] = outv;
-      else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(outv);
-    }
-    return;
-  }
-
-  // Split-K: write this k-slice's partial, then the last CTA of the tile sums the
-  // S partials in slice order.
-  for (int i = threadIdx.x; i < nout; i += blockDim.x) {
-    const int om = i / rows, on_i = i - om * rows;
-    float outv = 0.f;
-#pragma unroll
-    for (int w8 = 0; w8 < kGemvWarps; ++w8) outv += red[((size_t)w8 * MT + om) * kTileRows + on_i];
-    g.partial[((size_t)s * M + om) * N + t * kTileRows + on_i] = outv;
-  }
-  __threadfence();
-  __syncthreads();
-  __shared__ int s_last;
-  if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(&g.counters[t], 1u);
-    s_last = (prev == (unsigned)(S - 1));
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int i = threadIdx.x; i < nout; i += blockDim.x) {
-    const int om = i / rows, n = t * kTileRows + (i - om * rows);
-    float sum = 0.f;
-    int k = 0;
-    for (; k + 8 <= S; k += 8) {
-      float v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(g.partial + ((size_t)(k + u) * M + om) * N + n);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) sum += v[u];
-    }
-    for (; k < S; ++k) sum += __ldcg(g.partial + ((size_t)k * M + om) * N + n);
-    const size_t o = (size_t)om * N + n;
-    if (y_f32) reinterpret_cast<float*>(g.y)[o] = sum;
-    else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(sum);
-  }
-  if (threadIdx.x == 0) g.counters[t] = 0u;
 }
 
 template <int MT>
-__global__ void __launch_bounds__(kGemvWarps * 32, MT <= 2 ? 4 : 2)
+__global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
 gemv_kernel(const __grid_constant__ GemvKParams P) {
   extern __shared__ __align__(1024) unsigned char smem[];
   int mi = 0;
@@ -262,7 +375,7 @@ cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStre
   // before reading x).
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kGemvWarps * 32);
+  cfg.blockDim = dim3(gemv_warps(MT) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

@@ -18,9 +18,10 @@ struct GemvKMat {
   const int32_t* perm;    // [K]
   const uint16_t* x;      // fp16 [M][K], natural input order
   void* y;                // [M][N]
-  float* partial;         // [S][M][N]
-  unsigned* counters;     // [n_rc] (one per 128-row tile)
-  int N, K, b_d, S, n_rc, cta_begin, M;
+  float* partial;         // [n_tiles][kmax][MT][128] when kmax > 1
+  unsigned* counters;     // [n_tiles]
+  int N, K, b_d, M;
+  int ctas, cta_begin, kmax, npw;
 };
 
 struct GemvKParams {

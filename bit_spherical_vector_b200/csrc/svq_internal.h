@@ -17,8 +17,15 @@ cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint
 
 // ---------------------------------------------------------------- GEMV
 constexpr int kGemvMaxMats = 8;
-constexpr int kGemvWarps = 4;            // warps per CTA; they split the k-slice of one 128-row tile
 constexpr int kGemvMaxTokens = 8;        // tokens per pass (more are split into passes)
+
+// Warps per CTA of the GEMV (one CTA per SM): fewer for wider passes, whose
+// per-lane accumulators and activations take more registers.
+__host__ __device__ constexpr int gemv_warps(int mt) { return mt <= 2 ? 12 : 8; }
+
+// Codebook replicas in the GEMV's shared memory: 8 (conflict-free gathers) up to
+// 512 entries (64 KB), 4 for 1024 entries (64 KB).
+__host__ __device__ constexpr int gemv_cb_replicas(int b_d) { return b_d <= 9 ? 8 : 4; }
 
 struct GemvMatDesc {                      // host-side description of one matrix of a launch
   int N, K, b_d;
@@ -31,13 +38,22 @@ struct GemvMatDesc {                      // host-side description of one matrix
   void* y;                               // [M][N]
 };
 
+// A matrix's blocks (128-row tile t, 128-column block kb) are numbered
+// q = t * (K / 128) + kb.  Its ctas CTAs take equal contiguous ranges of q.
+// Workspace of a GEMV launch: completion counters (one per shared-capable row
+// tile) in a fixed region at its start, then the partial sums of each matrix.
+// The counter region never moves, so counters left at zero by one call are
+// zero for the next, whatever its shapes.
+constexpr size_t kGemvCounterBytes = 64 * 1024;
+constexpr int kGemvMaxCounters = (int)(kGemvCounterBytes / sizeof(unsigned));
+
 struct GemvPlanMat {
-  int S;                                 // k-splits
-  int n_rc;                              // 128-row tiles (one CTA per tile and k-slice)
-  int ctas;                              // S * n_rc
-  size_t ws_offset;                      // gathered x, partials, counters; 256-byte aligned
-  size_t xp_bytes, part_bytes;
-  size_t ws_bytes;
+  int ctas;                              // CTA c covers q in [c*T/ctas, (c+1)*T/ctas), T = blocks
+  int n_tiles;                           // 128-row tiles
+  int kmax;                              // most CTAs sharing one tile (1: no cross-CTA sums)
+  int npw;                               // most tiles that one warp's range touches
+  int counter0;                          // first counter of this matrix's tiles
+  size_t part_offset, part_bytes;        // partial sums [n_tiles][kmax][mt][128] (kmax > 1)
 };
 
 struct GemvPlan {
@@ -45,6 +61,7 @@ struct GemvPlan {
   GemvPlanMat m[kGemvMaxMats];
   size_t ws_total;
   int total_ctas;
+  size_t smem;                           // dynamic shared memory per CTA
 };
 
 // Deterministic launch plan (k-splits, CTA counts, workspace layout) for a group.

@@ -120,11 +120,13 @@ SVQ_API int svq_dequantize(const svq_matrix* W /* host struct */, int out_dtype,
                    svq_stream_t stream);
 
 /*
- * Workspace for svq_linear_gemv / svq_linear_gemv_batched: split-K partial sums
- * and completion counters.  The counter region must be zero before the first
- * call that uses a workspace (svq_workspace_init does that); every completed
- * call leaves it zero again, so one workspace can serve a stream of calls.
- * Calls that share a workspace must not overlap on the GPU.
+ * Workspace for svq_linear_gemv / svq_linear_gemv_batched (0 bytes when no
+ * 128-row tile is split across CTAs): completion counters in its first 64 KiB,
+ * then partial sums of the split tiles.  The counters must be zero before the
+ * first call that uses a workspace (svq_workspace_init zero-fills it); every
+ * completed call leaves them zero again, so one workspace can serve a stream of
+ * calls of any shapes it is large enough for.  Calls that share a workspace
+ * must not overlap on the GPU.
  */
 SVQ_API int svq_linear_gemv_workspace_size(const svq_matrix* W /* host */, int M, size_t* bytes);
 SVQ_API int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t stream);
@@ -145,8 +147,9 @@ SVQ_API int svq_linear_gemv(const svq_matrix* W /* host */, const uint16_t* x, i
  * (e.g. the seven linears of a decoder layer, or q|k|v sharing one x):
  *   y_i = W_i x_i for i < n_mats (n_mats <= 8), each with its own M-row input.
  * mats, x, y are HOST arrays of n_mats entries (x[i], y[i] device pointers).
- * Workspace: the sum over i of svq_linear_gemv_workspace_size(mats[i], M)
- * rounded up to 256 bytes each, in order (svq_linear_gemv_batched_workspace_size).
+ * The launch shares the GPU's SMs among the matrices in proportion to their
+ * sizes, so its workspace depends on the whole group:
+ * svq_linear_gemv_batched_workspace_size.
  */
 SVQ_API int svq_linear_gemv_batched_workspace_size(const svq_matrix* mats, int n_mats, int M,
                                            size_t* bytes);
@@ -166,8 +169,8 @@ SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const ui
  * until the process exits.  It allocates nothing and calls no allocating
  * routine.
  *   - A call whose scratch need (svq_linear_gemv_workspace_size) exceeds
- *     1 MiB returns SVQ_ERR_WORKSPACE and enqueues nothing (e.g. M = 5..8 on a
- *     2560 x 9728 matrix; split such a call into passes of at most 4 rows).
+ *     1 MiB returns SVQ_ERR_WORKSPACE and enqueues nothing (e.g. M = 8 on a
+ *     32768 x 2560 matrix; split such a call into passes of fewer rows).
  *   - The first call on a device looks up the array's device address and
  *     zero-fills it on `stream`; make that first call before any stream
  *     capture.

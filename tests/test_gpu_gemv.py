@@ -121,6 +121,26 @@ def test_workspace_too_small_rejected():
     assert e.value.status == svq.SVQ_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("M", [1, 3])
+def test_grouped_ragged_tiles_inside_long_ranges(M):
+    """Two matrices of different b_d in one grouped call, one with a 4-row last tile: CTA and warp
+    ranges cross tile boundaries and end inside the ragged tile."""
+    need_gpu()
+    shapes = [(4100, 2560, 7), (388, 1152, 9)]
+    mats = [synth.make_matrix(66, i, N, K, b_d) for i, (N, K, b_d) in enumerate(shapes)]
+    xs = [synth.make_x(66, 10 + i, M, K) for i, (N, K, b_d) in enumerate(shapes)]
+    Ws = [svq.SvqWeight.from_synth(m) for m in mats]
+    nb = svq.svq_linear_gemv_batched_workspace_size(Ws, M)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+    svq.svq_workspace_init(ws)
+    ys = [torch.empty((M, m.N), dtype=torch.float32, device="cuda") for m in mats]
+    svq.svq_linear_gemv_batched(Ws, [x_f16(x) for x in xs], ys, ws)
+    torch.cuda.synchronize()
+    for m, x, y in zip(mats, xs, ys):
+        y_ref, den = oracle.linear(m, x)
+        assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
+
+
 def test_decoder_layer_grouped_full_size():
     """The seven linears of a Qwen3-4B-shaped decoder layer (batch 1) in one grouped launch,
     every output checked against the oracle."""

@@ -50,10 +50,11 @@ def test_noalloc_matches_workspace_entry_two_calls(N, K, M, b_d):
 
 
 def test_noalloc_rejects_scratch_beyond_limit():
-    """A shape whose split-K scratch exceeds the fixed 1 MiB (2560 x 9728, 8 rows) is refused
-    before anything is enqueued (the pointers below are never dereferenced)."""
+    """A shape whose split-K scratch exceeds the fixed 1 MiB (32768 x 2560, 8 rows: 256 row tiles,
+    most of them shared by two or three CTAs) is refused before anything is enqueued (the
+    pointers below are never dereferenced)."""
     need_gpu()
-    desc = svq.svq_matrix(2560, 9728, 8, 0, 0x10000, 0x20000, 0x30000, 0x40000, 0x50000)
+    desc = svq.svq_matrix(32768, 2560, 8, 0, 0x10000, 0x20000, 0x30000, 0x40000, 0x50000)
     n = ctypes.c_size_t(0)
     assert svq.lib().svq_linear_gemv_workspace_size(ctypes.byref(desc), 8, ctypes.byref(n)) == svq.SVQ_OK
     assert n.value > LIMIT
