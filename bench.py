@@ -40,6 +40,31 @@ N_LAYERS = 14
 WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 1, one grouped launch per step"
 
 
+# DRAM bytes (read + written) of one gemv_kernel<1> launch on this workload,
+# from an ncu capture (profiles/gemv_kernel_qwen3_4b_layer_batch1.md), valid
+# only while the GEMV kernel sources hash to the value it was taken with.
+GEMV_TRAFFIC_CAPTURE = {
+    "bytes": 28748544,
+    "sources": ["gemv_impl.cuh", "gemv_device.cuh", "gemv.cu", "gemv_params.h", "gemv_mt1.cu", "layout.cuh",
+                "svq_internal.h"],
+    "sha256": "a2723da305ac9f8281b4c1b12e8508fcf8e782a40103457e4ae6253675e37aa7",
+}
+
+
+def gemv_traffic():
+    """Captured DRAM bytes per launch, or None once the kernel sources changed."""
+    import hashlib
+    h = hashlib.sha256()
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_spherical_vector_b200", "csrc")
+    try:
+        for f in GEMV_TRAFFIC_CAPTURE["sources"]:
+            with open(os.path.join(src, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return GEMV_TRAFFIC_CAPTURE["bytes"] if h.hexdigest() == GEMV_TRAFFIC_CAPTURE["sha256"] else None
+
+
 def layer_bytes():
     packed = sum(N * K * 9 // 32 for _, N, K in synth.QWEN3_4B_SHAPES)
     cb = sum((1 << b) * 16 for b in synth.QWEN3_4B_SPLITS)
@@ -320,7 +345,7 @@ def run_gpu(args, world, rank, local):
                          "of packed codes rotated",
                    "hbm_pct_of_peak": 100.0 * value / world / peak, "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": gemv_traffic(),
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s",
                      "kernel": "gemv_kernel<1> (grouped, 7 matrices)",
