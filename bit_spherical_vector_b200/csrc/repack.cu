@@ -133,6 +133,10 @@ __global__ void repack_kernel(const uint8_t* __restrict__ canon, int N, int K, i
     uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
     *reinterpret_cast<uint4*>(out + chunk_offset(N, K, lb.t, lb.b, c, lb.l)) = v;
   }
+  // A GEMV launched next on the stream may start (programmatic dependent launch)
+  // as soon as every block of this grid has exited, and it reads the packed codes
+  // before it waits for this grid: make the stores visible before exiting.
+  __threadfence();
 }
 
 __device__ void load_words(const uint8_t* packed, int N, int K, const LaneBlockId& lb, uint32_t w[kWords]) {

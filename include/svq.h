@@ -138,6 +138,13 @@ SVQ_API int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t strea
  * y: [M][N] of y_dtype SVQ_F16 or SVQ_F32.  fp32 accumulation across
  * subvectors; each subvector's eight products are summed in fp16x2 pairs.
  * Error bound used by the tests: |y - y_ref| <= 1e-3 * sum_j |W[n][j]||x[m][perm[j]]|.
+ * Launch: the kernel is launched as a programmatic dependent of the previous
+ * kernel on `stream`; it reads x only after that kernel has completed, but may
+ * read the weights (packed codes, codebook, radius parameters, perm) as soon as
+ * every block of that kernel has exited.  svq_repack makes its stores visible
+ * before its blocks exit; a caller whose own kernel writes the weights right
+ * before a GEMV on the same stream must do the same (e.g. end it with
+ * __threadfence()).
  */
 SVQ_API int svq_linear_gemv(const svq_matrix* W /* host */, const uint16_t* x, int M, void* y,
                     int y_dtype, void* workspace, size_t workspace_bytes, svq_stream_t stream);
