@@ -279,6 +279,8 @@ int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int m
   p.sorted = reinterpret_cast<int*>(b + w.sorted);
   p.active = reinterpret_cast<int*>(b + w.active);
   p.n_active = reinterpret_cast<int*>(b + w.n_active);
+  p.costpre = reinterpret_cast<int*>(b + w.costpre);
+  p.mt = mt;
   p.item_out = accumulate ? reinterpret_cast<float*>(b + w.item_out) : nullptr;
   p.status = status;
   return cuda_status(svq::launch_moe(p, mt, n_out_rows, sms, (cudaStream_t)stream));

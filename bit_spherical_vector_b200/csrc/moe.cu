@@ -9,11 +9,14 @@
 //      of touched matrices and groups the item indices by matrix -- all on the
 //      device, no host round trip;
 //   2. moe_kernel (persistent): one work unit = (touched matrix, 128-row tile);
-//      the unit decodes its weights once and applies them to all of that
-//      matrix's items (up to MT tokens per pass), 8 warps splitting K, partial
-//      sums combined in shared memory; the input row of an item is either fp16
-//      x or, for a down projection, fp16(silu(gate) * up) computed on the fly
-//      from an fp32 [gate | up] row;
+//      each CTA takes a contiguous range of units, so the codebook and the
+//      input rows of a matrix are staged once for all its tiles; the unit
+//      decodes its weights once and applies them to all of that matrix's items
+//      (up to MT tokens per pass, a one-token path when a matrix has a single
+//      item), 8 warps splitting K, partial sums combined in shared memory in
+//      warp order; the input row of an item is either fp16 x or, for a down
+//      projection, fp16(silu(gate) * up) computed on the fly from an fp32
+//      [gate | up] row;
 //   3. combine_kernel (when accumulating): y[r] = sum of the items with
 //      out_row r, in item order (deterministic).
 #include <cuda_fp16.h>
@@ -32,6 +35,19 @@ namespace {
 
 constexpr int kMoeWarps = 8;
 constexpr int kRouteThreads = 1024;
+
+// Work of one row tile of a matrix with ni items, in decode passes of up to mt
+// items: a pass over the codes costs about 19 instructions per subvector-row
+// plus 6 per item of the pass width (1, 2 or mt).
+__device__ __forceinline__ int moe_matrix_cost(int ni, int mt) {
+  int cost = 0;
+  for (int c0 = 0; c0 < ni; c0 += mt) {
+    const int nc = min(mt, ni - c0);
+    const int width = nc == 1 ? 1 : (nc == 2 ? 2 : mt);
+    cost += 19 + 6 * width;
+  }
+  return cost;
+}
 
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(MoeKParams p) {
   extern __shared__ int sh[];                   // [n_mats] counts, then scan scratch
@@ -101,11 +117,90 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(MoeKParams p) {
     const int slot = atomicAdd(&p.cursor[m], 1);
     p.sorted[p.offsets[m] + slot] = i;
   }
+  // Work estimate of every touched matrix (its row tiles times the decode
+  // passes over its items) and its exclusive prefix over the active list: the
+  // MoE kernel gives each CTA an equal share of the total.
+  const int na = base_active, R = num_tiles(p.N);
+  int base_cost = 0;
+  for (int c0 = 0; c0 < na; c0 += blockDim.x) {
+    const int a = c0 + threadIdx.x;
+    int v = 0;
+    if (a < na) {
+      const int m = p.active[a];
+      v = R * moe_matrix_cost(p.offsets[m + 1] - p.offsets[m], p.mt);
+    }
+    int x = v;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+      if (lane >= o) x += y;
+    }
+    __shared__ int s_c[kRouteThreads / 32];
+    if (lane == 31) s_c[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int w = lane < (int)(blockDim.x / 32) ? s_c[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < (int)(blockDim.x / 32)) s_c[lane] = w;
+    }
+    __syncthreads();
+    const int incl = x + (wid > 0 ? s_c[wid - 1] : 0);
+    if (a < na) p.costpre[a] = base_cost + incl - v;
+    const int tot = s_c[blockDim.x / 32 - 1];
+    __syncthreads();
+    base_cost += tot;
+  }
+  if (threadIdx.x == 0) p.costpre[na] = base_cost;
 }
 
+// Input rows of items sorted[i0 .. i0 + nc) in permuted order into xs ([MT][K]
+// fp16): x_mode 0 gathers fp16 x; x_mode 1 computes fp16(silu(gate) * up) from
+// an fp32 [gate | up] row.  Each thread handles 8 consecutive columns: 8
+// independent permutation loads, then 8 (or 16) independent gathers per row.
 template <int MT>
-__device__ void moe_unit(const MoeKParams& p, const svq_matrix& W, int m, int t, unsigned char* smem,
-                         int& cb_matrix) {
+__device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W, int i0, int nc,
+                                        unsigned char* xs, uint64_t pol_keep) {
+  const int K = p.K;
+  int xrow[MT];
+#pragma unroll
+  for (int c = 0; c < MT; ++c) xrow[c] = c < nc ? p.items[p.sorted[i0 + c]].x_row : 0;
+  for (int j8 = threadIdx.x * 8; j8 < K; j8 += blockDim.x * 8) {
+    int pj[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) pj[k] = ldg_keep_i32(W.perm + j8 + k, pol_keep);
+#pragma unroll
+    for (int c = 0; c < MT; ++c) {
+      if (c >= nc) break;
+      uint32_t h[8];
+      if (p.x_mode == 0) {
+        const uint16_t* xr = reinterpret_cast<const uint16_t*>(p.x) + (size_t)xrow[c] * K;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) h[k] = ldg_keep_u16(xr + pj[k], pol_keep);
+      } else {
+        const float* xr = reinterpret_cast<const float*>(p.x) + (size_t)xrow[c] * 2 * K;
+        float gv[8], uv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { gv[k] = __ldg(xr + pj[k]); uv[k] = __ldg(xr + K + pj[k]); }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          h[k] = __half_as_ushort(__float2half_rn(gv[k] / (1.0f + expf(-gv[k])) * uv[k]));
+      }
+      *reinterpret_cast<uint4*>(xs + ((size_t)c * K + j8) * 2) =
+          make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+    }
+  }
+}
+
+// One (matrix, row tile) unit for the nc staged items: the 8 warps split the
+// tile's blocks, their sums are combined in shared memory in warp order.
+template <int NC, int MT>
+__device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& W, int t, int i0, int nc,
+                                         const unsigned char* cbs, const unsigned char* xs, float* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = p.N, K = p.K, B = K / kBlockCols;
   const int BD = W.b_d, BR = 10 - BD;
@@ -116,113 +211,124 @@ __device__ void moe_unit(const MoeKParams& p, const svq_matrix& W, int m, int t,
   const int L = tile_lanes(N, t);
   const bool on = lane < L;
   const int row0 = t * kTileRows + 4 * lane;
-  uint4* cbs = reinterpret_cast<uint4*>(smem);
-  unsigned char* xs = smem + (size_t)32 * 1024;                  // [MT][K] fp16 after the codebook
-  const int xstride = K * 2;
-  float* red = reinterpret_cast<float*>(xs + (size_t)MT * xstride);   // [8][MT][128]
   const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
-  const uint8_t* packed = reinterpret_cast<const uint8_t*>(W.packed);
-  const uint8_t* tile_base = packed + tile_offset(K, t);
+  const uint8_t* tile_base = reinterpret_cast<const uint8_t*>(W.packed) + tile_offset(K, t);
   const size_t blk_bytes = (size_t)L * kLaneBlockBytes;
-
-  __syncthreads();                                  // previous unit done with shared memory
-  if (cb_matrix != m) {
-    const uint4* cb = reinterpret_cast<const uint4*>(W.codebook);
-    for (int i = threadIdx.x; i < (RR << BD); i += blockDim.x) cbs[i] = __ldg(cb + i / RR);
-    cb_matrix = m;
-  }
-  float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
-  if (on) {
+  float2 acc[2][NC];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int q = 0; q < NC; ++q) acc[h][q] = make_float2(0.f, 0.f);
+  if (on && nb > 0) {
+    uint4 d0[kChunks], d1[kChunks];
+    load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane, pol_stream);
+    float sc[4], of[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(W.radius_scale + row0 + r, pol_keep)));
       of[r] = __half2float(__ushort_as_half(ldg_keep_u16(W.radius_offset + row0 + r, pol_keep)));
     }
-  }
-  float2 scp[2], ofp[2];
-  {
-    float sp[4], op[4];
+    float2 scp[2], ofp[2];
+    {
+      float sp[4], op[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      if (BR > 0) { sp[r] = sc[r] * (float)(1 << BR); op[r] = of[r] - sp[r]; }
-      else { sp[r] = 0.f; op[r] = of[r]; }
-    }
-    scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
-    ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
-  }
-  const int i0 = p.offsets[m], ni = p.offsets[m + 1] - i0;
-  for (int c0 = 0; c0 < ni; c0 += MT) {
-    const int nc = min(MT, ni - c0);
-    if (c0 > 0) __syncthreads();                    // previous chunk done with x and red
-    // x[perm] rows of this chunk's items (or fp16(silu(g) * u) for x_mode 1).
-    for (int e = threadIdx.x; e < MT * K; e += blockDim.x) {
-      const int c = e / K, j = e - c * K;
-      __half v = __ushort_as_half(0);
-      if (c < nc) {
-        const svq_group_item it = p.items[p.sorted[i0 + c0 + c]];
-        const int pj = ldg_keep_i32(W.perm + j, pol_keep);
-        if (p.x_mode == 0) {
-          v = __ushort_as_half(reinterpret_cast<const uint16_t*>(p.x)[(size_t)it.x_row * K + pj]);
-        } else {
-          const float* xr = reinterpret_cast<const float*>(p.x) + (size_t)it.x_row * 2 * K;
-          const float gv = xr[pj], uv = xr[K + pj];
-          v = __float2half_rn(gv / (1.0f + expf(-gv)) * uv);
-        }
+      for (int r = 0; r < 4; ++r) {
+        if (BR > 0) { sp[r] = sc[r] * (float)(1 << BR); op[r] = of[r] - sp[r]; }
+        else { sp[r] = 0.f; op[r] = of[r]; }
       }
-      reinterpret_cast<__half*>(xs)[(size_t)c * K + j] = v;
+      scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
+      ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
     }
-    __syncthreads();
-    float2 acc[2][MT];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int q = 0; q < MT; ++q) acc[h][q] = make_float2(0.f, 0.f);
-    const unsigned char* cbb = reinterpret_cast<const unsigned char*>(cbs);
     const uint32_t q16 = (uint32_t)(lane % RR) * 16;
-    if (on && nb > 0) {
-      uint4 d0[kChunks], d1[kChunks];
-      load_block(d0, tile_base + (size_t)wb0 * blk_bytes, L, lane, pol_stream);
-      for (int b = 0; b < nb; ++b) {
-        if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
-        process_block<MT>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, xstride, cbb, q16, cs, CODEM, scp, ofp,
-                          acc);
+    for (int b = 0; b < nb; ++b) {
+      if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
+      process_block<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cbs, q16, cs, CODEM, scp, ofp, acc);
 #pragma unroll
-        for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < MT; ++q) {
-      float* rr = red + ((size_t)warp * MT + q) * kTileRows + 4 * lane;
-      *reinterpret_cast<float4*>(rr) = make_float4(acc[0][q].x, acc[0][q].y, acc[1][q].x, acc[1][q].y);
-    }
-    __syncthreads();
-    const int rows = L * 4;
-    for (int e = threadIdx.x; e < rows * nc; e += blockDim.x) {
-      const int c = e / rows, nl = e - c * rows;
-      float v = 0.f;
-#pragma unroll
-      for (int w8 = 0; w8 < kMoeWarps; ++w8) v += red[((size_t)w8 * MT + c) * kTileRows + nl];
-      const int item = p.sorted[i0 + c0 + c];
-      const svq_group_item it = p.items[item];
-      const int n = t * kTileRows + nl;
-      v *= it.out_scale;
-      if (p.accumulate) p.item_out[(size_t)item * N + n] = v;
-      else p.y[(size_t)it.out_row * N + n] = v;
+      for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     }
   }
+#pragma unroll
+  for (int q = 0; q < NC; ++q) {
+    float* rr = red + ((size_t)warp * MT + q) * kTileRows + 4 * lane;
+    *reinterpret_cast<float4*>(rr) = make_float4(acc[0][q].x, acc[0][q].y, acc[1][q].x, acc[1][q].y);
+  }
+  __syncthreads();
+  const int rows = L * 4;
+  for (int e = threadIdx.x; e < rows * nc; e += blockDim.x) {
+    const int c = e / rows, nl = e - c * rows;
+    float v = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < kMoeWarps; ++w8) v += red[((size_t)w8 * MT + c) * kTileRows + nl];
+    const int item = p.sorted[i0 + c];
+    const svq_group_item it = p.items[item];
+    const int n = t * kTileRows + nl;
+    v *= it.out_scale;
+    if (p.accumulate) p.item_out[(size_t)item * N + n] = v;
+    else p.y[(size_t)it.out_row * N + n] = v;
+  }
+  __syncthreads();                                   // red is reused by the next unit
 }
 
+// Persistent: CTA c takes a contiguous range of the (touched matrix, row tile)
+// units holding an equal share of the estimated work, so consecutive units
+// mostly share a matrix and its codebook and input rows stay staged in shared
+// memory.
 template <int MT>
 __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_constant__ MoeKParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int R = num_tiles(p.N);
-  const int units = *p.n_active * R;
-  int cb_matrix = -1;
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int a = u / R, t = u - a * R;
+  const int na = *p.n_active;
+  // This CTA's share [lo, hi) of the total work; unit (a, t) (active matrix a,
+  // row tile t) starts at costpre[a] + t * (its tile cost) and belongs to the
+  // CTA whose share holds that start.
+  const long long total = p.costpre[na];
+  const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
+  int a_lo = 0, a_hi = na;                         // last a with costpre[a] <= lo
+  while (a_hi - a_lo > 1) {
+    const int mid = (a_lo + a_hi) >> 1;
+    if (p.costpre[mid] <= lo) a_lo = mid; else a_hi = mid;
+  }
+  unsigned char* cbs = smem;
+  unsigned char* xs = smem + (size_t)32 * 1024;                 // [MT][K] fp16 after the codebook
+  float* red = reinterpret_cast<float*>(xs + (size_t)MT * p.K * 2);   // [8][MT][128]
+  const uint64_t pol_keep = policy_evict_last();
+  int cb_m = -1, x_m = -1, x_c0 = -1;
+  for (int a = a_lo; a < na && p.costpre[a] < hi; ++a) {
+    const int ca = p.costpre[a], tile_cost = (p.costpre[a + 1] - ca) / R;
+    int t0 = 0;
+    if (ca < lo) t0 = (int)((lo - ca + tile_cost - 1) / tile_cost);
+    const long long t1l = (hi - ca + tile_cost - 1) / tile_cost;
+    const int t1 = t1l < R ? (int)t1l : R;
+    for (int t = t0; t < t1; ++t) {
     const int m = p.active[a];
     const svq_matrix W = p.mats[m];
-    moe_unit<MT>(p, W, m, t, smem, cb_matrix);
+    const int i0 = p.offsets[m], ni = p.offsets[m + 1] - i0;
+    for (int c0 = 0; c0 < ni; c0 += MT) {
+      const int nc = min(MT, ni - c0);
+      if (cb_m != m || x_m != m || x_c0 != c0) {
+        __syncthreads();                                 // everyone is done with the staged data
+        if (cb_m != m) {
+          const int RR = cb_replicas(W.b_d);
+          const uint32_t cb_s = (uint32_t)__cvta_generic_to_shared(cbs);
+          const uint4* cb = reinterpret_cast<const uint4*>(W.codebook);
+          for (int i = threadIdx.x; i < (RR << W.b_d); i += blockDim.x)
+            asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(cb_s + 16u * i),
+                         "l"(cb + i / RR), "l"(pol_keep)
+                         : "memory");
+          asm volatile("cp.async.commit_group;" ::: "memory");
+          cb_m = m;
+        }
+        stage_x<MT>(p, W, i0 + c0, nc, xs, pol_keep);
+        x_m = m;
+        x_c0 = c0;
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+      }
+      if (MT > 1 && nc == 1) moe_tile<1, MT>(p, W, t, i0 + c0, nc, cbs, xs, red);
+      else if (MT > 2 && nc == 2) moe_tile<2, MT>(p, W, t, i0 + c0, nc, cbs, xs, red);
+      else moe_tile<MT, MT>(p, W, t, i0 + c0, nc, cbs, xs, red);
+    }
+    }
   }
 }
 
@@ -266,6 +372,7 @@ MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate
   w.sorted = off; off += up((size_t)n_items * 4);
   w.active = off; off += up((size_t)n_mats * 4);
   w.n_active = off; off += 256;
+  w.costpre = off; off += up((size_t)(n_mats + 1) * 4);
   w.item_out = off; off += accumulate ? up((size_t)n_items * N * 4) : 0;
   w.total = off;
   return w;

@@ -23,12 +23,14 @@ struct MoeKParams {
   int* sorted;                     // item indices grouped by matrix [n_items]
   int* active;                     // touched matrices [n_mats]
   int* n_active;                   // [1]
+  int* costpre;                    // [n_mats + 1]: cost prefix over the active list (balances CTAs)
+  int mt;                          // items per decode pass of the kernel (1, 2 or 4)
   float* item_out;                 // [n_items][N] (accumulate only)
   int* status;                     // device status word
 };
 
 struct MoeWorkspace {
-  size_t offsets, cursor, sorted, active, n_active, item_out, total;
+  size_t offsets, cursor, sorted, active, n_active, costpre, item_out, total;
 };
 
 MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate);
