@@ -121,9 +121,9 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 // the packed block by computed address), so the warps share instruction-cache
 // lines.
 template <bool BF16>
-__device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int kb, const uint8_t* pk,
-                                             uint8_t* a_tile, const uint8_t* cbs, int lane, int dw) {
-  const int L = tile_lanes(p.N, nt);
+__device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const uint8_t* pk, uint8_t* a_tile,
+                                             const uint8_t* cbs, int lane, int dw, int L, const float (&sc)[4],
+                                             const float (&of)[4]) {
   if (lane >= L) return;
   const int j = 8 * (kb & 1) + dw;                     // subvector group within the packed block
   // word wi of this lane's lane-block: chunk wi / 4 at ((wi / 4) * L + lane) * 16, word wi % 4
@@ -139,7 +139,21 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int k
   const int rep = p.cb_replicas;
   const uint8_t* cbq = cbs + (lane & (rep - 1)) * 16;
   const int cb_stride = rep * 16;                      // bytes per codebook entry (all replicas)
-  const int n0 = nt * kTileRows + 4 * lane;
+  uint32_t top[4] = {0u, 0u, 0u, 0u};
+  if (j == 15) {
+    // payloads 60..63 live in the top two bits of the 20 payload words (chunks
+    // 4..8): read the five chunks whole (16-byte loads, conflict free)
+    uint32_t pw[20];
+#pragma unroll
+    for (int c = 0; c < 5; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(lb + (4 + c) * cstride);
+      pw[4 * c] = v.x; pw[4 * c + 1] = v.y; pw[4 * c + 2] = v.z; pw[4 * c + 3] = v.w;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int i = 0; i < 5; ++i) top[r] |= (pw[5 * r + i] >> 30) << (8 - 2 * i);
+  }
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int v = 4 * j + r;
@@ -148,17 +162,12 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int k
       const int wi = 16 + v / 3;
       pay = word(wi) >> (10 * (v - 3 * (wi - 16)));
     } else {
-      // payloads 60..63 live in the top two bits of five payload words each
-      pay = 0;
-#pragma unroll
-      for (int i = 0; i < 5; ++i) pay |= (word(16 + 5 * r + i) >> 30) << (8 - 2 * i);
+      pay = top[r];
     }
     const uint32_t id = pay & imask;
     const uint32_t code = (pay >> bd) & cmask;
     const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
-    const float sc = __half2float(__ushort_as_half(p.scale[n0 + r]));
-    const float of = __half2float(__ushort_as_half(p.offset[n0 + r]));
-    const float rad = __fmaf_rn(sc, (float)code, of);
+    const float rad = __fmaf_rn(sc[r], (float)code, of[r]);
     const float2 rr = make_float2(rad, rad);
     const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
     uint32_t o4[4];
@@ -168,7 +177,7 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int nt, int k
       const float2 pr = __fmul2_rn(rr, cf);                 // binary32 products r * c
       o4[q] = pack2<BF16>(pr.x, pr.y) ^ ((S << (4 * r + q)) & 0x80008000u);
     }
-    const int rho = lane + 32 * r;                       // A-tile row of weight row n0 + r
+    const int rho = lane + 32 * r;                       // A-tile row of weight row 4 * lane + r
     const int kc = dw;                                   // 16-byte chunk within the 128-byte row
     uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);
     *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
@@ -292,6 +301,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);
+      // radius parameters of this lane's 4 rows of the unit's row tile
+      const int L = tile_lanes(p.N, w.nt);
+      float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
+      if (lane < L) {
+        const int n0 = w.nt * kTileRows + 4 * lane;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          sc[r] = __half2float(__ushort_as_half(p.scale[n0 + r]));
+          of[r] = __half2float(__ushort_as_half(p.offset[n0 + r]));
+        }
+      }
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
@@ -302,7 +322,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         }
         good = __shfl_sync(0xFFFFFFFFu, good, 0);
         if (!good) { ok = false; break; }
-        decode_stage<BF16>(p, w.nt, kb, p_st + s * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d);
+        decode_stage<BF16>(p, kb, p_st + s * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d, L, sc, of);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->full_a[s]);

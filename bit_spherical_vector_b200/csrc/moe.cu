@@ -34,6 +34,7 @@ namespace svq {
 namespace {
 
 constexpr int kMoeWarps = 8;
+constexpr int kMoeCostSmem = 2048;              // cost-prefix entries kept in shared memory
 constexpr int kRouteThreads = 1024;
 
 // Work of one row tile of a matrix with ni items, in decode passes of up to mt
@@ -281,20 +282,29 @@ __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_con
   // This CTA's share [lo, hi) of the total work; unit (a, t) (active matrix a,
   // row tile t) starts at costpre[a] + t * (its tile cost) and belongs to the
   // CTA whose share holds that start.
-  const long long total = p.costpre[na];
+  unsigned char* cbs = smem;
+  unsigned char* xs = smem + (size_t)32 * 1024;                 // [MT][K] fp16 after the codebook
+  float* red = reinterpret_cast<float*>(xs + (size_t)MT * p.K * 2);   // [8][MT][128]
+  // the cost prefix, copied to shared memory when it is short (one parallel
+  // load instead of a chain of dependent global loads in the search below)
+  int* csm = reinterpret_cast<int*>(red + (size_t)kMoeWarps * MT * kTileRows);
+  const int* cpre = p.costpre;
+  if (na + 1 <= kMoeCostSmem) {
+    for (int i = threadIdx.x; i <= na; i += blockDim.x) csm[i] = p.costpre[i];
+    __syncthreads();
+    cpre = csm;
+  }
+  const long long total = cpre[na];
   const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
   int a_lo = 0, a_hi = na;                         // last a with costpre[a] <= lo
   while (a_hi - a_lo > 1) {
     const int mid = (a_lo + a_hi) >> 1;
-    if (p.costpre[mid] <= lo) a_lo = mid; else a_hi = mid;
+    if (cpre[mid] <= lo) a_lo = mid; else a_hi = mid;
   }
-  unsigned char* cbs = smem;
-  unsigned char* xs = smem + (size_t)32 * 1024;                 // [MT][K] fp16 after the codebook
-  float* red = reinterpret_cast<float*>(xs + (size_t)MT * p.K * 2);   // [8][MT][128]
   const uint64_t pol_keep = policy_evict_last();
   int cb_m = -1, x_m = -1, x_c0 = -1;
-  for (int a = a_lo; a < na && p.costpre[a] < hi; ++a) {
-    const int ca = p.costpre[a], tile_cost = (p.costpre[a + 1] - ca) / R;
+  for (int a = a_lo; a < na && cpre[a] < hi; ++a) {
+    const int ca = cpre[a], tile_cost = (cpre[a + 1] - ca) / R;
     int t0 = 0;
     if (ca < lo) t0 = (int)((lo - ca + tile_cost - 1) / tile_cost);
     const long long t1l = (hi - ca + tile_cost - 1) / tile_cost;
@@ -360,7 +370,7 @@ cudaError_t launch_moe_mt(const MoeKParams& p, int grid, size_t smem, cudaStream
 
 size_t moe_smem_bytes(int max_b_d, int K, int mt) {
   (void)max_b_d;                                   // replicas keep every codebook within 32 KB
-  return (size_t)32 * 1024 + (size_t)mt * K * 2 + (size_t)kMoeWarps * mt * kTileRows * 4;
+  return (size_t)32 * 1024 + (size_t)mt * K * 2 + (size_t)kMoeWarps * mt * kTileRows * 4 + kMoeCostSmem * 4;
 }
 
 MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate) {
