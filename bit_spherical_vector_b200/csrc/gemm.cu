@@ -11,7 +11,8 @@
 //     activation tiles become plain 2-D boxes for TMA;
 //   * pass 2 (this kernel, persistent, one CTA per SM, 14 warps):
 //       warp 0      TMA producer: X_p tiles [BN tokens x 64 k], 128-byte swizzle,
-//                   and bulk copies of the matching packed-code blocks
+//                   into the A/B ring, and bulk copies of the packed-code
+//                   blocks into a deeper ring of their own, issued ahead
 //       warp 1      TMEM allocator and the single MMA-issuing thread:
 //                   tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
 //                   N = BN tokens, K = 16 per instruction, fp32 accumulators
@@ -58,14 +59,19 @@ constexpr int kStageCols = 32;                    // epilogue columns per round
 constexpr int kStgBytes = kStageCols * 128 * 4;
 
 
+// Packed-code ring: deeper than the A/B ring so the codes of a stage are
+// requested several stages before its decode.
+template <int NS>
+__host__ __device__ constexpr int p_slots() { return NS + 3 <= 8 ? NS + 3 : 8; }
+
 template <int BN, int NS>
 __host__ __device__ constexpr uint32_t smem_bytes() {
-  return NS * kATileBytes + NS * BN * 128 + NS * kPTileBytes + kCbBytes + kStgBytes + 1024 /* barriers */ +
-         1024 /* align */;
+  return NS * kATileBytes + NS * BN * 128 + p_slots<NS>() * kPTileBytes + kCbBytes + kStgBytes +
+         1024 /* barriers */ + 1024 /* align */;
 }
 
 struct Bars {
-  uint64_t full_a[8], full_b[8], empty[8], acc_full[2], acc_empty[2], drain;
+  uint64_t full_a[8], full_b[8], empty[8], full_p[8], empty_p[8], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   int epi_ok;
@@ -191,8 +197,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* a_st = base;
   uint8_t* b_st = a_st + NS * kATileBytes;
-  uint8_t* p_st = b_st + NS * BN * 128;             // packed codes per stage
-  uint8_t* cbs = p_st + NS * kPTileBytes;
+  constexpr int NP = p_slots<NS>();
+  uint8_t* p_st = b_st + NS * BN * 128;             // packed-code ring (NP slots)
+  uint8_t* cbs = p_st + NP * kPTileBytes;
   float* stg = reinterpret_cast<float*>(cbs + kCbBytes);
   Bars* bars = reinterpret_cast<Bars*>(reinterpret_cast<uint8_t*>(stg) + kStgBytes);
 
@@ -205,6 +212,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       mbar_init(&bars->full_a[s], kNumDec);
       mbar_init(&bars->full_b[s], 1);
       mbar_init(&bars->empty[s], 1);
+    }
+    for (int s = 0; s < NP; ++s) {
+      mbar_init(&bars->full_p[s], 1);
+      mbar_init(&bars->empty_p[s], kNumDec);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->acc_full[i], 1);
@@ -233,28 +244,55 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   const int n_units = p.n_tiles * p.m_tiles * p.S;
 
   if (warp == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer: activation tiles into the A/B ring (slot
+    // freed by the MMA), packed codes into the P ring up to NP - 2 stages
+    // ahead (slot freed by the decoders)
     if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const Unit w = unit_of(p, u);
-        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-          const int s = it % NS;
-          const uint32_t ph = (it / NS) & 1;
-          if (it >= NS && !wait_bar(&bars->empty[s], ph ^ 1, p, bars)) { ok = false; break; }
-          // activations (TMA tile) and the packed codes of this stage's 128-column block
-          const int L = tile_lanes(p.N, w.nt);
-          const uint32_t pbytes = (uint32_t)L * kLaneBlockBytes;
-          mbar_arrive_expect_tx(&bars->full_b[s], BN * 128 + pbytes);
-          tma_load_2d(b_st + s * BN * 128, &tmap_x, &bars->full_b[s], kb * 64, w.mt * BN);
-          bulk_load(p_st + s * kPTileBytes, p.packed + tile_offset(p.K, w.nt) + (size_t)(kb >> 1) * pbytes, pbytes,
-                    &bars->full_b[s]);
+      struct Cursor {
+        int u, kb;
+        Unit w;
+      };
+      auto start = [&](Cursor& c) {
+        c.u = blockIdx.x;
+        if (c.u < n_units) { c.w = unit_of(p, c.u); c.kb = c.w.kb0; }
+      };
+      auto advance = [&](Cursor& c) {
+        if (++c.kb >= c.w.kb1) {
+          c.u += gridDim.x;
+          if (c.u < n_units) { c.w = unit_of(p, c.u); c.kb = c.w.kb0; }
         }
+      };
+      Cursor cb_, cp_;
+      start(cb_);
+      start(cp_);
+      int itb = 0, itp = 0;
+      bool ok = true;
+      while (ok && cb_.u < n_units) {
+        while (cp_.u < n_units && itp < itb + NP - 2) {
+          const int s = itp % NP;
+          const uint32_t ph = (itp / NP) & 1;
+          if (itp >= NP && !wait_bar(&bars->empty_p[s], ph ^ 1, p, bars)) { ok = false; break; }
+          const int L = tile_lanes(p.N, cp_.w.nt);
+          const uint32_t pbytes = (uint32_t)L * kLaneBlockBytes;
+          mbar_arrive_expect_tx(&bars->full_p[s], pbytes);
+          bulk_load(p_st + s * kPTileBytes, p.packed + tile_offset(p.K, cp_.w.nt) + (size_t)(cp_.kb >> 1) * pbytes,
+                    pbytes, &bars->full_p[s]);
+          advance(cp_);
+          ++itp;
+        }
+        if (!ok) break;
+        const int s = itb % NS;
+        const uint32_t ph = (itb / NS) & 1;
+        if (itb >= NS && !wait_bar(&bars->empty[s], ph ^ 1, p, bars)) { ok = false; break; }
+        mbar_arrive_expect_tx(&bars->full_b[s], BN * 128);
+        tma_load_2d(b_st + s * BN * 128, &tmap_x, &bars->full_b[s], cb_.kb * 64, cb_.w.mt * BN);
+        advance(cb_);
+        ++itb;
       }
       if (!ok) {
         // Let copies already issued land before the CTA exits.
-        for (int k = std::max(0, it - NS); k < it; ++k) mbar_wait(&bars->full_b[k % NS], (k / NS) & 1);
+        for (int k = std::max(0, itb - NS); k < itb; ++k) mbar_wait(&bars->full_b[k % NS], (k / NS) & 1);
+        for (int k = std::max(0, itp - NP); k < itp; ++k) mbar_wait(&bars->full_p[k % NP], (k / NP) & 1);
       }
     }
   } else if (warp == 1) {
@@ -315,17 +353,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
         const int s = it % NS;
         const uint32_t ph = (it / NS) & 1;
+        const int sp = it % NP;
+        const uint32_t php = (it / NP) & 1;
         int good = 1;
         if (lane == 0) {
-          if (it >= NS) good = wait_bar(&bars->empty[s], ph ^ 1, p, bars) ? 1 : 0;
-          if (good) good = wait_bar(&bars->full_b[s], ph, p, bars) ? 1 : 0;      // packed codes landed
+          if (it >= NS) good = wait_bar(&bars->empty[s], ph ^ 1, p, bars) ? 1 : 0;   // A slot free
+          if (good) good = wait_bar(&bars->full_p[sp], php, p, bars) ? 1 : 0;       // packed codes landed
         }
         good = __shfl_sync(0xFFFFFFFFu, good, 0);
         if (!good) { ok = false; break; }
-        decode_stage<BF16>(p, kb, p_st + s * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d, L, sc, of);
+        decode_stage<BF16>(p, kb, p_st + sp * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d, L, sc, of);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->full_a[s]);
+        if (lane == 0) {
+          mbar_arrive(&bars->full_a[s]);
+          mbar_arrive(&bars->empty_p[sp]);
+        }
       }
     }
   } else {
@@ -476,15 +519,18 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   g.n_tiles = num_tiles(N);
   const int T = g.n_tiles * g.m_tiles;
   const int KB = K / 64;
-  // Split K only when the output tiles alone cannot fill the GPU: split-K
-  // partials cost S * M * N * 8 bytes of traffic and a reduction pass.
+  // Split K when it shortens the estimated time: waves of units times the
+  // k-blocks per unit (about 1 us per 64-column k-block, set by the latency of
+  // the staging ring rather than by the MMA), plus the reduction pass over the
+  // S fp32 partials (S + 1) * M * N * 4 bytes at ~4 TB/s and one launch.
   g.S = 1;
-  if (T * 5 < num_sms * 4) {
+  {
     double best = 1e30;
     for (int S = 1; S <= std::min(16, std::max(1, KB / 8)); ++S) {
       const double waves = std::ceil((double)T * S / num_sms);
-      const double est = waves / S * (1.0 + 0.04 * (S - 1));
-      if (est < best - 1e-9) { best = est; g.S = S; }
+      double est = waves * std::ceil((double)KB / S) * 1.0e-6;
+      if (S > 1) est += (double)(S + 1) * M * N * 4.0 / 4.0e12 + 3.0e-6;
+      if (est < best * 0.97) { best = est; g.S = S; }
     }
   }
   g.grid = std::min(T * g.S, num_sms);
