@@ -9,7 +9,7 @@
 //
 //   * pass 1 (permute kernel): X_p[m][j] = X[m][perm[j]] into the workspace, so
 //     activation tiles become plain 2-D boxes for TMA;
-//   * pass 2 (this kernel, persistent, one CTA per SM, 14 warps):
+//   * pass 2 (this kernel, persistent, one CTA per SM, 22 warps):
 //       warp 0      TMA producer: X_p tiles [BN tokens x 64 k], 128-byte swizzle,
 //                   into the A/B ring, and bulk copies of the packed-code
 //                   blocks into a deeper ring of their own, issued ahead
@@ -17,12 +17,12 @@
 //                   tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
 //                   N = BN tokens, K = 16 per instruction, fp32 accumulators
 //                   in TMEM (two buffers of BN columns)
-//       warps 2..9  decoders: packed codes (bulk-copied into shared memory by
+//       warps 2..17 decoders: packed codes (bulk-copied into shared memory by
 //                   the producer) -> 128 x 64 bf16/fp16 weight tile in shared
 //                   memory (K-major, 128-byte swizzle), codebook from
-//                   shared-memory replicas; the eight warps share every stage
-//                   (one of its eight subvector groups each)
-//       warps 10..13 epilogue: tcgen05.ld -> registers -> shared staging ->
+//                   shared-memory replicas; the sixteen warps share every
+//                   stage (one of its eight subvector groups, half the rows)
+//       warps 18..21 epilogue: tcgen05.ld -> registers -> shared staging ->
 //                   coalesced stores of y (or of split-K partials)
 //   * pass 3 (split K only): y = sum of the partials in slice order.
 //   * weights are the A operand (swap-AB), so small token counts still map to
@@ -49,7 +49,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kDecWarp0 = 2, kNumDec = 8;
+constexpr int kDecWarp0 = 2, kNumDec = 16;
 constexpr int kEpiWarp0 = kDecWarp0 + kNumDec, kNumEpi = 4;
 constexpr int kThreads = (kEpiWarp0 + kNumEpi) * 32;
 constexpr int kATileBytes = 128 * 128;           // 128 rows x 64 k x 2 bytes
@@ -120,9 +120,9 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 // Decode decoder warp dw's share of one 64-column stage of one 128-row tile
-// into the swizzled A tile: subvector group j = 8 * (kb & 1) + dw of the
-// packed block, all 128 rows (4 per lane).  The eight decoder warps together
-// fill the stage.  Every decoder warp runs the same instructions (the group is
+// into the swizzled A tile: subvector group j = 8 * (kb & 1) + dw % 8 of the
+// packed block, rows 2 * (dw / 8) and 2 * (dw / 8) + 1 of every lane (64 of
+// the 128 rows).  The sixteen decoder warps together fill the stage.  Every decoder warp runs the same instructions (the group is
 // a runtime value and the code words are read from the shared-memory copy of
 // the packed block by computed address), so the warps share instruction-cache
 // lines.
@@ -131,7 +131,9 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
                                              const uint8_t* cbs, int lane, int dw, int L, const float (&sc)[4],
                                              const float (&of)[4]) {
   if (lane >= L) return;
-  const int j = 8 * (kb & 1) + dw;                     // subvector group within the packed block
+  const int kc = dw & 7;                               // 16-byte chunk within the 128-byte A row
+  const int r0 = 2 * (dw >> 3);                        // this warp decodes rows r0, r0 + 1 of each lane
+  const int j = 8 * (kb & 1) + kc;                     // subvector group within the packed block
   // word wi of this lane's lane-block: chunk wi / 4 at ((wi / 4) * L + lane) * 16, word wi % 4
   const uint8_t* lb = pk + lane * 16;
   const int cstride = L * 16;
@@ -145,7 +147,7 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
   const int rep = p.cb_replicas;
   const uint8_t* cbq = cbs + (lane & (rep - 1)) * 16;
   const int cb_stride = rep * 16;                      // bytes per codebook entry (all replicas)
-  uint32_t top[4] = {0u, 0u, 0u, 0u};
+  uint32_t top[2] = {0u, 0u};
   if (j == 15) {
     // payloads 60..63 live in the top two bits of the 20 payload words (chunks
     // 4..8): read the five chunks whole (16-byte loads, conflict free)
@@ -155,36 +157,40 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
       const uint4 v = *reinterpret_cast<const uint4*>(lb + (4 + c) * cstride);
       pw[4 * c] = v.x; pw[4 * c + 1] = v.y; pw[4 * c + 2] = v.z; pw[4 * c + 3] = v.w;
     }
+    uint32_t t4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-      for (int i = 0; i < 5; ++i) top[r] |= (pw[5 * r + i] >> 30) << (8 - 2 * i);
+      for (int i = 0; i < 5; ++i) t4[r] |= (pw[5 * r + i] >> 30) << (8 - 2 * i);
+    top[0] = r0 == 0 ? t4[0] : t4[2];
+    top[1] = r0 == 0 ? t4[1] : t4[3];
   }
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
+  for (int rr = 0; rr < 2; ++rr) {
+    const int r = r0 + rr;
     const int v = 4 * j + r;
     uint32_t pay;
     if (j < 15) {
       const int wi = 16 + v / 3;
       pay = word(wi) >> (10 * (v - 3 * (wi - 16)));
     } else {
-      pay = top[r];
+      pay = top[rr];
     }
     const uint32_t id = pay & imask;
     const uint32_t code = (pay >> bd) & cmask;
     const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
-    const float rad = __fmaf_rn(sc[r], (float)code, of[r]);
-    const float2 rr = make_float2(rad, rad);
+    const float scr = r0 == 0 ? sc[rr] : sc[2 + rr], ofr = r0 == 0 ? of[rr] : of[2 + rr];
+    const float rad = __fmaf_rn(scr, (float)code, ofr);
+    const float2 rad2 = make_float2(rad, rad);
     const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
     uint32_t o4[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 cf = __half22float2(*reinterpret_cast<const __half2*>(&c4[q]));
-      const float2 pr = __fmul2_rn(rr, cf);                 // binary32 products r * c
+      const float2 pr = __fmul2_rn(rad2, cf);               // binary32 products r * c
       o4[q] = pack2<BF16>(pr.x, pr.y) ^ ((S << (4 * r + q)) & 0x80008000u);
     }
     const int rho = lane + 32 * r;                       // A-tile row of weight row 4 * lane + r
-    const int kc = dw;                                   // 16-byte chunk within the 128-byte row
     uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);
     *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
   }
@@ -331,7 +337,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       mbar_wait(&bars->drain, 0);
     }
   } else if (warp < kEpiWarp0) {
-    // ---------------- decoders: all four warps fill every stage together, so each
+    // ---------------- decoders: all sixteen warps fill every stage together, so each
     // waits on every phase of every barrier in order (a warp that skipped
     // phases could alias an mbarrier parity).
     const int d = warp - kDecWarp0;
