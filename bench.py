@@ -253,8 +253,23 @@ def run_gpu(args, world, rank, local):
         for w in W:
             w._canon_d = None
 
-    xs = [[torch.from_numpy(x.view(np.int16)).to(dev).view(torch.float16) for x in xl] for xl in xs_host]
-    ys = [[torch.empty((1, m.N), dtype=torch.float32, device=dev) for m, _ in layer] for layer in layers]
+    # One contiguous device buffer per layer for the seven inputs and one for the
+    # seven outputs (views per matrix), so the end-to-end leg moves each step's
+    # activations with one copy each way.
+    y_len = [sum(m.N for m, _ in layer) for layer in layers]
+    xbuf = [torch.from_numpy(np.concatenate([x.reshape(-1) for x in xl]).view(np.int16)).to(dev).view(torch.float16)
+            for xl in xs_host]
+    ybuf = [torch.empty(n, dtype=torch.float32, device=dev) for n in y_len]
+
+    def views(buf, sizes, shapes):
+        out, o = [], 0
+        for n, shp in zip(sizes, shapes):
+            out.append(buf[o:o + n].view(shp))
+            o += n
+        return out
+
+    xs = [views(xbuf[L], [x.size for x in xs_host[L]], [x.shape for x in xs_host[L]]) for L in range(N_LAYERS)]
+    ys = [views(ybuf[L], [m.N for m, _ in layers[L]], [(1, m.N) for m, _ in layers[L]]) for L in range(N_LAYERS)]
     nb = max(svq.svq_linear_gemv_batched_workspace_size(W, 1) for W in Ws)
     ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
     with torch.cuda.stream(stream):
@@ -311,10 +326,10 @@ def run_gpu(args, world, rank, local):
 
     # ---- end-to-end through the public API: pinned host x -> device, layer, y -> pinned host
     e2e_steps = min(args.steps, 2000)
-    xh = [[torch.from_numpy(x.view(np.int16)).view(torch.float16).pin_memory() for x in xl] for xl in xs_host]
-    yh = [[torch.empty((1, m.N), dtype=torch.float32).pin_memory() for m, _ in layer] for layer in layers]
-    h2d = sum(x.numel() * 2 for x in xh[0])
-    d2h = sum(y.numel() * 4 for y in yh[0])
+    xh = [xb.cpu().pin_memory() for xb in xbuf]
+    yh = [torch.empty(n, dtype=torch.float32).pin_memory() for n in y_len]
+    h2d = xh[0].numel() * 2
+    d2h = yh[0].numel() * 4
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -322,11 +337,9 @@ def run_gpu(args, world, rank, local):
         e0.record(stream)
         for i in range(e2e_steps):
             L = i % N_LAYERS
-            for xd, xhh in zip(xs[L], xh[L]):
-                xd.copy_(xhh, non_blocking=True)
+            xbuf[L].copy_(xh[L], non_blocking=True)
             svq.svq_linear_gemv_batched(Ws[L], xs[L], ys[L], ws)
-            for yd, yhh in zip(ys[L], yh[L]):
-                yhh.copy_(yd, non_blocking=True)
+            yh[L].copy_(ybuf[L], non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)

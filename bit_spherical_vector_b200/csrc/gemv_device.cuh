@@ -45,6 +45,14 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
   return v;
 }
 
+__device__ __forceinline__ uint4 ldg_keep_v4(const uint4* p, uint64_t pol) {
+  uint4 v;
+  asm("ld.global.nc.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "l"(pol));
+  return v;
+}
+
 __device__ __forceinline__ int ldg_keep_i32(const int32_t* p, uint64_t pol) {
   int v;
   asm("ld.global.nc.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(v) : "l"(p), "l"(pol));

@@ -210,22 +210,26 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   uint4 d0[kChunks], d1[kChunks];
   if (nb > 0 && lane < L_cur) load_block(d0, block_ptr(q_of(0), L_cur), L_cur, lane, pol_stream);
 
-  // Codebook replicas: thread i fills slot i (entry i / R, replica i % R) with an
-  // asynchronous global->shared copy; a warp covers consecutive slots.
-  const uint32_t cb_s = (uint32_t)__cvta_generic_to_shared(cbs);
-  for (int i = threadIdx.x; i < (R << BD); i += blockDim.x)
-    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(cb_s + 16u * i),
-                 "l"(g.codebook + i / R), "l"(pol_keep)
-                 : "memory");
-  asm volatile("cp.async.commit_group;" ::: "memory");
+  // Codebook: each entry is read from global memory once (up to 4 entries per
+  // thread, loads kept in flight through the prologue) and written to its R
+  // replica slots e*R + q after the dependency wait.
+  constexpr int kCbPer = 4;                            // 1024 entries / 256+ threads
+  uint4 cbv[kCbPer];
+#pragma unroll
+  for (int k = 0; k < kCbPer; ++k) {
+    const int e = threadIdx.x + k * blockDim.x;
+    if (e < (1 << BD)) cbv[k] = ldg_keep_v4(g.codebook + e, pol_keep);
+  }
   // Radius parameters of this lane's rows of the first tile and the permutation
   // of the warp's first two blocks (all weights: independent of earlier kernels).
-  float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
+  // (kept as raw fp16 bits until they are needed, so the loads stay in flight
+  // through the rest of the prologue)
+  uint16_t sc[4] = {0, 0, 0, 0}, of[4] = {0, 0, 0, 0};
   if (nb > 0 && lane < L_cur) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.scale + t_cur * kTileRows + 4 * lane + r, pol_keep)));
-      of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + t_cur * kTileRows + 4 * lane + r, pol_keep)));
+      sc[r] = ldg_keep_u16(g.scale + t_cur * kTileRows + 4 * lane + r, pol_keep);
+      of[r] = ldg_keep_u16(g.offset + t_cur * kTileRows + 4 * lane + r, pol_keep);
     }
   }
   // x[perm] pipeline: lane l owns columns l, l+32, l+64, l+96 of a block.  The
@@ -260,18 +264,26 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // Radius r = offset + scale * code, written as r = scp * v + ofp with v = 1 + code * 2^-BR.
   float2 scp[2], ofp[2];
-  auto radius_pairs = [&](const float (&s4)[4], const float (&o4)[4]) {
+  auto radius_pairs = [&](const uint16_t (&s4)[4], const uint16_t (&o4)[4]) {
     float sp[4], op[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      if (BR > 0) { sp[r] = s4[r] * (float)(1 << BR); op[r] = o4[r] - sp[r]; }
-      else { sp[r] = 0.f; op[r] = o4[r]; }
+      const float sf = __half2float(__ushort_as_half(s4[r])), of_ = __half2float(__ushort_as_half(o4[r]));
+      if (BR > 0) { sp[r] = sf * (float)(1 << BR); op[r] = of_ - sp[r]; }
+      else { sp[r] = 0.f; op[r] = of_; }
     }
     scp[0] = make_float2(sp[0], sp[1]); scp[1] = make_float2(sp[2], sp[3]);
     ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
   };
   radius_pairs(sc, of);
-  asm volatile("cp.async.wait_all;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < kCbPer; ++k) {
+    const int e = threadIdx.x + k * blockDim.x;
+    // thread e writes its replicas in the order (q + e) % R, so the eight
+    // threads of a store phase hit eight different bank groups
+    if (e < (1 << BD))
+      for (int q = 0; q < R; ++q) cbs[e * R + ((q + e) & (R - 1))] = cbv[k];
+  }
   __syncthreads();
 
   float2 acc[2][MT];
@@ -306,8 +318,8 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
         if (t_next != t_cur) {
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            sc[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.scale + t_next * kTileRows + 4 * lane + r, pol_keep)));
-            of[r] = __half2float(__ushort_as_half(ldg_keep_u16(g.offset + t_next * kTileRows + 4 * lane + r, pol_keep)));
+            sc[r] = ldg_keep_u16(g.scale + t_next * kTileRows + 4 * lane + r, pol_keep);
+            of[r] = ldg_keep_u16(g.offset + t_next * kTileRows + 4 * lane + r, pol_keep);
           }
         }
       }
