@@ -8,9 +8,10 @@
 // (Figure 6 caption); weights are reconstructed on demand, never stored dense
 // (Figures 1 and 5).
 //
-// Work split: one CTA per SM.  Each matrix gets a number of CTAs in proportion
-// to its blocks (greedy min-max, so every SM streams about the same number of
-// packed bytes), and each of its CTAs a contiguous range of its blocks in
+// Work split: one CTA per SM.  Each matrix gets a number of CTAs by a greedy
+// min-max over the estimated time of its slowest CTA (rounds of blocks per
+// warp, plus the cross-CTA hand-off when it cannot overlap other work), and
+// each of its CTAs a contiguous range of its blocks in
 // storage order (tile-major), which may cross tile boundaries.  Inside a CTA
 // the warps split the range again contiguously.  Partial sums are combined in
 // a fixed order: warps of a CTA in shared memory (the last warp to leave a tile
@@ -71,12 +72,25 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
     int ctas[kGemvMaxMats];
     long long used = 0;
     for (int i = 0; i < n_mats; ++i) { ctas[i] = 1; ++used; }
+    // Estimated time of a matrix's slowest CTA, in block times of one warp: the
+    // rounds of blocks its warps run (range length / W, rounded up), plus about
+    // 0.6 when the CTA range holds no whole row tile besides the ones it shares
+    // at its ends, so the cross-CTA hand-off of those tiles ends the CTA instead
+    // of overlapping its other work.  Greedy min-max: the next CTA goes to the
+    // matrix with the largest estimate (ties: more blocks per CTA).
+    auto est = [&](int i) -> double {
+      const long long n = (T[i] + ctas[i] - 1) / ctas[i];
+      const double rounds = (double)((n + W - 1) / W);
+      const bool exposed = ctas[i] > 1 && 2LL * B[i] > n;
+      return rounds + (exposed ? 0.6 : 0.0);
+    };
     while (used < G) {
       int best = -1;
-      double worst = 0.0;
+      double worst = -1.0, worst_per = 0.0;
       for (int i = 0; i < n_mats; ++i) {
-        const double per = (double)T[i] / ctas[i];
-        if (ctas[i] < T[i] && per > worst) { worst = per; best = i; }
+        if (ctas[i] >= T[i]) continue;
+        const double e = est(i), per = (double)T[i] / ctas[i];
+        if (e > worst + 1e-9 || (e > worst - 1e-9 && per > worst_per)) { worst = e; worst_per = per; best = i; }
       }
       if (best < 0) break;
       ++ctas[best];
