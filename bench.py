@@ -44,10 +44,10 @@ WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 
 # from an ncu capture (profiles/gemv_kernel_qwen3_4b_layer_batch1.md), valid
 # only while the GEMV kernel sources hash to the value it was taken with.
 GEMV_TRAFFIC_CAPTURE = {
-    "bytes": 28748544,
+    "bytes": 28753664,
     "sources": ["gemv_impl.cuh", "gemv_device.cuh", "gemv.cu", "gemv_params.h", "gemv_mt1.cu", "layout.cuh",
                 "svq_internal.h"],
-    "sha256": "a2723da305ac9f8281b4c1b12e8508fcf8e782a40103457e4ae6253675e37aa7",
+    "sha256": "46932727a77a4a5fae0f7f031b5f09250576fc76b97cd7e6653c6a2d0e72e917",
 }
 
 
