@@ -264,7 +264,7 @@ int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int m
   if (!aligned(mats, 8) || !aligned(items, 4) || !aligned(y, 4) || !aligned(x, x_mode == SVQ_X_F16 ? 2 : 4))
     return SVQ_ERR_INVALID_ARG;
   const int mt = max_items_per_matrix == 1 ? 1 : (max_items_per_matrix == 2 ? 2 : 4);
-  if (svq::moe_smem_bytes(max_b_d, K, mt) > 220 * 1024) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (svq::moe_smem_bytes(max_b_d, K, mt, n_mats, n_items) > 220 * 1024) return SVQ_ERR_UNSUPPORTED_SHAPE;
   const svq::MoeWorkspace w = svq::moe_workspace_layout(n_mats, n_items, N, accumulate ? 1 : 0);
   if (!workspace || workspace_bytes < w.total || !aligned(workspace, 256)) return SVQ_ERR_WORKSPACE;
   const int sms = num_sms();
@@ -281,6 +281,7 @@ int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int m
   p.n_active = reinterpret_cast<int*>(b + w.n_active);
   p.costpre = reinterpret_cast<int*>(b + w.costpre);
   p.mt = mt;
+  p.local_route = svq::moe_local_route(n_mats, n_items) ? 1 : 0;
   p.item_out = accumulate ? reinterpret_cast<float*>(b + w.item_out) : nullptr;
   p.status = status;
   return cuda_status(svq::launch_moe(p, mt, n_out_rows, sms, (cudaStream_t)stream));

@@ -5,9 +5,11 @@
 // (Figure 2 caption) applied with its own ESG permutation (Figure 6 caption);
 // the pages evaluate an MoE model (Qwen3-30B-A3B, abstract) but describe no
 // MoE kernel.  Design here:
-//   1. route_kernel (one CTA): counts the items of every matrix, builds the list
-//      of touched matrices and groups the item indices by matrix -- all on the
-//      device, no host round trip;
+//   1. routing: count the items of every matrix, build the list of touched
+//      matrices, group the item indices by matrix and estimate each matrix's
+//      work -- on the device, no host round trip; every CTA of moe_kernel builds
+//      these tables in shared memory when they are small, else route_kernel
+//      (one CTA) writes them to the workspace first;
 //   2. moe_kernel (persistent): one work unit = (touched matrix, 128-row tile);
 //      each CTA takes a contiguous range of units, so the codebook and the
 //      input rows of a matrix are staged once for all its tiles; the unit
@@ -164,12 +166,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(MoeKParams p) {
 // an fp32 [gate | up] row.  Each thread handles 8 consecutive columns: 8
 // independent permutation loads, then 8 (or 16) independent gathers per row.
 template <int MT>
-__device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W, int i0, int nc,
-                                        unsigned char* xs, uint64_t pol_keep) {
+__device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W, const int* sorted, int i0,
+                                        int nc, unsigned char* xs, uint64_t pol_keep) {
   const int K = p.K;
   int xrow[MT];
 #pragma unroll
-  for (int c = 0; c < MT; ++c) xrow[c] = c < nc ? p.items[p.sorted[i0 + c]].x_row : 0;
+  for (int c = 0; c < MT; ++c) xrow[c] = c < nc ? p.items[sorted[i0 + c]].x_row : 0;
   for (int j8 = threadIdx.x * 8; j8 < K; j8 += blockDim.x * 8) {
     int pj[8];
 #pragma unroll
@@ -200,8 +202,9 @@ __device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W
 // One (matrix, row tile) unit for the nc staged items: the 8 warps split the
 // tile's blocks, their sums are combined in shared memory in warp order.
 template <int NC, int MT>
-__device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& W, int t, int i0, int nc,
-                                         const unsigned char* cbs, const unsigned char* xs, float* red) {
+__device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& W, const int* sorted, int t,
+                                         int i0, int nc, const unsigned char* cbs, const unsigned char* xs,
+                                         float* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = p.N, K = p.K, B = K / kBlockCols;
   const int BD = W.b_d, BR = 10 - BD;
@@ -260,7 +263,7 @@ __device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& 
     float v = 0.f;
 #pragma unroll
     for (int w8 = 0; w8 < kMoeWarps; ++w8) v += red[((size_t)w8 * MT + c) * kTileRows + nl];
-    const int item = p.sorted[i0 + c];
+    const int item = sorted[i0 + c];
     const svq_group_item it = p.items[item];
     const int n = t * kTileRows + nl;
     v *= it.out_scale;
@@ -268,6 +271,95 @@ __device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& 
     else p.y[(size_t)it.out_row * N + n] = v;
   }
   __syncthreads();                                   // red is reused by the next unit
+}
+
+// Exclusive scan of v over the CTA; *total receives the sum.  ws: 32 ints of
+// shared scratch.  Every thread of the CTA must call it.
+__device__ __forceinline__ int block_scan_excl(int v, int* ws, int* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) ws[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int w = lane < nw ? ws[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) ws[lane] = w;
+  }
+  __syncthreads();
+  const int incl = x + (wid > 0 ? ws[wid - 1] : 0);
+  *total = ws[nw - 1];
+  __syncthreads();
+  return incl - v;
+}
+
+// The routing tables of route_kernel, built by this CTA in shared memory:
+// offsets [n_mats + 1], active [n_mats], cost prefix [n_mats + 1], sorted
+// [n_items], cursors [n_mats].  Every CTA computes the same offsets, active
+// list and cost prefix; the order of the items inside a matrix may differ
+// between CTAs, which changes no result (each item is computed on its own).
+__device__ void moe_local_route(const MoeKParams& p, int* rt, int& n_active) {
+  __shared__ int s_ws[32];
+  const int nm = p.n_mats, R = num_tiles(p.N);
+  int* offs = rt;
+  int* act = offs + nm + 1;
+  int* cst = act + nm;
+  int* srt = cst + nm + 1;
+  int* cur = srt + p.n_items;
+  for (int i = threadIdx.x; i < nm; i += blockDim.x) { offs[i] = 0; cur[i] = 0; }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.n_items; i += blockDim.x) {
+    const int m = p.items[i].matrix;
+    if (m >= 0 && m < nm) atomicAdd(&offs[m], 1);
+    else if (blockIdx.x == 0) atomicExch(p.status, SVQ_ERR_INVALID_ARG);
+  }
+  __syncthreads();
+  int base = 0, base_a = 0;
+  for (int c0 = 0; c0 < nm; c0 += blockDim.x) {
+    const int m = c0 + threadIdx.x;
+    const int v = m < nm ? offs[m] : 0;
+    const int f = v > 0 ? 1 : 0;
+    int tv, tf;
+    const int ev = block_scan_excl(v, s_ws, &tv);
+    const int ef = block_scan_excl(f, s_ws, &tf);
+    if (m < nm) {
+      offs[m] = base + ev;
+      if (f) act[base_a + ef] = m;
+    }
+    base += tv;
+    base_a += tf;
+  }
+  if (threadIdx.x == 0) offs[nm] = base;
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.n_items; i += blockDim.x) {
+    const int m = p.items[i].matrix;
+    if (m < 0 || m >= nm) continue;
+    srt[offs[m] + atomicAdd(&cur[m], 1)] = i;
+  }
+  int bc = 0;
+  for (int c0 = 0; c0 < base_a; c0 += blockDim.x) {
+    const int a = c0 + threadIdx.x;
+    int v = 0;
+    if (a < base_a) {
+      const int m = act[a];
+      v = R * moe_matrix_cost(offs[m + 1] - offs[m], p.mt);
+    }
+    int tv;
+    const int ev = block_scan_excl(v, s_ws, &tv);
+    if (a < base_a) cst[a] = bc + ev;
+    bc += tv;
+  }
+  if (threadIdx.x == 0) cst[base_a] = bc;
+  __syncthreads();
+  n_active = base_a;
 }
 
 // Persistent: CTA c takes a contiguous range of the (touched matrix, row tile)
@@ -278,22 +370,36 @@ template <int MT>
 __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_constant__ MoeKParams p) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int R = num_tiles(p.N);
-  const int na = *p.n_active;
-  // This CTA's share [lo, hi) of the total work; unit (a, t) (active matrix a,
-  // row tile t) starts at costpre[a] + t * (its tile cost) and belongs to the
-  // CTA whose share holds that start.
   unsigned char* cbs = smem;
   unsigned char* xs = smem + (size_t)32 * 1024;                 // [MT][K] fp16 after the codebook
   float* red = reinterpret_cast<float*>(xs + (size_t)MT * p.K * 2);   // [8][MT][128]
-  // the cost prefix, copied to shared memory when it is short (one parallel
-  // load instead of a chain of dependent global loads in the search below)
-  int* csm = reinterpret_cast<int*>(red + (size_t)kMoeWarps * MT * kTileRows);
-  const int* cpre = p.costpre;
-  if (na + 1 <= kMoeCostSmem) {
-    for (int i = threadIdx.x; i <= na; i += blockDim.x) csm[i] = p.costpre[i];
-    __syncthreads();
-    cpre = csm;
+  int* rt = reinterpret_cast<int*>(red + (size_t)kMoeWarps * MT * kTileRows);   // routing tables
+  // Routing tables: built here (small tables) or read from route_kernel's
+  // output, whose cost prefix is then copied to shared memory when it is short
+  // (one parallel load instead of a chain of dependent loads in the search).
+  const int *offs, *act, *srt, *cpre;
+  int na;
+  if (p.local_route) {
+    moe_local_route(p, rt, na);
+    offs = rt;
+    act = offs + p.n_mats + 1;
+    cpre = act + p.n_mats;
+    srt = cpre + p.n_mats + 1;
+  } else {
+    na = *p.n_active;
+    offs = p.offsets;
+    act = p.active;
+    srt = p.sorted;
+    cpre = p.costpre;
+    if (na + 1 <= kMoeCostSmem) {
+      for (int i = threadIdx.x; i <= na; i += blockDim.x) rt[i] = p.costpre[i];
+      __syncthreads();
+      cpre = rt;
+    }
   }
+  // This CTA's share [lo, hi) of the total work; unit (a, t) (active matrix a,
+  // row tile t) starts at costpre[a] + t * (its tile cost) and belongs to the
+  // CTA whose share holds that start.
   const long long total = cpre[na];
   const long long lo = total * blockIdx.x / gridDim.x, hi = total * (blockIdx.x + 1) / gridDim.x;
   int a_lo = 0, a_hi = na;                         // last a with costpre[a] <= lo
@@ -310,9 +416,9 @@ __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_con
     const long long t1l = (hi - ca + tile_cost - 1) / tile_cost;
     const int t1 = t1l < R ? (int)t1l : R;
     for (int t = t0; t < t1; ++t) {
-    const int m = p.active[a];
+    const int m = act[a];
     const svq_matrix W = p.mats[m];
-    const int i0 = p.offsets[m], ni = p.offsets[m + 1] - i0;
+    const int i0 = offs[m], ni = offs[m + 1] - i0;
     for (int c0 = 0; c0 < ni; c0 += MT) {
       const int nc = min(MT, ni - c0);
       if (cb_m != m || x_m != m || x_c0 != c0) {
@@ -328,15 +434,15 @@ __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_con
           asm volatile("cp.async.commit_group;" ::: "memory");
           cb_m = m;
         }
-        stage_x<MT>(p, W, i0 + c0, nc, xs, pol_keep);
+        stage_x<MT>(p, W, srt, i0 + c0, nc, xs, pol_keep);
         x_m = m;
         x_c0 = c0;
         asm volatile("cp.async.wait_all;" ::: "memory");
         __syncthreads();
       }
-      if (MT > 1 && nc == 1) moe_tile<1, MT>(p, W, t, i0 + c0, nc, cbs, xs, red);
-      else if (MT > 2 && nc == 2) moe_tile<2, MT>(p, W, t, i0 + c0, nc, cbs, xs, red);
-      else moe_tile<MT, MT>(p, W, t, i0 + c0, nc, cbs, xs, red);
+      if (MT > 1 && nc == 1) moe_tile<1, MT>(p, W, srt, t, i0 + c0, nc, cbs, xs, red);
+      else if (MT > 2 && nc == 2) moe_tile<2, MT>(p, W, srt, t, i0 + c0, nc, cbs, xs, red);
+      else moe_tile<MT, MT>(p, W, srt, t, i0 + c0, nc, cbs, xs, red);
     }
     }
   }
@@ -368,9 +474,13 @@ cudaError_t launch_moe_mt(const MoeKParams& p, int grid, size_t smem, cudaStream
 
 }  // namespace
 
-size_t moe_smem_bytes(int max_b_d, int K, int mt) {
+bool moe_local_route(int n_mats, int n_items) { return n_mats <= 2048 && n_items <= 4096; }
+
+size_t moe_smem_bytes(int max_b_d, int K, int mt, int n_mats, int n_items) {
   (void)max_b_d;                                   // replicas keep every codebook within 32 KB
-  return (size_t)32 * 1024 + (size_t)mt * K * 2 + (size_t)kMoeWarps * mt * kTileRows * 4 + kMoeCostSmem * 4;
+  const size_t tables = moe_local_route(n_mats, n_items) ? (size_t)(4 * n_mats + 2 + n_items) * 4
+                                                         : (size_t)kMoeCostSmem * 4;
+  return (size_t)32 * 1024 + (size_t)mt * K * 2 + (size_t)kMoeWarps * mt * kTileRows * 4 + tables;
 }
 
 MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate) {
@@ -389,12 +499,15 @@ MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate
 }
 
 cudaError_t launch_moe(MoeKParams p, int mt, int n_out_rows, int num_sms, cudaStream_t st) {
-  const size_t route_smem = (size_t)p.n_mats * 4;
-  cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_smem);
-  if (e != cudaSuccess) return e;
-  route_kernel<<<1, kRouteThreads, route_smem, st>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t smem = moe_smem_bytes(p.max_b_d, p.K, mt);
+  cudaError_t e = cudaSuccess;
+  if (!p.local_route) {
+    const size_t route_smem = (size_t)p.n_mats * 4;
+    e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)route_smem);
+    if (e != cudaSuccess) return e;
+    route_kernel<<<1, kRouteThreads, route_smem, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t smem = moe_smem_bytes(p.max_b_d, p.K, mt, p.n_mats, p.n_items);
   switch (mt) {
     case 1: e = launch_moe_mt<1>(p, num_sms, smem, st); break;
     case 2: e = launch_moe_mt<2>(p, num_sms, smem, st); break;

@@ -25,6 +25,7 @@ struct MoeKParams {
   int* n_active;                   // [1]
   int* costpre;                    // [n_mats + 1]: cost prefix over the active list (balances CTAs)
   int mt;                          // items per decode pass of the kernel (1, 2 or 4)
+  int local_route;                 // 1: every CTA builds the routing tables in shared memory
   float* item_out;                 // [n_items][N] (accumulate only)
   int* status;                     // device status word
 };
@@ -34,7 +35,10 @@ struct MoeWorkspace {
 };
 
 MoeWorkspace moe_workspace_layout(int n_mats, int n_items, int N, int accumulate);
-size_t moe_smem_bytes(int max_b_d, int K, int mt);
+// Whether the routing tables are small enough to be built by every CTA in
+// shared memory (no separate routing kernel).
+bool moe_local_route(int n_mats, int n_items);
+size_t moe_smem_bytes(int max_b_d, int K, int mt, int n_mats, int n_items);
 cudaError_t launch_moe(MoeKParams p, int mt, int n_out_rows, int num_sms, cudaStream_t st);
 
 }  // namespace svq

@@ -90,3 +90,36 @@ def test_moe_reproducible(moe_setup):
     _, out1 = _run_moe(gu, down, x, ids, w)
     _, out2 = _run_moe(gu, down, x, ids, w)
     assert np.array_equal(out1, out2)
+
+
+def test_moe_large_routing_table_stage1(moe_setup):
+    """300 tokens x top-8: 4800 (matrix, token) items in the gate/up stage, more than the
+    kernel builds in shared memory, so the routing goes through route_kernel and the
+    workspace.  Sampled items against the oracle's single-matrix layer."""
+    experts, gu, _ = moe_setup
+    T = 300
+    x = synth.moe_x(T)
+    ids, _ = synth.moe_routing(T)
+    k = ids.shape[1]
+    dev = "cuda"
+    e = torch.from_numpy(ids.astype(np.int64)).to(dev).reshape(-1)
+    tok = torch.arange(T, device=dev).repeat_interleave(k)
+    pair = torch.arange(T * k, device=dev)
+    items = svq.item_table(torch.stack([2 * e, 2 * e + 1], 1).reshape(-1), tok.repeat_interleave(2),
+                           torch.stack([2 * pair, 2 * pair + 1], 1).reshape(-1), torch.ones(2 * T * k, device=dev))
+    y = torch.empty((2 * T * k, 768), dtype=torch.float32, device=dev)
+    ws = torch.empty(svq.svq_moe_grouped_gemv_workspace_size(len(gu), 2 * T * k, 768, False),
+                     dtype=torch.uint8, device=dev)
+    counts = np.bincount(ids.reshape(-1), minlength=len(experts))
+    svq.svq_moe_grouped_gemv(svq.descriptor_table(gu), len(gu), 768, 2048, 8, items, 2 * T * k,
+                             int(counts.max()), x_f16(x), svq.SVQ_X_F16, y, 2 * T * k, False, ws)
+    torch.cuda.synchronize()
+    assert svq.svq_get_device_status() == svq.SVQ_OK
+    y = y.cpu().numpy().reshape(T, k, 2, 768)
+    rng = np.random.default_rng(7)
+    for t in rng.choice(T, 12, replace=False):
+        s = int(rng.integers(k))
+        g, u, _ = experts[ids[t, s]]
+        for which, m in ((0, g), (1, u)):
+            y_ref, den = oracle.linear(m, x[t:t + 1])
+            assert rel_err(y[t, s, which][None], y_ref, den) <= TOL
