@@ -141,7 +141,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_init():
+def dist_init(backend: str | None = None):
+    """One process per GPU, ranks from the launcher's environment.  NCCL on GPUs;
+    `backend="gloo"` (or SVQ_BENCH_BACKEND=gloo) runs the same rank logic on CPUs."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -149,9 +151,13 @@ def dist_init():
         import torch
         import torch.distributed as dist
         from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or os.environ.get("SVQ_BENCH_BACKEND", "nccl")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timedelta(seconds=120))
     return world, rank, local
 
 
@@ -166,9 +172,15 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(world: int, units_per_rank: float, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time (units/s)."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 # --------------------------------------------------------------------------- CPU oracle (reference arm, cpu_baseline)
@@ -319,7 +331,7 @@ def run_gpu(args, world, rank, local):
         barrier(world)
     ms = ev0.elapsed_time(ev1)
     ms_max = max_over_ranks(ms, world)
-    value = world * args.steps * packed_b / (ms_max * 1e-3) / 1e9
+    value = job_rate(world, args.steps * packed_b, ms_max) / 1e9
     per_launch_s = ms * 1e-3 / args.steps
     peak, peak_kind = read_peaks()
     achieved = alg_b / per_launch_s / 1e9
@@ -344,7 +356,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = world * e2e_steps * packed_b / (e2e_ms * 1e-3) / 1e9
+    e2e_value = job_rate(world, e2e_steps * packed_b, e2e_ms) / 1e9
 
     if rank != 0:
         return 0
