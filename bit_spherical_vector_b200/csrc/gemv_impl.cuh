@@ -60,15 +60,15 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v
 
 // Called by a whole warp after it parked its sums of tile t.  The last warp of
 // the CTA to do so adds the parked sums of every warp range touching t in range
-// order (rb: the CTA's W + 1 range boundaries, then each range's first tile); a tile that lies wholly in the
-// CTA's range (c0 == c1) goes to y, a tile shared by CTAs c0..c1 to its
-// workspace slot (k = c - c0), and the last CTA to deposit a slot adds all slots
-// in CTA order.  Kept out of line: it
+// order (rb: the CTA's W + 1 range boundaries, then each range's first tile); a
+// tile that lies wholly in the CTA's range goes to y, a tile shared by CTAs
+// c0..c1 to its workspace slot (k = c - c0), and the last CTA to deposit a slot
+// adds all slots in CTA order.  Kept out of line: it
 // runs once or twice per warp, and inlining it would cost the hot loop registers.
 template <int MT>
 __device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, const float* red, int* tcnt,
-                                             const int* rb, int ta, int c0, int c1, int npw, int y_f32,
-                                             int lane) {
+                                             const int* rb, int ta, bool whole, long long G, long long T,
+                                             int npw, int y_f32, int lane) {
   constexpr int W = gemv_warps(MT);
   const int N = g.N, B = g.K / kBlockCols, M = g.M;
   const int tq0 = t * B, tq1 = tq0 + B;               // blocks of tile t
@@ -114,10 +114,13 @@ __device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, co
     }
   };
   const bool in_tile = lane < tile_lanes(N, t);
-  if (c0 == c1) {                                      // the tile lies wholly in this CTA's range
+  if (whole) {                                         // the tile lies wholly in this CTA's range
     if (in_tile) write_y();
     return;
   }
+  // CTAs c0..c1 share tile t (CTA of block q: ((q + 1) G - 1) / T)
+  const int c0 = (int)((((long long)t * B + 1) * G - 1) / T);
+  const int c1 = (int)((((long long)(t + 1) * B) * G - 1) / T);
   float* slots = g.partial + (size_t)t * g.kmax * MT * kTileRows + 4 * lane;
   if (in_tile) {
 #pragma unroll
@@ -193,10 +196,6 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   for (int i = threadIdx.x; i <= tb - ta; i += blockDim.x) tcnt[i] = 0;
   if (threadIdx.x <= W) rbt[threadIdx.x] = range_begin(threadIdx.x);
   if (threadIdx.x < W) rbt[W + 1 + threadIdx.x] = range_begin(threadIdx.x) / B;   // first tile of range
-  // CTAs sharing the first and the last tile of the range (interior tiles are whole)
-  auto cta_of = [&](long long q) -> int { return (int)(((q + 1) * G - 1) / T); };
-  const int c0a = cta_of((long long)ta * B), c1a = cta_of((long long)(ta + 1) * B - 1);
-  const int c0b = cta_of((long long)tb * B), c1b = cta_of((long long)(tb + 1) * B - 1);
 
   const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
   auto block_ptr = [&](int q, int L) -> const uint8_t* {
@@ -336,9 +335,8 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
         acc[0][m] = make_float2(0.f, 0.f);
         acc[1][m] = make_float2(0.f, 0.f);
       }
-      const int c0 = t_cur == ta ? c0a : (t_cur == tb ? c0b : c);
-      const int c1 = t_cur == ta ? c1a : (t_cur == tb ? c1b : c);
-      tile_piece_done<MT>(g, c, t_cur, red, tcnt, rbt, ta, c0, c1, npw, y_f32, lane);
+      const bool whole = t_cur * B >= qa && (t_cur + 1) * B <= qb;
+      tile_piece_done<MT>(g, c, t_cur, red, tcnt, rbt, ta, whole, G, T, npw, y_f32, lane);
       if (b + 1 < nb) {
         t_cur = t_next;
         L_cur = L_next;
