@@ -342,6 +342,7 @@ def run_gpu(args, world, rank, local):
     yh = [torch.empty(n, dtype=torch.float32).pin_memory() for n in y_len]
     h2d = xh[0].numel() * 2
     d2h = yh[0].numel() * 4
+    calls = [svq.GemvBatchCall(Ws[L], xs[L], ys[L], ws) for L in range(N_LAYERS)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
@@ -350,7 +351,7 @@ def run_gpu(args, world, rank, local):
         for i in range(e2e_steps):
             L = i % N_LAYERS
             xbuf[L].copy_(xh[L], non_blocking=True)
-            svq.svq_linear_gemv_batched(Ws[L], xs[L], ys[L], ws)
+            calls[L](stream)
             yh[L].copy_(ybuf[L], non_blocking=True)
         e1.record(stream)
     torch.cuda.synchronize()

@@ -203,6 +203,23 @@ def svq_linear_gemv_batched(Ws, xs, ys, ws=None, stream=None):
                                          _stream(stream)), "svq_linear_gemv_batched")
 
 
+class GemvBatchCall:
+    """svq_linear_gemv_batched with its arguments marshalled once, for loops that call
+    the same layers on the same buffers (one decode step after another)."""
+
+    def __init__(self, Ws, xs, ys, ws=None):
+        n = len(Ws)
+        self._keep = (list(Ws), list(xs), list(ys), ws)           # the buffers must outlive the calls
+        self._args = ((svq_matrix * n)(*[w.desc for w in Ws]), n,
+                      (ctypes.c_void_p * n)(*[x.data_ptr() for x in xs]), xs[0].shape[0],
+                      (ctypes.c_void_p * n)(*[y.data_ptr() for y in ys]), _dtype_code(ys[0].dtype), _ptr(ws),
+                      0 if ws is None else ws.numel() * ws.element_size())
+        self._fn = lib().svq_linear_gemv_batched
+
+    def __call__(self, stream=None):
+        _check(self._fn(*self._args, _stream(stream)), "svq_linear_gemv_batched")
+
+
 def svq_linear_gemv_noalloc(W: SvqWeight, x, y, stream=None):
     """svq_linear_gemv with the library's fixed internal scratch (no workspace argument)."""
     M = x.shape[0]

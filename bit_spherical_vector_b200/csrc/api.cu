@@ -3,6 +3,8 @@
 // the kernel launchers.  No entry point allocates or frees memory.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include <cstdint>
 #include <cstring>
 
@@ -58,7 +60,42 @@ int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
   }
   const int sms = num_sms();
   if (sms <= 0) return SVQ_ERR_CUDA;
+  // The plan depends only on the shapes, M and the SM count: keep the last few
+  // (a decode loop calls the same layers over and over).
+  struct Key {
+    int sms, M, n, dims[3 * svq::kGemvMaxMats];
+    bool operator==(const Key& o) const {
+      if (sms != o.sms || M != o.M || n != o.n) return false;
+      for (int i = 0; i < 3 * n; ++i)
+        if (dims[i] != o.dims[i]) return false;
+      return true;
+    }
+  };
+  struct Entry {
+    Key key;
+    svq::GemvPlan plan;
+    bool used;
+  };
+  static Entry cache[32];
+  static int next_slot = 0;
+  static std::mutex mu;
+  Key key{};
+  key.sms = sms; key.M = M; key.n = n_mats;
+  for (int i = 0; i < n_mats; ++i) {
+    key.dims[3 * i] = mats[i].N; key.dims[3 * i + 1] = mats[i].K; key.dims[3 * i + 2] = mats[i].b_d;
+  }
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (e.used && e.key == key) {
+        *plan = e.plan;
+        return SVQ_OK;
+      }
+  }
   if (!svq::plan_gemv(descs, n_mats, M, sms, plan)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[next_slot] = Entry{key, *plan, true};
+  next_slot = (next_slot + 1) % 32;
   return SVQ_OK;
 }
 

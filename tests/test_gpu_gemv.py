@@ -157,6 +157,12 @@ def test_decoder_layer_grouped_full_size():
     for (m, x), y in zip(layer, ys):
         y_ref, den = oracle.linear(m, x)
         assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL, m.name
+    # the prepared-call form of the same launch gives the same bits
+    ys2 = [torch.empty_like(y) for y in ys]
+    svq.GemvBatchCall(Ws, xs, ys2, ws)()
+    torch.cuda.synchronize()
+    for y, y2 in zip(ys, ys2):
+        assert torch.equal(y, y2)
     # the grouped launch equals the per-matrix launches
     for (m, x), W, y in zip(layer, Ws, ys):
         y1, _ = _run(W, x)
