@@ -343,16 +343,45 @@ def run_gpu(args, world, rank, local):
     h2d = xh[0].numel() * 2
     d2h = yh[0].numel() * 4
     calls = [svq.GemvBatchCall(Ws[L], xs[L], ys[L], ws) for L in range(N_LAYERS)]
+    # One CUDA graph per N_LAYERS steps: for each step, the host->device copy of
+    # its input (copy stream), the layer (compute stream, through the C ABI) and
+    # the device->host copy of its output (second copy stream), chained by
+    # events, so the copies of one step overlap the layer of the next.
+    h2d_s, d2h_s = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e, stream=stream):
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        h2d_s.wait_event(fork)
+        d2h_s.wait_event(fork)
+        ev_in = [torch.cuda.Event() for _ in range(N_LAYERS)]
+        ev_k = [torch.cuda.Event() for _ in range(N_LAYERS)]
+        ev_out = [torch.cuda.Event() for _ in range(N_LAYERS)]
+        for L in range(N_LAYERS):
+            with torch.cuda.stream(h2d_s):
+                xbuf[L].copy_(xh[L], non_blocking=True)
+                ev_in[L].record(h2d_s)
+            stream.wait_event(ev_in[L])
+            calls[L](stream)
+            ev_k[L].record(stream)
+            d2h_s.wait_event(ev_k[L])
+            with torch.cuda.stream(d2h_s):
+                yh[L].copy_(ybuf[L], non_blocking=True)
+                ev_out[L].record(d2h_s)
+        stream.wait_event(ev_in[N_LAYERS - 1])
+        stream.wait_event(ev_out[N_LAYERS - 1])
+    replays = (e2e_steps + N_LAYERS - 1) // N_LAYERS
+    e2e_steps = replays * N_LAYERS
+    with torch.cuda.stream(stream):
+        g_e2e.replay()                                   # warm-up
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         e0.record(stream)
-        for i in range(e2e_steps):
-            L = i % N_LAYERS
-            xbuf[L].copy_(xh[L], non_blocking=True)
-            calls[L](stream)
-            yh[L].copy_(ybuf[L], non_blocking=True)
+        for _ in range(replays):
+            g_e2e.replay()
         e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
