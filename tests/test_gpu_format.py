@@ -39,7 +39,7 @@ def test_repack_unpack_bit_exact(N, K, b_d):
     assert np.array_equal(c, rc)
 
 
-@pytest.mark.parametrize("b_d", [1, 3, 6, 7, 8, 9, 10])
+@pytest.mark.parametrize("b_d", range(1, 11))
 @pytest.mark.parametrize("N,K", SHAPES)
 @pytest.mark.parametrize("kind", ["f16", "bf16"])
 def test_dequantize_bit_exact(N, K, b_d, kind):

@@ -43,7 +43,7 @@ def test_gemm_small_shapes_every_output(N, K, M, b_d):
     assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
 
 
-@pytest.mark.parametrize("b_d", [1, 3, 5, 7, 10])
+@pytest.mark.parametrize("b_d", [1, 2, 3, 4, 5, 7, 10])
 def test_gemm_every_split(b_d):
     need_gpu()
     m = synth.make_matrix(71, b_d, 256, 640, b_d)

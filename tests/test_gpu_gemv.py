@@ -178,3 +178,22 @@ def test_square_8192_sweep(M):
     y, _ = _run(W, x)
     y_ref, den = oracle.linear(m, x)
     assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
+
+
+def test_lm_head_sized_matrix_sampled_rows():
+    """A vocabulary-sized matrix (151936 x 2560, b_d 8, 109 MB of codes): every CTA range spans
+    ten row tiles, most of them whole.  Sampled 4-row groups against the oracle."""
+    need_gpu()
+    N, K = 151936, 2560
+    m = synth.make_matrix(67, 0, N, K, 8)
+    x = synth.make_x(67, 0, 1, K)
+    W = svq.SvqWeight.from_synth(m)
+    y, _ = _run(W, x)
+    y = y.cpu().numpy()
+    rng = np.random.default_rng(3)
+    for r0 in list(rng.choice(N // 4, 24, replace=False) * 4) + [0, N - 4]:
+        sub = synth.SvqMatrix(4, K, 8, np.ascontiguousarray(m.canonical[r0:r0 + 4]), m.codebook,
+                              np.ascontiguousarray(m.scale[r0:r0 + 4]), np.ascontiguousarray(m.offset[r0:r0 + 4]),
+                              m.perm)
+        y_ref, den = oracle.linear(sub, x)
+        assert rel_err(y[:, r0:r0 + 4], y_ref, den) <= TOL
