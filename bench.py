@@ -44,10 +44,10 @@ WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 
 # from an ncu capture (profiles/gemv_kernel_qwen3_4b_layer_batch1.md), valid
 # only while the GEMV kernel sources hash to the value it was taken with.
 GEMV_TRAFFIC_CAPTURE = {
-    "bytes": 28753664,
+    "bytes": 28751872,
     "sources": ["gemv_impl.cuh", "gemv_device.cuh", "gemv.cu", "gemv_params.h", "gemv_mt1.cu", "layout.cuh",
                 "svq_internal.h"],
-    "sha256": "46932727a77a4a5fae0f7f031b5f09250576fc76b97cd7e6653c6a2d0e72e917",
+    "sha256": "4c02e3f2c890c4536da10cdc63d36c85d42dac35afd232769060042620287103",
 }
 
 
