@@ -225,9 +225,12 @@ SVQ_API int svq_linear_gemm(const svq_matrix* W /* host */, const uint16_t* x, i
  * mats: DEVICE array of n_mats descriptors (same layout as svq_matrix), every
  *   one N x K with b_d <= max_b_d; the host cannot read them, so the caller
  *   guarantees them (the host checks N, K, max_b_d and the pointers it sees).
- * items: DEVICE array of n_items.  Each touched matrix is decoded once per call
- *   and applied to all of its items (up to max_items_per_matrix, a bound the
- *   caller guarantees; it selects how many rows share one decode pass).
+ * items: DEVICE array of n_items.  Each touched matrix is decoded once per
+ *   pass and applied to up to P of its items in that pass, P = 1, 2 or 4 chosen
+ *   from max_items_per_matrix (1 -> 1, 2 -> 2, else 4); a matrix with more
+ *   items takes more passes.  The grouping of items by matrix (routing) is done
+ *   on the device, by every CTA in shared memory for up to 2048 matrices and
+ *   4096 items, else by a separate routing kernel through the workspace.
  * y: fp32 [n_out_rows][N].  Workspace: svq_moe_grouped_gemv_workspace_size.
  * Tolerance used by the tests: as svq_linear_gemv (1e-3 of sum |W| |in|).
  */
