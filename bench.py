@@ -44,10 +44,10 @@ WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 
 # from an ncu capture (profiles/gemv_kernel_qwen3_4b_layer_batch1.md), valid
 # only while the GEMV kernel sources hash to the value it was taken with.
 GEMV_TRAFFIC_CAPTURE = {
-    "bytes": 28751872,
+    "bytes": 28770560,
     "sources": ["gemv_impl.cuh", "gemv_device.cuh", "gemv.cu", "gemv_params.h", "gemv_mt1.cu", "layout.cuh",
                 "svq_internal.h"],
-    "sha256": "4c02e3f2c890c4536da10cdc63d36c85d42dac35afd232769060042620287103",
+    "sha256": "4c5dfd41210b558978f66b0c136fc777b93789497f36272b31c755fa89b2ff05",
 }
 
 

@@ -128,13 +128,18 @@ def svq_unpack_fields(packed, N: int, K: int, b_d: int, signs, idx, code, stream
 
 class SvqWeight:
     """Device-resident SVQ matrix (packed codes, codebook, radius params, perm) and its
-    C descriptor.  Built from canonical host arrays by ``from_canonical``."""
+    C descriptor.  Built from canonical host arrays by ``from_canonical``.  ``perm``
+    None means x is supplied already in the stored column order."""
 
     def __init__(self, N, K, b_d, packed, codebook, scale, offset, perm):
         self.N, self.K, self.b_d = N, K, b_d
         self.packed, self.codebook, self.scale, self.offset, self.perm = packed, codebook, scale, offset, perm
         self.desc = svq_matrix(N, K, b_d, 0, packed.data_ptr(), codebook.data_ptr(), scale.data_ptr(),
-                               offset.data_ptr(), perm.data_ptr())
+                               offset.data_ptr(), 0 if perm is None else perm.data_ptr())
+
+    def without_perm(self):
+        """The same device arrays with perm NULL: its calls take x in stored column order."""
+        return SvqWeight(self.N, self.K, self.b_d, self.packed, self.codebook, self.scale, self.offset, None)
 
     @classmethod
     def from_canonical(cls, N, K, b_d, canonical, codebook, scale, offset, perm, device="cuda", stream=None):

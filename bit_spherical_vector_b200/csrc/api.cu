@@ -33,10 +33,10 @@ int check_matrix(const svq_matrix* W) {
   if (!W) return SVQ_ERR_INVALID_ARG;
   if (W->b_d < 1 || W->b_d > 10) return SVQ_ERR_UNSUPPORTED_SHAPE;
   if (W->K % 8 != 0 || !svq::layout_supported(W->N, W->K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
-  if (!W->packed || !W->codebook || !W->radius_scale || !W->radius_offset || !W->perm)
+  if (!W->packed || !W->codebook || !W->radius_scale || !W->radius_offset)
     return SVQ_ERR_INVALID_ARG;
   if (!aligned(W->packed, 16) || !aligned(W->codebook, 16) || !aligned(W->radius_scale, 2) ||
-      !aligned(W->radius_offset, 2) || !aligned(W->perm, 4))
+      !aligned(W->radius_offset, 2) || (W->perm && !aligned(W->perm, 4)))
     return SVQ_ERR_INVALID_ARG;
   return SVQ_OK;
 }
@@ -271,6 +271,7 @@ int svq_linear_gemm(const svq_matrix* W, const uint16_t* x, int x_dtype, int M, 
   if (x_dtype != SVQ_BF16 && x_dtype != SVQ_F16) return SVQ_ERR_INVALID_ARG;
   if (y_dtype != SVQ_BF16 && y_dtype != SVQ_F32) return SVQ_ERR_INVALID_ARG;
   if (!aligned(x, 2) || !aligned(y, 16)) return SVQ_ERR_INVALID_ARG;
+  if (!W->perm && !aligned(x, 16)) return SVQ_ERR_INVALID_ARG;     // read directly by TMA
   const int sms = num_sms();
   if (sms <= 0) return SVQ_ERR_CUDA;
   const svq::GemmPlan g = svq::plan_gemm(W->N, W->K, M, sms);

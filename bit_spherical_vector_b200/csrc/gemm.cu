@@ -550,12 +550,16 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
 
 cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* status, cudaStream_t st) {
   uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
-  uint16_t* xp = reinterpret_cast<uint16_t*>(wsb + g.xp_offset);
-  {
+  // X[:, perm] into the workspace, or X itself when it is already in stored
+  // column order (perm NULL)
+  const uint16_t* xp = d.x;
+  if (d.perm) {
+    uint16_t* xw = reinterpret_cast<uint16_t*>(wsb + g.xp_offset);
     const long long work = (long long)d.M * (d.K / 8);
-    permute_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(d.x, d.perm, d.M, d.K, xp);
+    permute_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(d.x, d.perm, d.M, d.K, xw);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    xp = xw;
   }
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -564,7 +568,8 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   const cuuint64_t strides[1] = {(cuuint64_t)d.K * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)g.BN};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(&tm, d.x_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xp,
+  const CUresult r = enc(&tm, d.x_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         const_cast<uint16_t*>(xp),
                          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;

@@ -150,8 +150,10 @@ __device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, co
   if (lane == 0) g.counters[t] = 0u;
 }
 
-// One CTA = one contiguous range of one matrix's blocks.
-template <int MT>
+// One CTA = one contiguous range of one matrix's blocks.  kPerm: the matrix has
+// a permutation (x is gathered through it); without one, x is already in stored
+// column order and lane l reads columns l, l+32, l+64, l+96 of each block.
+template <int MT, bool kPerm>
 __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char* smem, int y_f32) {
   constexpr int W = gemv_warps(MT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -203,6 +205,10 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
     return g.packed + tile_offset(K, t) + (size_t)kb * L * kLaneBlockBytes;
   };
   auto perm_ptr = [&](int q) -> const int32_t* { return g.perm + (size_t)(q % B) * kBlockCols + lane; };
+  auto cols = [&](int q, int (&pj)[4]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) pj[u] = (q % B) * kBlockCols + lane + 32 * u;
+  };
 
   int t_cur = nb > 0 ? q_of(0) / B : 0;
   int L_cur = tile_lanes(N, t_cur);
@@ -236,7 +242,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   // block b is decoded; the activations land in the other x slot.
   const uint16_t* xg = g.x;
   int pj_a[4], pj_b[4];
-  {
+  if constexpr (kPerm) {
     const int32_t* pa = perm_ptr(nb > 0 ? q_of(0) : 0);
     const int32_t* pb = perm_ptr(nb > 1 ? q_of(1) : 0);
 #pragma unroll
@@ -244,6 +250,9 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       pj_a[u] = nb > 0 ? ldg_keep_i32(pa + 32 * u, pol_keep) : 0;
       pj_b[u] = nb > 1 ? ldg_keep_i32(pb + 32 * u, pol_keep) : 0;
     }
+  } else {
+    cols(nb > 0 ? q_of(0) : 0, pj_a);
+    cols(nb > 1 ? q_of(1) : 0, pj_b);
   }
   // The activations may be written by the previous kernel in the stream
   // (programmatic dependent launch): wait for it before reading x.
@@ -301,9 +310,13 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 #pragma unroll
         for (int u = 0; u < 4; ++u) hx[m][u] = m < M ? ldg_keep_u16(xg + (size_t)m * K + pj_b[u], pol_keep) : 0;
       if (b + 2 < nb) {
-        const int32_t* pn = perm_ptr(q_of(b + 2));
+        if constexpr (kPerm) {
+          const int32_t* pn = perm_ptr(q_of(b + 2));
 #pragma unroll
-        for (int u = 0; u < 4; ++u) pj_b[u] = ldg_keep_i32(pn + 32 * u, pol_keep);
+          for (int u = 0; u < 4; ++u) pj_b[u] = ldg_keep_i32(pn + 32 * u, pol_keep);
+        } else {
+          cols(q_of(b + 2), pj_b);
+        }
       }
     }
     // packed codes of block b+1, and the radius parameters of its tile if it is a new one
@@ -363,7 +376,8 @@ gemv_kernel(const __grid_constant__ GemvKParams P) {
   while (mi + 1 < P.n_mats && (int)blockIdx.x >= P.mats[mi + 1].cta_begin) ++mi;
   const GemvKMat& g = P.mats[mi];
   const int c = (int)blockIdx.x - g.cta_begin;
-  gemv_cta<MT>(g, c, smem, P.y_f32);
+  if (g.perm) gemv_cta<MT, true>(g, c, smem, P.y_f32);
+  else gemv_cta<MT, false>(g, c, smem, P.y_f32);
 }
 
 }  // namespace

@@ -175,7 +175,7 @@ __device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W
   for (int j8 = threadIdx.x * 8; j8 < K; j8 += blockDim.x * 8) {
     int pj[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) pj[k] = ldg_keep_i32(W.perm + j8 + k, pol_keep);
+    for (int k = 0; k < 8; ++k) pj[k] = W.perm ? ldg_keep_i32(W.perm + j8 + k, pol_keep) : j8 + k;
 #pragma unroll
     for (int c = 0; c < MT; ++c) {
       if (c >= nc) break;

@@ -56,7 +56,12 @@ enum svq_status {
 
 enum svq_dtype { SVQ_F16 = 1, SVQ_BF16 = 2, SVQ_F32 = 3 };
 
-/* One SVQ matrix W[N][K].  Column j of the stored order multiplies x[perm[j]]. */
+/* One SVQ matrix W[N][K].  Column j of the stored order multiplies x[perm[j]].
+ * perm may be NULL: the caller then supplies x already in the stored column
+ * order (the producer of x applied the permutation, as a decoder layer does
+ * when the previous kernel writes its output permuted), every call below reads
+ * x[m][j] for column j, and the permutation pass of svq_linear_gemm is
+ * skipped. */
 typedef struct svq_matrix {
   int32_t N;                      /* output features (rows of W)                            */
   int32_t K;                      /* input features                                         */
@@ -66,7 +71,7 @@ typedef struct svq_matrix {
   const uint16_t* codebook;       /* fp16 [1 << b_d][8], 16-byte aligned                    */
   const uint16_t* radius_scale;   /* fp16 [N]                                               */
   const uint16_t* radius_offset;  /* fp16 [N]                                               */
-  const int32_t* perm;            /* [K], a permutation of 0..K-1                           */
+  const int32_t* perm;            /* [K], a permutation of 0..K-1, 4-byte aligned, or NULL  */
 } svq_matrix;
 
 /* Message for a status code (static string). */
@@ -134,7 +139,8 @@ SVQ_API int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t strea
 /*
  * svq_linear_gemv -- decode-and-multiply for batch 1 to 16:
  *   y[m][n] = sum_j W[n][j] * x[m][perm[j]],  m < M, with W decoded on the fly.
- * x: fp16 [M][K] (natural input order; the kernel applies perm, Figure 6).
+ * x: fp16 [M][K] (natural input order; the kernel applies perm, Figure 6;
+ * stored order when perm is NULL).
  * y: [M][N] of y_dtype SVQ_F16 or SVQ_F32.  fp32 accumulation across
  * subvectors; each subvector's eight products are summed in fp16x2 pairs.
  * Error bound used by the tests: |y - y_ref| <= 1e-3 * sum_j |W[n][j]||x[m][perm[j]]|.
@@ -197,9 +203,11 @@ SVQ_API int svq_linear_gemv_noalloc(const svq_matrix* W /* host */, const uint16
  * shared memory as bf16 (x_dtype SVQ_BF16) or fp16 (x_dtype SVQ_F16) -- the
  * weights are the same rounded values svq_dequantize exports -- and multiplied
  * with fp32 accumulation in tensor memory.  x: [M][K] of x_dtype (natural input
- * order).  y: [M][N] of y_dtype SVQ_F32 or SVQ_BF16.
+ * order; stored order when perm is NULL, x then 16-byte aligned because the
+ * Tensor Memory Accelerator (TMA) reads it directly).  y: [M][N] of y_dtype SVQ_F32
+ * or SVQ_BF16.
  * Workspace (svq_linear_gemm_workspace_size): the permuted activations
- * x[:, perm] plus, when K is split across CTAs, the fp32 partial sums (summed
+ * x[:, perm] (unused when perm is NULL) plus, when K is split across CTAs, the fp32 partial sums (summed
  * by a second kernel in split order); it carries no state between calls and
  * needs no initialisation.  Error bound used by the tests:
  * |y - y_ref| <= 1e-2 * sum_j |W[n][j]||x[m][perm[j]]|.
