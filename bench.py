@@ -199,19 +199,33 @@ def oracle_rows_sample(layer, step: int, rows: int = 8):
     return rows * m.K * 9 // 32, dt
 
 
-def cpu_baseline(layer, budget_s: float = 12.0):
-    import oracle
-    oracle.linear(*layer[1])  # warm (builds the library)
+def _time_oracle(layer, budget_s: float, rows: int):
     nbytes, secs, steps = 0, 0.0, 0
-    rows = 64
     while secs < budget_s:
         b, dt = oracle_rows_sample(layer, steps, rows)
         nbytes += b
         secs += dt
         steps += 1
-    return {"value": nbytes / secs / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+    return nbytes, secs, steps
+
+
+def cpu_baseline(layer, budget_s: float = 12.0, single_budget_s: float = 6.0):
+    """The oracle on all host threads (OpenMP over rows) and, beside it, on one thread."""
+    import oracle
+    oracle.linear(*layer[1])  # warm (builds the library)
+    rows = 64
+    cores = oracle.num_threads()
+    nbytes, secs, steps = _time_oracle(layer, budget_s, rows)
+    oracle.set_threads(1)
+    try:
+        nb1, secs1, steps1 = _time_oracle(layer, single_budget_s, rows)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": nbytes / secs / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{steps} calls of the fp64 C++ oracle, each {rows} rows of one of the seven layer "
-                      f"matrices (decode + fp64 dot), {nbytes} packed bytes in {secs:.1f} s"}
+                      f"matrices (decode + fp64 dot), {nbytes} packed bytes in {secs:.1f} s",
+            "single_thread": {"value": nb1 / secs1 / 1e9, "unit": UNIT, "cores": 1,
+                              "sample": f"{steps1} calls of {rows} rows, {nb1} packed bytes in {secs1:.1f} s"}}
 
 
 def run_reference(args, world, rank):

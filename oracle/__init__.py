@@ -80,6 +80,8 @@ def _load():
         lib.svqref_encode.restype = None
         lib.svqref_num_threads.argtypes = []
         lib.svqref_num_threads.restype = i32
+        lib.svqref_set_threads.argtypes = [i32]
+        lib.svqref_set_threads.restype = None
         _lib = lib
         return lib
 
@@ -202,6 +204,11 @@ def encode(N, K, b_d, W, codebook, scale, offset, energy=None):
 
 def num_threads() -> int:
     return int(_load().svqref_num_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads used by the C++ oracle's parallel loops (timing only; results are independent of it)."""
+    _load().svqref_set_threads(int(n))
 
 
 # --------------------------------------------------------------------------- MoE

@@ -349,4 +349,14 @@ int svqref_num_threads(void) {
 #endif
 }
 
+// Thread count of the later parallel loops (timing only: results do not depend
+// on it, every output is computed by one thread in a fixed order).
+void svqref_set_threads(int n) {
+#ifdef _OPENMP
+  omp_set_num_threads(n > 0 ? n : 1);
+#else
+  (void)n;
+#endif
+}
+
 }  // extern "C"
