@@ -10,7 +10,9 @@ The arithmetic lives in ``svqref.cpp`` (plain C++, fp64 loops, IEEE fp16/bf16
 conversions written from the definitions).  This module compiles it with g++
 on first use and wraps it with numpy-friendly functions.  The MoE composition
 (routing weights, SiLU gate, weighted combine) is written here in numpy fp64
-on top of the C linear layer.
+on top of the C linear layer, and so are the decoder-layer producers (RMS
+normalisation and the SiLU-gated product written in a consumer's stored column
+order).
 """
 from __future__ import annotations
 
@@ -252,3 +254,52 @@ def moe_ffn(experts, x_bits, topk_ids, topk_w, h_bits=None):
             out[t] += float(topk_w[t, s]) * dy[0]
             den[t] += abs(float(topk_w[t, s])) * dden[0]
     return gate_y, up_y, out, den
+
+
+# --------------------------------------------------------------------------- decoder-layer producers
+# The pages only say that each subvector multiplies eight reordered
+# activations ("SAGE", Figure 6 caption).  A decoder layer can have the kernel
+# that produces a linear layer's input write it in that layer's stored column
+# order; these are the two producers of a Qwen3-style decoder layer (the models
+# the pages evaluate), written out from their definitions.
+def f64_to_h_rne(v) -> np.ndarray:
+    """binary64 -> binary16 bit patterns, one round-to-nearest-even step (numpy's conversion;
+    pinned against the C conversion on binary32 inputs and on double-rounding cases)."""
+    with np.errstate(over="ignore"):           # overflow to +-inf is the defined result
+        return np.asarray(v, np.float64).astype(np.float16).view(np.uint16)
+
+
+def act_to_f64(bits, kind: str = "f16") -> np.ndarray:
+    """fp16 or bf16 bit patterns -> fp64 (exact)."""
+    bits = _c(bits, np.uint16)
+    if kind == "f16":
+        return h2f(bits).astype(np.float64).reshape(bits.shape)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rmsnorm(h_bits, h_kind, gamma_bits, eps: float) -> np.ndarray:
+    """RMS normalisation of each row, fp64 before any rounding:
+        x[m][k] = h[m][k] * gamma[k] / sqrt( (1/K) sum_k' h[m][k']^2 + eps )."""
+    h = act_to_f64(h_bits, h_kind)
+    g = act_to_f64(gamma_bits, "f16")
+    ms = np.mean(h * h, axis=1, keepdims=True)
+    return h * g / np.sqrt(ms + float(eps))
+
+
+def rmsnorm_permute(h_bits, h_kind, gamma_bits, eps: float, perms):
+    """The normalised rows written for each consumer in its stored column order,
+    x_g[m][j] = RNE_fp16(rmsnorm(h)[m][p_g[j]]); p_g None = natural order.
+    Returns a list of fp16 bit arrays [M][K]."""
+    xn = rmsnorm(h_bits, h_kind, gamma_bits, eps)
+    return [f64_to_h_rne(xn if p is None else xn[:, np.asarray(p, np.int64)]) for p in perms]
+
+
+def swiglu(gate, up) -> np.ndarray:
+    """silu(gate) * up in fp64 (gate/up: the fp32 outputs of the gate and up projections)."""
+    return silu(np.asarray(gate, np.float64)) * np.asarray(up, np.float64)
+
+
+def swiglu_permute(gate, up, perm) -> np.ndarray:
+    """x[m][j] = RNE_fp16(silu(gate[m][p[j]]) * up[m][p[j]]), p None = natural order (fp16 bits)."""
+    a = swiglu(gate, up)
+    return f64_to_h_rne(a if perm is None else a[:, np.asarray(perm, np.int64)])
