@@ -573,6 +573,75 @@ def run_moe(args):
                           "note": "L2-warm: the same routed experts every replay"}), flush=True)
 
 
+def run_chain(args):
+    """Qwen3-4B decoder-layer chain at batch 1 and 4: the layer's linears in dependency order with their
+    producers (norm -> q|k|v, o, norm -> gate|up, SiLU-gated product -> down; attention itself is not part of
+    the chain, o reads a synthetic attention output).  Two variants: the producers write x in natural order
+    and every SVQ call gathers x[perm] ("gather"), or the producers write each consumer's stored order and the
+    SVQ calls take perm NULL ("stored").  14 rotated layer copies (inputs larger than L2)."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    stream = torch.cuda.Stream()
+    packed_b, _ = layer_bytes()
+    eps = float(np.float32(1e-6))
+    layers = []
+    for L in range(N_LAYERS):
+        Ws = [svq.SvqWeight.from_synth(m) for m, _ in synth.qwen3_4b_layer(L)]
+        layers.append((Ws, [W.without_perm() for W in Ws]))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(12)
+    f16 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float16)).cuda()
+    g1, g2 = f16(rng.uniform(0.5, 1.5, 2560)), f16(rng.uniform(0.5, 1.5, 2560))
+    for M in (1, 4):
+        h1 = torch.from_numpy(synth.make_x(12, 0, M, 2560, energies=True).view(np.int16)).cuda().view(torch.float16)
+        h2 = torch.from_numpy(synth.make_x(12, 1, M, 2560, energies=True).view(np.int16)).cuda().view(torch.float16)
+        att = torch.from_numpy(synth.make_x(12, 2, M, 4096).view(np.int16)).cuda().view(torch.float16)
+        e16 = lambda k: torch.empty((M, k), dtype=torch.float16, device="cuda")
+        xn, xn2, xd = e16(2560), e16(2560), e16(9728)
+        xq, xk, xv, xg, xu = e16(2560), e16(2560), e16(2560), e16(2560), e16(2560)
+        ys = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _, N, _ in synth.QWEN3_4B_SHAPES]
+        groups = lambda Ws: [Ws, Ws[0:3], Ws[3:4], Ws[4:6], Ws[6:7]]
+        nb = max(svq.svq_linear_gemv_batched_workspace_size(G, M) for Ws, _ in layers for G in groups(Ws))
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+        with torch.cuda.stream(stream):
+            svq.svq_workspace_init(ws)
+
+        def gather():
+            for Ws, _ in layers:
+                svq.svq_rmsnorm_permute(h1, g1, eps, [None], [xn])
+                svq.svq_linear_gemv_batched(Ws[0:3], [xn] * 3, ys[0:3], ws)
+                svq.svq_linear_gemv(Ws[3], att, ys[3], ws)
+                svq.svq_rmsnorm_permute(h2, g2, eps, [None], [xn2])
+                svq.svq_linear_gemv_batched(Ws[4:6], [xn2] * 2, ys[4:6], ws)
+                svq.svq_swiglu_permute(ys[4], ys[5], None, xd)
+                svq.svq_linear_gemv(Ws[6], xd, ys[6], ws)
+
+        def stored():
+            for Ws, Wn in layers:
+                svq.svq_rmsnorm_permute(h1, g1, eps, [W.perm for W in Ws[0:3]], [xq, xk, xv])
+                svq.svq_linear_gemv_batched(Wn[0:3], [xq, xk, xv], ys[0:3], ws)
+                svq.svq_linear_gemv(Ws[3], att, ys[3], ws)
+                svq.svq_rmsnorm_permute(h2, g2, eps, [W.perm for W in Ws[4:6]], [xg, xu])
+                svq.svq_linear_gemv_batched(Wn[4:6], [xg, xu], ys[4:6], ws)
+                svq.svq_swiglu_permute(ys[4], ys[5], Ws[6].perm, xd)
+                svq.svq_linear_gemv(Wn[6], xd, ys[6], ws)
+
+        def one_launch():
+            for Ws, _ in layers:
+                svq.svq_linear_gemv_batched(Ws, [xn] * 3 + [att, xn2, xn2, xd], ys, ws)
+
+        res = {}
+        for name, fn in (("one_launch", one_launch), ("gather", gather), ("stored", stored)):
+            res[name] = _time_graph(fn, 50, stream) / N_LAYERS
+        print(json.dumps({"workload": "qwen3-4b decoder-layer chain", "M": M,
+                          "us_per_layer": {k: round(v, 2) for k, v in res.items()},
+                          "GBps_packed": {k: round(packed_b / v / 1e3, 1) for k, v in res.items()},
+                          "launches_per_layer": {"one_launch": 1, "gather": 7, "stored": 7},
+                          "note": "one_launch = the seven linears in one grouped launch without their data "
+                                  "dependencies (the headline); gather/stored = dependency order with producers"}),
+              flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -580,11 +649,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=1400)
     ap.add_argument("--impl", default="svq", choices=["svq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="layer", choices=["layer", "sweep", "prefill", "moe"],
+    ap.add_argument("--workload", default="layer", choices=["layer", "sweep", "prefill", "moe", "chain"],
                     help="layer = the headline line; the others print one JSON line per configuration")
     args = ap.parse_args()
     if args.workload != "layer":
-        return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe}[args.workload](args)
+        return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe, "chain": run_chain}[args.workload](args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_init() if args.impl == "svq" else (int(os.environ.get("WORLD_SIZE", "1")),

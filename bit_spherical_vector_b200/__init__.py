@@ -71,6 +71,8 @@ def lib():
         "svq_linear_gemm": ([MP, P, I, I, P, I, P, SZ, P], I),
         "svq_moe_grouped_gemv_workspace_size": ([I, I, I, I, ctypes.POINTER(SZ)], I),
         "svq_moe_grouped_gemv": ([P, I, I, I, I, P, I, I, P, I, P, I, I, P, SZ, P], I),
+        "svq_rmsnorm_permute": ([P, I, P, ctypes.c_float, I, I, ctypes.POINTER(P), ctypes.POINTER(P), I, P], I),
+        "svq_swiglu_permute": ([P, P, I, I, P, P, P], I),
         "svq_get_device_status": ([P], I),
     }
     for name, (args, res) in sig.items():
@@ -285,6 +287,25 @@ def svq_moe_grouped_gemv(mats_dev, n_mats, N, K, max_b_d, items_dev, n_items, ma
                                       max_items_per_matrix, _ptr(x), x_mode, _ptr(y), n_out_rows, int(accumulate),
                                       _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "svq_moe_grouped_gemv")
+
+
+# ----------------------------------------------------------------------------- decoder-layer producers
+def svq_rmsnorm_permute(h, gamma, eps: float, perms, outs, stream=None):
+    """outs[g][m][j] = fp16(rmsnorm(h)[m][perms[g][j]]) (perms[g] None: natural order).
+    h: [M][K] fp16/bf16, gamma: fp16 [K], outs: list of fp16 [M][K]."""
+    n = len(outs)
+    M, K = h.shape
+    pp = (ctypes.c_void_p * n)(*[0 if p is None else p.data_ptr() for p in perms])
+    op = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    _check(lib().svq_rmsnorm_permute(_ptr(h), _dtype_code(h.dtype), _ptr(gamma), float(eps), M, K, pp, op, n,
+                                     _stream(stream)), "svq_rmsnorm_permute")
+
+
+def svq_swiglu_permute(gate, up, perm, x, stream=None):
+    """x[m][j] = fp16(silu(gate[m][s]) * up[m][s]), s = perm[j] (perm None: s = j); gate/up fp32 [M][I]."""
+    M, I = gate.shape
+    _check(lib().svq_swiglu_permute(_ptr(gate), _ptr(up), M, I, _ptr(perm), _ptr(x), _stream(stream)),
+           "svq_swiglu_permute")
 
 
 def svq_get_device_status(stream=None) -> int:

@@ -15,6 +15,14 @@ cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint
                            const uint16_t* scale, const uint16_t* offset, int out_bf16, uint16_t* out,
                            cudaStream_t st);
 
+// ---------------------------------------------------------------- producers
+constexpr int kMaxProducerOuts = 8;
+cudaError_t launch_rmsnorm_permute(const uint16_t* h, int h_bf16, const uint16_t* gamma, float eps, int M, int K,
+                                   const int32_t* const* perms, uint16_t* const* outs, int n_out,
+                                   cudaStream_t st);
+cudaError_t launch_swiglu_permute(const float* gate, const float* up, int M, int I, const int32_t* perm,
+                                  uint16_t* out, cudaStream_t st);
+
 // ---------------------------------------------------------------- GEMV
 constexpr int kGemvMaxMats = 8;
 constexpr int kGemvMaxTokens = 8;        // tokens per pass (more are split into passes)

@@ -258,6 +258,43 @@ SVQ_API int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int 
                                  void* workspace, size_t workspace_bytes, svq_stream_t stream);
 
 /*
+ * Decoder-layer producers: kernels that write a linear layer's input directly
+ * in the stored column order of its SVQ matrices, so those matrices can be
+ * called with perm NULL.  Each subvector multiplies eight reordered activations
+ * (Figure 6 caption); the pages leave open where the reordering happens.  The
+ * two producers of a Qwen3-style decoder layer (the models the pages evaluate)
+ * are below.  Both are launched as programmatic dependents like the GEMV: they
+ * read their input only after the previous kernel on `stream` has completed,
+ * and the kernel after them may start its weight-only prologue early (its own
+ * wait still covers their writes).  Results are deterministic.
+ *
+ * svq_rmsnorm_permute -- RMS normalisation of M rows of the residual stream h,
+ * written once for each of n_out consumers (1..8):
+ *   inv_m = 1 / sqrt( (1/K) sum_k h[m][k]^2 + eps )          (fp32)
+ *   outs[g][m][j] = fp16( (h[m][s] * inv_m) * gamma[s] ),  s = perms[g][j]
+ * (s = j when perms is NULL or perms[g] is NULL).  h: [M][K] of h_dtype
+ * SVQ_F16 or SVQ_BF16, 16-byte aligned; gamma: fp16 [K], 16-byte aligned;
+ * perms: HOST array of n_out device pointers ([K] int32, 4-byte aligned) or
+ * NULL; outs: HOST array of n_out device pointers, fp16 [M][K], 16-byte
+ * aligned, not overlapping h.  K a multiple of 8, 0 <= M <= 65535, eps finite
+ * and >= 0.  Tolerance used by the tests: 1 fp16 unit in the last place of the
+ * fp64 value rounded once.
+ *
+ * svq_swiglu_permute -- the gated activation in front of an MLP's down
+ * projection, written in that matrix's stored column order:
+ *   x[m][j] = fp16( silu(gate[m][s]) * up[m][s] ),  s = perm[j] (or j if NULL),
+ *   silu(v) = v / (1 + e^-v) in fp32 (the expression SVQ_X_SWIGLU_F32 uses).
+ * gate, up: fp32 [M][I] (e.g. the fp32 outputs of the gate and up GEMVs),
+ * 16-byte aligned; perm: [I] int32, 4-byte aligned, or NULL; x: fp16 [M][I],
+ * 16-byte aligned.  I a multiple of 8, 0 <= M <= 65535.  Tolerance: as above.
+ */
+SVQ_API int svq_rmsnorm_permute(const uint16_t* h, int h_dtype, const uint16_t* gamma, float eps, int M, int K,
+                                const int32_t* const* perms /* host array */, uint16_t* const* outs /* host array */,
+                                int n_out, svq_stream_t stream);
+SVQ_API int svq_swiglu_permute(const float* gate, const float* up, int M, int I, const int32_t* perm, uint16_t* x,
+                               svq_stream_t stream);
+
+/*
  * Synchronising read-and-clear of the device status word that kernels set
  * when a bounded wait runs out (SVQ_OK or SVQ_ERR_TIMEOUT).  Tests only.
  */
