@@ -40,7 +40,7 @@ N_LAYERS = 14
 WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 1, one grouped launch per step"
 
 
-# DRAM bytes (read + written) of one gemv_kernel<1> launch on this workload,
+# DRAM bytes (read + written) of one gemv_kernel<1, 1> launch on this workload,
 # from an ncu capture (profiles/gemv_kernel_qwen3_4b_layer_batch1.md), valid
 # only while the GEMV kernel sources hash to the value it was taken with.
 GEMV_TRAFFIC_CAPTURE = {
@@ -417,7 +417,7 @@ def run_gpu(args, world, rank, local):
                      "frac": achieved / peak, "traffic": gemv_traffic(),
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s",
-                     "kernel": "gemv_kernel<1> (grouped, 7 matrices)",
+                     "kernel": "gemv_kernel<1, 1> (grouped, 7 matrices)",
                      "achieved_bytes": "all algorithmic bytes per launch (packed codes, codebooks, radius "
                                        "params, perm, x, y)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -626,19 +626,31 @@ def run_chain(args):
                 svq.svq_swiglu_permute(ys[4], ys[5], Ws[6].perm, xd)
                 svq.svq_linear_gemv(Wn[6], xd, ys[6], ws)
 
+        def stored_o():
+            # as stored, with the attention output also taken in o's stored order
+            for Ws, Wn in layers:
+                svq.svq_rmsnorm_permute(h1, g1, eps, [W.perm for W in Ws[0:3]], [xq, xk, xv])
+                svq.svq_linear_gemv_batched(Wn[0:3], [xq, xk, xv], ys[0:3], ws)
+                svq.svq_linear_gemv(Wn[3], att, ys[3], ws)
+                svq.svq_rmsnorm_permute(h2, g2, eps, [W.perm for W in Ws[4:6]], [xg, xu])
+                svq.svq_linear_gemv_batched(Wn[4:6], [xg, xu], ys[4:6], ws)
+                svq.svq_swiglu_permute(ys[4], ys[5], Ws[6].perm, xd)
+                svq.svq_linear_gemv(Wn[6], xd, ys[6], ws)
+
         def one_launch():
             for Ws, _ in layers:
                 svq.svq_linear_gemv_batched(Ws, [xn] * 3 + [att, xn2, xn2, xd], ys, ws)
 
         res = {}
-        for name, fn in (("one_launch", one_launch), ("gather", gather), ("stored", stored)):
+        for name, fn in (("one_launch", one_launch), ("gather", gather), ("stored", stored), ("stored_o", stored_o)):
             res[name] = _time_graph(fn, 50, stream) / N_LAYERS
         print(json.dumps({"workload": "qwen3-4b decoder-layer chain", "M": M,
                           "us_per_layer": {k: round(v, 2) for k, v in res.items()},
                           "GBps_packed": {k: round(packed_b / v / 1e3, 1) for k, v in res.items()},
-                          "launches_per_layer": {"one_launch": 1, "gather": 7, "stored": 7},
+                          "launches_per_layer": {"one_launch": 1, "gather": 7, "stored": 7, "stored_o": 7},
                           "note": "one_launch = the seven linears in one grouped launch without their data "
-                                  "dependencies (the headline); gather/stored = dependency order with producers"}),
+                                  "dependencies (the headline); gather/stored = dependency order with producers; "
+                                  "stored_o = stored with the attention output also in o's stored order"}),
               flush=True)
 
 

@@ -332,12 +332,12 @@ int svq_rmsnorm_permute(const uint16_t* h, int h_dtype, const uint16_t* gamma, f
   if (!(eps >= 0.0f) || eps > 3.0e38f) return SVQ_ERR_INVALID_ARG;   // rejects NaN and infinity
   if (M < 0 || M > 65535) return SVQ_ERR_INVALID_ARG;
   if (K < 8 || K % 8 != 0) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVQ_OK;                     // nothing to read or write
   if (!h || !gamma || !aligned(h, 16) || !aligned(gamma, 16)) return SVQ_ERR_INVALID_ARG;
   for (int g = 0; g < n_out; ++g) {
     if (!outs[g] || !aligned(outs[g], 16)) return SVQ_ERR_INVALID_ARG;
     if (perms && perms[g] && !aligned(perms[g], 4)) return SVQ_ERR_INVALID_ARG;
   }
-  if (M == 0) return SVQ_OK;
   return cuda_status(svq::launch_rmsnorm_permute(h, h_dtype == SVQ_BF16, gamma, eps, M, K, perms, outs, n_out,
                                                  (cudaStream_t)stream));
 }
@@ -346,9 +346,9 @@ int svq_swiglu_permute(const float* gate, const float* up, int M, int I, const i
                        svq_stream_t stream) {
   if (M < 0 || M > 65535) return SVQ_ERR_INVALID_ARG;
   if (I < 8 || I % 8 != 0) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SVQ_OK;                     // nothing to read or write
   if (!gate || !up || !x || !aligned(gate, 16) || !aligned(up, 16) || !aligned(x, 16)) return SVQ_ERR_INVALID_ARG;
   if (perm && !aligned(perm, 4)) return SVQ_ERR_INVALID_ARG;
-  if (M == 0) return SVQ_OK;
   return cuda_status(svq::launch_swiglu_permute(gate, up, M, I, perm, x, (cudaStream_t)stream));
 }
 

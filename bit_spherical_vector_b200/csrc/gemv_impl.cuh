@@ -368,7 +368,10 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   }
 }
 
-template <int MT>
+// PM: 1 = every matrix of the launch has a permutation, 0 = none has, 2 = mixed
+// (each CTA follows its own matrix).  The uniform cases get kernels of their own
+// so each is compiled (registers, schedule) for one path only.
+template <int MT, int PM>
 __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
 gemv_kernel(const __grid_constant__ GemvKParams P) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -376,20 +379,24 @@ gemv_kernel(const __grid_constant__ GemvKParams P) {
   while (mi + 1 < P.n_mats && (int)blockIdx.x >= P.mats[mi + 1].cta_begin) ++mi;
   const GemvKMat& g = P.mats[mi];
   const int c = (int)blockIdx.x - g.cta_begin;
-  if (g.perm) gemv_cta<MT, true>(g, c, smem, P.y_f32);
-  else gemv_cta<MT, false>(g, c, smem, P.y_f32);
+  if constexpr (PM == 1) {
+    gemv_cta<MT, true>(g, c, smem, P.y_f32);
+  } else if constexpr (PM == 0) {
+    gemv_cta<MT, false>(g, c, smem, P.y_f32);
+  } else {
+    if (g.perm) gemv_cta<MT, true>(g, c, smem, P.y_f32);
+    else gemv_cta<MT, false>(g, c, smem, P.y_f32);
+  }
 }
 
-}  // namespace
-
-template <int MT>
-cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
+template <int MT, int PM>
+cudaError_t launch_gemv_pm(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
   static unsigned long long attr_set = 0;       // one bit per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !((attr_set >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemv_kernel<MT, PM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kGemvSmemMax);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set |= 1ull << dev;
@@ -407,9 +414,20 @@ cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT>, p);
+  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT, PM>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+template <int MT>
+cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
+  int with = 0;
+  for (int i = 0; i < p.n_mats; ++i) with += p.mats[i].perm != nullptr;
+  if (with == p.n_mats) return launch_gemv_pm<MT, 1>(p, grid, smem, st);
+  if (with == 0) return launch_gemv_pm<MT, 0>(p, grid, smem, st);
+  return launch_gemv_pm<MT, 2>(p, grid, smem, st);
 }
 
 }  // namespace svq

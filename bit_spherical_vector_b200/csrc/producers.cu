@@ -56,11 +56,53 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_permute_kernel(const __g
   const int m = blockIdx.z, g = blockIdx.y;
   const int K = p.K;
   const uint16_t* hr = p.h + (size_t)m * K;
+  const int j8 = blockIdx.x * kProdCols + threadIdx.x * 8;
+  const bool act = j8 < K;
+  const int32_t* pm = p.perm[g];
+  // The permutation and gamma are weights, not written by the previous kernel:
+  // read them before waiting for it, so only the h loads follow the wait.
+  int s[8];
+  float gm[8];
+  if (act) {
+    if (pm) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) s[k] = __ldg(pm + j8 + k);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) gm[k] = __half2float(__ushort_as_half(__ldg(p.gamma + s[k])));
+    } else {
+      const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gamma + j8));
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        s[2 * k] = j8 + 2 * k;
+        s[2 * k + 1] = j8 + 2 * k + 1;
+        gm[2 * k] = __half2float(__ushort_as_half((uint16_t)(gw[k] & 0xFFFFu)));
+        gm[2 * k + 1] = __half2float(__ushort_as_half((uint16_t)(gw[k] >> 16)));
+      }
+    }
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
+  // this thread's 8 inputs (gathered through the permutation) are loaded
+  // together with the row's sum-of-squares loads
+  float hv[8];
+  if (act) {
+    if (pm) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) hv[k] = act_to_f32(hr[s[k]], p.h_bf16);
+    } else {
+      const uint4 v = *reinterpret_cast<const uint4*>(hr + j8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        hv[2 * k] = act_to_f32((uint16_t)(w[k] & 0xFFFFu), p.h_bf16);
+        hv[2 * k + 1] = act_to_f32((uint16_t)(w[k] >> 16), p.h_bf16);
+      }
+    }
+  }
   float ss = 0.f;
-  for (int j8 = threadIdx.x * 8; j8 < K; j8 += kProdCols) {
-    const uint4 v = *reinterpret_cast<const uint4*>(hr + j8);
+  for (int i8 = threadIdx.x * 8; i8 < K; i8 += kProdCols) {
+    const uint4 v = *reinterpret_cast<const uint4*>(hr + i8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -79,29 +121,10 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_permute_kernel(const __g
   for (int w = 0; w < kProdThreads / 32; ++w) tot += wsum[w];
   const float inv = 1.0f / sqrtf(tot / (float)K + p.eps);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  const int j8 = blockIdx.x * kProdCols + threadIdx.x * 8;
-  if (j8 >= K) return;
-  const int32_t* pm = p.perm[g];
+  if (!act) return;
   float x[8];
-  if (pm) {
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int s = __ldg(pm + j8 + k);
-      x[k] = act_to_f32(hr[s], p.h_bf16) * inv * __half2float(__ushort_as_half(__ldg(p.gamma + s)));
-    }
-  } else {
-    const uint4 hv = *reinterpret_cast<const uint4*>(hr + j8);
-    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gamma + j8));
-    const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      x[2 * k] = act_to_f32((uint16_t)(hw[k] & 0xFFFFu), p.h_bf16) * inv *
-                 __half2float(__ushort_as_half((uint16_t)(gw[k] & 0xFFFFu)));
-      x[2 * k + 1] = act_to_f32((uint16_t)(hw[k] >> 16), p.h_bf16) * inv *
-                     __half2float(__ushort_as_half((uint16_t)(gw[k] >> 16)));
-    }
-  }
+  for (int k = 0; k < 8; ++k) x[k] = hv[k] * inv * gm[k];
   uint4 o;
   o.x = pack_h2(x[0], x[1]);
   o.y = pack_h2(x[2], x[3]);
@@ -119,18 +142,23 @@ __global__ void __launch_bounds__(kProdThreads) swiglu_permute_kernel(const floa
                                                                       uint16_t* __restrict__ out, int I) {
   const int m = blockIdx.y;
   const int j8 = blockIdx.x * kProdCols + threadIdx.x * 8;
+  const bool act = j8 < I;
+  int s[8];
+  if (act && perm) {                                   // weights: read before the wait
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s[k] = __ldg(perm + j8 + k);
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (j8 >= I) return;
+  if (!act) return;
   const float* gr = gate + (size_t)m * I;
   const float* ur = up + (size_t)m * I;
   float gv[8], uv[8];
   if (perm) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const int s = __ldg(perm + j8 + k);
-      gv[k] = gr[s];
-      uv[k] = ur[s];
+      gv[k] = gr[s[k]];
+      uv[k] = ur[s[k]];
     }
   } else {
     const float4 g0 = *reinterpret_cast<const float4*>(gr + j8), g1 = *reinterpret_cast<const float4*>(gr + j8 + 4);

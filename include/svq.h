@@ -277,7 +277,7 @@ SVQ_API int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int 
  * perms: HOST array of n_out device pointers ([K] int32, 4-byte aligned) or
  * NULL; outs: HOST array of n_out device pointers, fp16 [M][K], 16-byte
  * aligned, not overlapping h.  K a multiple of 8, 0 <= M <= 65535, eps finite
- * and >= 0.  Tolerance used by the tests: 1 fp16 unit in the last place of the
+ * and >= 0.  M = 0 returns SVQ_OK without looking at any pointer.  Tolerance used by the tests: 1 fp16 unit in the last place of the
  * fp64 value rounded once.
  *
  * svq_swiglu_permute -- the gated activation in front of an MLP's down
@@ -286,7 +286,8 @@ SVQ_API int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int 
  *   silu(v) = v / (1 + e^-v) in fp32 (the expression SVQ_X_SWIGLU_F32 uses).
  * gate, up: fp32 [M][I] (e.g. the fp32 outputs of the gate and up GEMVs),
  * 16-byte aligned; perm: [I] int32, 4-byte aligned, or NULL; x: fp16 [M][I],
- * 16-byte aligned.  I a multiple of 8, 0 <= M <= 65535.  Tolerance: as above.
+ * 16-byte aligned.  I a multiple of 8, 0 <= M <= 65535 (M = 0: SVQ_OK, no
+ * pointer looked at).  Tolerance: as above.
  */
 SVQ_API int svq_rmsnorm_permute(const uint16_t* h, int h_dtype, const uint16_t* gamma, float eps, int M, int K,
                                 const int32_t* const* perms /* host array */, uint16_t* const* outs /* host array */,
