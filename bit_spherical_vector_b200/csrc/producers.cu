@@ -25,7 +25,8 @@ namespace svq {
 namespace {
 
 constexpr int kProdThreads = 256;
-constexpr int kProdCols = kProdThreads * 8;       // columns written by one CTA
+constexpr int kProdCols = kProdThreads * 2;       // columns written by one CTA (2 per thread)
+constexpr int kSumStride = kProdThreads * 8;      // the sum of squares reads 8 columns per thread and step
 
 struct NormParams {
   const uint16_t* h;
@@ -45,10 +46,11 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   return (uint32_t)__half_as_ushort(__float2half_rn(a)) | ((uint32_t)__half_as_ushort(__float2half_rn(b)) << 16);
 }
 
-// grid (ceil(K / 2048), consumers, M).  Every CTA of a row computes the row's
-// sum of squares in the same fixed order (8 consecutive elements per thread,
-// butterfly over the warp, warps in index order), so all consumers of a row
-// see the same scale; then it writes 2048 columns of its consumer:
+// grid (ceil(K / 512), consumers, M).  Every CTA of a row computes the row's
+// sum of squares in the same fixed order (8 consecutive elements per thread and
+// step, butterfly over the warp, warps in index order), so all consumers of a
+// row see the same scale; then it writes 512 columns of its consumer, two per
+// thread (small CTAs spread the permutation gathers over many SMs):
 //   x_g[m][j] = fp16( (h[m][s] * inv) * gamma[s] ),  s = p_g[j] (or j),
 //   inv = 1 / sqrt(sum_k h[m][k]^2 / K + eps)   (fp32).
 __global__ void __launch_bounds__(kProdThreads) rmsnorm_permute_kernel(const __grid_constant__ NormParams p) {
@@ -56,52 +58,41 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_permute_kernel(const __g
   const int m = blockIdx.z, g = blockIdx.y;
   const int K = p.K;
   const uint16_t* hr = p.h + (size_t)m * K;
-  const int j8 = blockIdx.x * kProdCols + threadIdx.x * 8;
-  const bool act = j8 < K;
+  const int j2 = blockIdx.x * kProdCols + threadIdx.x * 2;
+  const bool act = j2 < K;                       // K is a multiple of 8: j2 + 1 < K as well
   const int32_t* pm = p.perm[g];
   // The permutation and gamma are weights, not written by the previous kernel:
   // read them before waiting for it, so only the h loads follow the wait.
-  int s[8];
-  float gm[8];
+  int s0 = j2, s1 = j2 + 1;
+  float gm0 = 0.f, gm1 = 0.f;
   if (act) {
     if (pm) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) s[k] = __ldg(pm + j8 + k);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) gm[k] = __half2float(__ushort_as_half(__ldg(p.gamma + s[k])));
+      s0 = __ldg(pm + j2);
+      s1 = __ldg(pm + j2 + 1);
+      gm0 = __half2float(__ushort_as_half(__ldg(p.gamma + s0)));
+      gm1 = __half2float(__ushort_as_half(__ldg(p.gamma + s1)));
     } else {
-      const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gamma + j8));
-      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        s[2 * k] = j8 + 2 * k;
-        s[2 * k + 1] = j8 + 2 * k + 1;
-        gm[2 * k] = __half2float(__ushort_as_half((uint16_t)(gw[k] & 0xFFFFu)));
-        gm[2 * k + 1] = __half2float(__ushort_as_half((uint16_t)(gw[k] >> 16)));
-      }
+      const uint32_t gw = __ldg(reinterpret_cast<const unsigned int*>(p.gamma + j2));
+      gm0 = __half2float(__ushort_as_half((uint16_t)(gw & 0xFFFFu)));
+      gm1 = __half2float(__ushort_as_half((uint16_t)(gw >> 16)));
     }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // this thread's 8 inputs (gathered through the permutation) are loaded
-  // together with the row's sum-of-squares loads
-  float hv[8];
+  // this thread's two inputs are loaded together with the sum-of-squares loads
+  float h0 = 0.f, h1 = 0.f;
   if (act) {
     if (pm) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) hv[k] = act_to_f32(hr[s[k]], p.h_bf16);
+      h0 = act_to_f32(hr[s0], p.h_bf16);
+      h1 = act_to_f32(hr[s1], p.h_bf16);
     } else {
-      const uint4 v = *reinterpret_cast<const uint4*>(hr + j8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        hv[2 * k] = act_to_f32((uint16_t)(w[k] & 0xFFFFu), p.h_bf16);
-        hv[2 * k + 1] = act_to_f32((uint16_t)(w[k] >> 16), p.h_bf16);
-      }
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(hr + j2);
+      h0 = act_to_f32((uint16_t)(w & 0xFFFFu), p.h_bf16);
+      h1 = act_to_f32((uint16_t)(w >> 16), p.h_bf16);
     }
   }
   float ss = 0.f;
-  for (int i8 = threadIdx.x * 8; i8 < K; i8 += kProdCols) {
+  for (int i8 = threadIdx.x * 8; i8 < K; i8 += kSumStride) {
     const uint4 v = *reinterpret_cast<const uint4*>(hr + i8);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -122,59 +113,41 @@ __global__ void __launch_bounds__(kProdThreads) rmsnorm_permute_kernel(const __g
   const float inv = 1.0f / sqrtf(tot / (float)K + p.eps);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (!act) return;
-  float x[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) x[k] = hv[k] * inv * gm[k];
-  uint4 o;
-  o.x = pack_h2(x[0], x[1]);
-  o.y = pack_h2(x[2], x[3]);
-  o.z = pack_h2(x[4], x[5]);
-  o.w = pack_h2(x[6], x[7]);
-  *reinterpret_cast<uint4*>(p.out[g] + (size_t)m * K + j8) = o;
+  *reinterpret_cast<uint32_t*>(p.out[g] + (size_t)m * K + j2) = pack_h2(h0 * inv * gm0, h1 * inv * gm1);
 }
 
-// grid (ceil(I / 2048), M): x[m][j] = fp16( silu(gate[m][s]) * up[m][s] ),
+// grid (ceil(I / 512), M): x[m][j] = fp16( silu(gate[m][s]) * up[m][s] ),
 // s = perm[j] (or j), silu(v) = v / (1 + e^-v) in fp32 -- the same expression
-// the MoE kernel evaluates for its fused down-projection input.
+// the MoE kernel evaluates for its fused down-projection input.  Two columns
+// per thread.
 __global__ void __launch_bounds__(kProdThreads) swiglu_permute_kernel(const float* __restrict__ gate,
                                                                       const float* __restrict__ up,
                                                                       const int32_t* __restrict__ perm,
                                                                       uint16_t* __restrict__ out, int I) {
   const int m = blockIdx.y;
-  const int j8 = blockIdx.x * kProdCols + threadIdx.x * 8;
-  const bool act = j8 < I;
-  int s[8];
-  if (act && perm) {                                   // weights: read before the wait
-#pragma unroll
-    for (int k = 0; k < 8; ++k) s[k] = __ldg(perm + j8 + k);
+  const int j2 = blockIdx.x * kProdCols + threadIdx.x * 2;
+  const bool act = j2 < I;                       // I is a multiple of 8
+  int s0 = j2, s1 = j2 + 1;
+  if (act && perm) {                             // weights: read before the wait
+    s0 = __ldg(perm + j2);
+    s1 = __ldg(perm + j2 + 1);
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (!act) return;
   const float* gr = gate + (size_t)m * I;
   const float* ur = up + (size_t)m * I;
-  float gv[8], uv[8];
+  float g0, g1, u0, u1;
   if (perm) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      gv[k] = gr[s[k]];
-      uv[k] = ur[s[k]];
-    }
+    g0 = gr[s0]; g1 = gr[s1];
+    u0 = ur[s0]; u1 = ur[s1];
   } else {
-    const float4 g0 = *reinterpret_cast<const float4*>(gr + j8), g1 = *reinterpret_cast<const float4*>(gr + j8 + 4);
-    const float4 u0 = *reinterpret_cast<const float4*>(ur + j8), u1 = *reinterpret_cast<const float4*>(ur + j8 + 4);
-    gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w; gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
-    uv[0] = u0.x; uv[1] = u0.y; uv[2] = u0.z; uv[3] = u0.w; uv[4] = u1.x; uv[5] = u1.y; uv[6] = u1.z; uv[7] = u1.w;
+    const float2 gv = *reinterpret_cast<const float2*>(gr + j2), uv = *reinterpret_cast<const float2*>(ur + j2);
+    g0 = gv.x; g1 = gv.y; u0 = uv.x; u1 = uv.y;
   }
-  float x[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) x[k] = gv[k] / (1.0f + expf(-gv[k])) * uv[k];
-  uint4 o;
-  o.x = pack_h2(x[0], x[1]);
-  o.y = pack_h2(x[2], x[3]);
-  o.z = pack_h2(x[4], x[5]);
-  o.w = pack_h2(x[6], x[7]);
-  *reinterpret_cast<uint4*>(out + (size_t)m * I + j8) = o;
+  const float x0 = g0 / (1.0f + expf(-g0)) * u0;
+  const float x1 = g1 / (1.0f + expf(-g1)) * u1;
+  *reinterpret_cast<uint32_t*>(out + (size_t)m * I + j2) = pack_h2(x0, x1);
 }
 
 template <typename Kern, typename... Args>
