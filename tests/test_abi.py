@@ -60,3 +60,63 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(svq, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         svq.lib()
+
+
+def test_header_compiles_as_c_and_links(tmp_path):
+    """include/svq.h is plain C (C99, warnings as errors); a C program links against libsvq.so and calls the
+    host-only entry points."""
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_svq.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "svq.h"\n'
+        "int main(void) {\n"
+        "  svq_matrix m = {128, 128, 8, 0, 0, 0, 0, 0, 0};\n"
+        "  size_t n = 0;\n"
+        "  int st = svq_linear_gemv_workspace_size(&m, 1, &n);\n"
+        '  printf("%zu %zu %d %s\\n", svq_packed_bytes(1024, 1024), svq_canonical_bytes(3, 40), st,\n'
+        "         svq_status_string(SVQ_ERR_WORKSPACE));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "use_svq"
+    libdir = os.path.dirname(svq.LIB_PATH)
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                         str(src), "-L", libdir, "-lsvq", "-Wl,-rpath," + libdir, "-o", str(exe)],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, run.stderr
+    packed, canon, st, msg = run.stdout.split(" ", 3)
+    assert int(packed) == 1024 * 1024 * 9 // 32 and int(canon) == 36
+    assert int(st) == svq.SVQ_ERR_INVALID_ARG          # NULL weight pointers are refused on the host
+    assert msg.strip()
+
+
+def test_stored_order_and_producer_validation_without_gpu():
+    """Checks that return before any CUDA call: perm NULL is accepted by the matrix check, the GEMM then
+    wants a 16-byte aligned x; producers refuse bad counts, shapes and alignments, and M = 0 is a no-op."""
+    L = svq.lib()
+    nullp = ctypes.c_void_p(0)
+    m = svq.svq_matrix(128, 128, 8, 0, 0x1000, 0x2000, 0x3000, 0x4000, 0)     # perm NULL
+    x_unaligned = ctypes.c_void_p(0x6002)
+    assert L.svq_linear_gemm(ctypes.byref(m), x_unaligned, svq.SVQ_BF16, 16, ctypes.c_void_p(0x7000),
+                             svq.SVQ_F32, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    badperm = svq.svq_matrix(128, 128, 8, 0, 0x1000, 0x2000, 0x3000, 0x4000, 0x5002)
+    assert L.svq_dequantize(ctypes.byref(badperm), svq.SVQ_F16, ctypes.c_void_p(0x7000), nullp) == \
+        svq.SVQ_ERR_INVALID_ARG
+    P = ctypes.c_void_p
+    outs = (P * 2)(0x8000, 0x9000)
+    perms = (P * 2)(0, 0)
+    h, gamma = P(0x1000), P(0x2000)
+    f = L.svq_rmsnorm_permute
+    assert f(h, svq.SVQ_F16, gamma, 1e-6, 1, 64, perms, outs, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert f(h, svq.SVQ_F16, gamma, 1e-6, 1, 64, perms, outs, 9, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert f(h, svq.SVQ_F32, gamma, 1e-6, 1, 64, perms, outs, 2, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert f(h, svq.SVQ_F16, gamma, -1.0, 1, 64, perms, outs, 2, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert f(h, svq.SVQ_F16, gamma, 1e-6, 1, 60, perms, outs, 2, nullp) == svq.SVQ_ERR_UNSUPPORTED_SHAPE
+    assert f(P(0x1002), svq.SVQ_F16, gamma, 1e-6, 1, 64, perms, outs, 2, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert f(h, svq.SVQ_F16, gamma, 1e-6, 0, 64, perms, outs, 2, nullp) == svq.SVQ_OK
+    g = L.svq_swiglu_permute
+    assert g(P(0x1000), P(0x2000), 1, 12, nullp, P(0x3000), nullp) == svq.SVQ_ERR_UNSUPPORTED_SHAPE
+    assert g(P(0x1000), P(0x2004), 1, 16, nullp, P(0x3000), nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert g(P(0x1000), P(0x2000), 1, 16, P(0x4002), P(0x3000), nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert g(nullp, nullp, 0, 16, nullp, nullp, nullp) == svq.SVQ_OK
