@@ -40,9 +40,9 @@ N_LAYERS = 14
 WORKLOAD = "qwen3-4b decoder layer: 7 SVQ linears (q,k,v,o,gate,up,down), batch 1, one grouped launch per step"
 
 
-# DRAM bytes (read + written) of one gemv_kernel<1, 1> launch on this workload,
-# from an ncu capture (profiles/gemv_kernel_qwen3_4b_layer_batch1.md), valid
-# only while the GEMV kernel sources hash to the value it was taken with.
+# DRAM bytes (read + written) of one GEMV launch on this workload, from an ncu
+# capture of the kernel built from the sources whose hash is recorded here;
+# reported only while the sources still hash to that value.
 GEMV_TRAFFIC_CAPTURE = {
     "bytes": 28770560,
     "sources": ["gemv_impl.cuh", "gemv_device.cuh", "gemv.cu", "gemv_params.h", "gemv_mt1.cu", "layout.cuh",

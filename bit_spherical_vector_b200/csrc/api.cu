@@ -111,8 +111,10 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 // address returned by cudaGetSymbolAddress.
 void* noalloc_scratch(cudaStream_t stream) {
   static void* ptr[64] = {nullptr};
+  static std::mutex mu;                          // first calls from several host threads
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
@@ -125,8 +127,10 @@ void* noalloc_scratch(cudaStream_t stream) {
 
 int* status_word() {
   static int* ptr[64] = {nullptr};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!ptr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;

@@ -185,8 +185,12 @@ SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const ui
  *     1 MiB returns SVQ_ERR_WORKSPACE and enqueues nothing (e.g. M = 8 on a
  *     32768 x 2560 matrix; split such a call into passes of fewer rows).
  *   - The first call on a device looks up the array's device address and
- *     zero-fills it on `stream`; make that first call before any stream
- *     capture.
+ *     zero-fills it on `stream`; under lazy module loading that first call may
+ *     also be what loads the library's device code, which reserves the array
+ *     and the kernels' code on that device.  Make the first call on each
+ *     device at set-up time: before the host freezes its memory pools and
+ *     before any stream capture.  The first-call set-up is guarded, so host
+ *     threads may make their first calls concurrently.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other threads) race and give wrong results; serialise them.
  *   - The array keeps the last call's contents; the counters that must start

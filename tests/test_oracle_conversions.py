@@ -53,8 +53,8 @@ def test_f16_to_f32_all_65536():
 def test_bf16_to_f32_all_65536():
     bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
     ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
-    got = np.array([oracle.bf2f_scalar(int(b)) for b in bits[::97]], np.float32)
-    r = ref[::97]
+    got = np.array([oracle.bf2f_scalar(int(b)) for b in bits], np.float32)
+    r = ref
     nan = np.isnan(r)
     assert np.array_equal(np.isnan(got), nan)
     assert np.array_equal(got[~nan].view(np.uint32), r[~nan].view(np.uint32))
