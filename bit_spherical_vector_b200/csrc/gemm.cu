@@ -140,44 +140,93 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
   auto word = [&](int wi) -> uint32_t {
     return *reinterpret_cast<const uint32_t*>(lb + (wi >> 2) * cstride + (wi & 3) * 4);
   };
-  const uint32_t S = word(j);
   const int bd = p.b_d;
   const uint32_t imask = (1u << bd) - 1u;
   const uint32_t cmask = (1u << (10 - bd)) - 1u;
   const int rep = p.cb_replicas;
   const uint8_t* cbq = cbs + (lane & (rep - 1)) * 16;
   const int cb_stride = rep * 16;                      // bytes per codebook entry (all replicas)
-  uint32_t top[2] = {0u, 0u};
-  if (j == 15) {
-    // payloads 60..63 live in the top two bits of the 20 payload words (chunks
-    // 4..8): read the five chunks whole (16-byte loads, conflict free)
-    uint32_t pw[20];
+  // Fields of the lane's subvectors (row 4 * lane + r, group j) of this block:
+  // sign byte, direction index, radius code.
+  uint32_t sgn[2], pidx[2], pcode[2];
+  if (L == 32) {
+    // fragment arrangement (full tile): signs from the four sign-holder lanes of
+    // the lane's quad, the index from its address lane, the code from itself
+    auto wordl = [&](int l, int wi) -> uint32_t {
+      return *reinterpret_cast<const uint32_t*>(pk + word_offset_in_block(32, l, wi));
+    };
+    auto slot = [&](int l, int u, int k) -> uint32_t {
+      const int pb = frag_slot_bit(u, k);
+      uint32_t P[2];
+      P[0] = wordl(l, frag_payload_word(pb >> 5));
+      P[1] = (pb & 31) > 22 ? wordl(l, frag_payload_word((pb >> 5) + 1)) : 0u;
+      return payload_field(P, pb & 31);
+    };
 #pragma unroll
-    for (int c = 0; c < 5; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(lb + (4 + c) * cstride);
-      pw[4 * c] = v.x; pw[4 * c + 1] = v.y; pw[4 * c + 2] = v.z; pw[4 * c + 3] = v.w;
+    for (int rr = 0; rr < 2; ++rr) {
+      const int r = r0 + rr;
+      const int u = frag_round(r, j);
+      pcode[rr] = (slot(lane, u, frag_code_slot(r, j)) >> bd) & cmask;
+      pidx[rr] = slot(frag_addr_lane(lane, r, j), u, frag_addr_slot(lane)) & imask;
+      const int ww = frag_sign_pos(lane, r, j);
+      uint32_t sg = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t S = wordl(frag_sign_lane(lane, q), frag_sign_word(u));
+        sg |= ((S >> (15 - ww)) & 1u) << (2 * q);
+        sg |= ((S >> (31 - ww)) & 1u) << (2 * q + 1);
+      }
+      sgn[rr] = sg;
     }
-    uint32_t t4[4] = {0u, 0u, 0u, 0u};
+  } else {
+    // owner arrangement (partial tile): everything in the lane's own words
+    const uint32_t S = word(j);
+    uint32_t top[2] = {0u, 0u};
+    if (j == 15) {
+      // payloads 60..63 live in the top two bits of the 20 payload words (chunks
+      // 4..8): read the five chunks whole (16-byte loads, conflict free)
+      uint32_t pw[20];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+      for (int c = 0; c < 5; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(lb + (4 + c) * cstride);
+        pw[4 * c] = v.x; pw[4 * c + 1] = v.y; pw[4 * c + 2] = v.z; pw[4 * c + 3] = v.w;
+      }
+      uint32_t t4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int i = 0; i < 5; ++i) t4[r] |= (pw[5 * r + i] >> 30) << (8 - 2 * i);
-    top[0] = r0 == 0 ? t4[0] : t4[2];
-    top[1] = r0 == 0 ? t4[1] : t4[3];
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int i = 0; i < 5; ++i) t4[r] |= (pw[5 * r + i] >> 30) << (8 - 2 * i);
+      top[0] = r0 == 0 ? t4[0] : t4[2];
+      top[1] = r0 == 0 ? t4[1] : t4[3];
+    }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int r = r0 + rr;
+      const int v = 4 * j + r;
+      uint32_t pay;
+      if (j < 15) {
+        const int wi = 16 + v / 3;
+        pay = word(wi) >> (10 * (v - 3 * (wi - 16)));
+      } else {
+        pay = top[rr];
+      }
+      pidx[rr] = pay & imask;
+      pcode[rr] = (pay >> bd) & cmask;
+      uint32_t sg = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int t = 4 * r + q;
+        sg |= ((S >> (15 - t)) & 1u) << (2 * q);
+        sg |= ((S >> (31 - t)) & 1u) << (2 * q + 1);
+      }
+      sgn[rr] = sg;
+    }
   }
 #pragma unroll
   for (int rr = 0; rr < 2; ++rr) {
     const int r = r0 + rr;
-    const int v = 4 * j + r;
-    uint32_t pay;
-    if (j < 15) {
-      const int wi = 16 + v / 3;
-      pay = word(wi) >> (10 * (v - 3 * (wi - 16)));
-    } else {
-      pay = top[rr];
-    }
-    const uint32_t id = pay & imask;
-    const uint32_t code = (pay >> bd) & cmask;
+    const uint32_t id = pidx[rr];
+    const uint32_t code = pcode[rr];
     const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
     const float scr = r0 == 0 ? sc[rr] : sc[2 + rr], ofr = r0 == 0 ? of[rr] : of[2 + rr];
     const float rad = __fmaf_rn(scr, (float)code, ofr);
@@ -188,7 +237,8 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
     for (int q = 0; q < 4; ++q) {
       const float2 cf = __half22float2(*reinterpret_cast<const __half2*>(&c4[q]));
       const float2 pr = __fmul2_rn(rad2, cf);               // binary32 products r * c
-      o4[q] = pack2<BF16>(pr.x, pr.y) ^ ((S << (4 * r + q)) & 0x80008000u);
+      const uint32_t sm = (((sgn[rr] >> (2 * q)) & 1u) << 15) | (((sgn[rr] >> (2 * q + 1)) & 1u) << 31);
+      o4[q] = pack2<BF16>(pr.x, pr.y) ^ sm;
     }
     const int rho = lane + 32 * r;                       // A-tile row of weight row 4 * lane + r
     uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);

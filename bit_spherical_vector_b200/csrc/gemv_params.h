@@ -22,12 +22,14 @@ struct GemvKMat {
   unsigned* counters;     // [n_tiles]
   int N, K, b_d, M;
   int ctas, cta_begin, kmax, npw;
+  int x_smem;             // 1: the CTA stages x (natural order, MT rows) in shared memory
 };
 
 struct GemvKParams {
   GemvKMat mats[kGemvMaxMats];
   int n_mats;
   int y_f32;
+  uint32_t one;           // always 1: shift amounts derived from it stay opaque to the compiler
 };
 
 constexpr size_t kGemvSmemMax = 220 * 1024;

@@ -244,9 +244,22 @@ __device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& 
       ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
     }
     const uint32_t q16 = (uint32_t)(lane % RR) * 16;
+    // full tiles: fragment decode on the tensor cores (gemv_device.cuh)
+    const FragK fk = frag_consts(p.one, BD, RR);
+    const uint32_t cb_base_q = (uint32_t)__cvta_generic_to_shared(cbs) + q16;
+    uint32_t bm[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) bm[i][h] = ((lane >> 3) == i && ((lane >> 2) & 1) == h) ? 0xFFFFFFFFu : 0u;
+    const uint32_t xw_off = 16u * ((lane >> 2) & 1) + 4u * (lane & 3);
     for (int b = 0; b < nb; ++b) {
       if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
-      process_block<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cbs, q16, cs, CODEM, scp, ofp, acc);
+      if (L == 32)
+        process_block_frag<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cb_base_q, fk, bm, xw_off, scp,
+                               ofp, acc);
+      else
+        process_block<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cbs, q16, cs, CODEM, scp, ofp, acc);
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     }

@@ -225,6 +225,8 @@ void svqref_decode_exact(int N, int K, int b_d, const uint8_t* canon, const uint
   std::vector<uint8_t> s((size_t)N * G);
   std::vector<uint16_t> id((size_t)N * G), cd((size_t)N * G);
   svqref_unpack(N, K, b_d, canon, s.data(), id.data(), cd.data());
+  // rows are independent: decoded in parallel (the values do not depend on the thread count)
+#pragma omp parallel for schedule(static)
   for (int n = 0; n < N; ++n) {
     for (int g = 0; g < G; ++g) {
       const int64_t f = (int64_t)n * G + g;
