@@ -518,7 +518,7 @@ def _time_graph(fn, reps, stream):
 
 def run_sweep(args, quiet=False):
     """8192 x 8192 (7,3) matrix, M = 1..16 tokens: GEMV and tensor-core GEMM, 20 rotated copies (378 MB)."""
-    out = []
+    recs = []
     import torch
     import bit_spherical_vector_b200 as svq
     stream = torch.cuda.Stream()
@@ -554,18 +554,18 @@ def run_sweep(args, quiet=False):
                "gemv_GBps": round(packed / tv / 1e3, 1), "gemm_us": round(tg, 3),
                "gemm_GBps": round(packed / tg / 1e3, 1), "faster": "gemv" if tv <= tg else "gemm",
                "tokens_per_s_best": round(M / min(tv, tg) * 1e6, 1)}
-        out.append(rec)
+        recs.append(rec)
         if not quiet:
             print(json.dumps(rec), flush=True)
-    cross = next((r["M"] for r in out if r["faster"] == "gemm"), None)
+    cross = next((r["M"] for r in recs if r["faster"] == "gemm"), None)
     if quiet:
-        return {"per_M": out, "gemv_to_gemm_crossover_M": cross}
+        return {"per_M": recs, "gemv_to_gemm_crossover_M": cross}
     return 0
 
 
 def run_prefill(args, quiet=False):
     """Qwen3-4B gate/up (2560->9728) and down (9728->2560), (8,2), M = 512 and 2048, bf16."""
-    out = []
+    recs = []
     import torch
     import bit_spherical_vector_b200 as svq
     stream = torch.cuda.Stream()
@@ -596,15 +596,15 @@ def run_prefill(args, quiet=False):
                    "svq_frac_of_bf16_peak": round(flop / t / 1e6 / tpeak, 3),
                    "cublas_dense_bf16_us": round(tc, 2), "cublas_TFLOPs": round(flop / tc / 1e6, 1),
                    "peak_bf16_TFLOPs": tpeak, "note": "svq time includes the x[:,perm] pass"}
-            out.append(rec)
+            recs.append(rec)
             if not quiet:
                 print(json.dumps(rec), flush=True)
-    return out if quiet else 0
+    return recs if quiet else 0
 
 
 def run_moe(args, quiet=False):
     """Qwen3-30B-A3B-shaped MoE FFN (hidden 2048, 128 experts, inter 768, top-8), T = 1 and 16."""
-    out = []
+    recs = []
     import torch
     import bit_spherical_vector_b200 as svq
     stream = torch.cuda.Stream()
@@ -644,10 +644,10 @@ def run_moe(args, quiet=False):
                "tokens_per_s": round(T / t * 1e6, 1), "experts_touched": touched,
                "GBps_distinct_packed": round(nbytes / t / 1e3, 1),
                "note": "L2-warm: the same routed experts every replay"}
-        out.append(rec)
+        recs.append(rec)
         if not quiet:
             print(json.dumps(rec), flush=True)
-    return out if quiet else 0
+    return recs if quiet else 0
 
 
 def run_chain(args):

@@ -70,7 +70,8 @@ def lib():
         "svq_linear_gemm_workspace_size": ([MP, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemm": ([MP, P, I, I, P, I, P, SZ, P], I),
         "svq_moe_grouped_gemv_workspace_size": ([I, I, I, I, ctypes.POINTER(SZ)], I),
-        "svq_moe_grouped_gemv": ([P, I, I, I, I, P, I, I, P, I, P, I, I, P, SZ, P], I),
+        "svq_debug_set_wait_polls": ([ctypes.c_uint], ctypes.c_uint),
+        "svq_moe_grouped_gemv": ([P, I, I, I, I, P, I, I, P, I, I, P, I, I, P, SZ, P], I),
         "svq_rmsnorm_permute": ([P, I, P, ctypes.c_float, I, I, ctypes.POINTER(P), ctypes.POINTER(P), I, P], I),
         "svq_swiglu_permute": ([P, P, I, I, P, P, P], I),
         "svq_get_device_status": ([P], I),
@@ -283,9 +284,10 @@ def svq_moe_grouped_gemv_workspace_size(n_mats: int, n_items: int, N: int, accum
 
 def svq_moe_grouped_gemv(mats_dev, n_mats, N, K, max_b_d, items_dev, n_items, max_items_per_matrix, x, x_mode,
                          y, n_out_rows, accumulate, ws, stream=None):
+    n_x_rows = int(x.shape[0])                 # items' x_row must lie below (checked on the device)
     _check(lib().svq_moe_grouped_gemv(_ptr(mats_dev), n_mats, N, K, max_b_d, _ptr(items_dev), n_items,
-                                      max_items_per_matrix, _ptr(x), x_mode, _ptr(y), n_out_rows, int(accumulate),
-                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+                                      max_items_per_matrix, _ptr(x), x_mode, n_x_rows, _ptr(y), n_out_rows,
+                                      int(accumulate), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "svq_moe_grouped_gemv")
 
 
@@ -310,6 +312,11 @@ def svq_swiglu_permute(gate, up, perm, x, stream=None):
 
 def svq_get_device_status(stream=None) -> int:
     return int(lib().svq_get_device_status(_stream(stream)))
+
+
+def svq_debug_set_wait_polls(polls: int) -> int:
+    """Poll bound of the GEMM's bounded waits for later launches (tests); returns the previous bound."""
+    return int(lib().svq_debug_set_wait_polls(int(polls)))
 
 
 def header_functions() -> list[str]:

@@ -296,10 +296,11 @@ int svq_moe_grouped_gemv_workspace_size(int n_mats, int n_items, int N, int accu
 }
 
 int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int max_b_d, const svq_group_item* items,
-                         int n_items, int max_items_per_matrix, const void* x, int x_mode, float* y,
+                         int n_items, int max_items_per_matrix, const void* x, int x_mode, int n_x_rows, float* y,
                          int n_out_rows, int accumulate, void* workspace, size_t workspace_bytes,
                          svq_stream_t stream) {
-  if (!mats || !items || !x || !y || n_mats < 1 || n_items < 1 || n_out_rows < 1) return SVQ_ERR_INVALID_ARG;
+  if (!mats || !items || !x || !y || n_mats < 1 || n_items < 1 || n_out_rows < 1 || n_x_rows < 1)
+    return SVQ_ERR_INVALID_ARG;
   if (max_b_d < 1 || max_b_d > 10 || !svq::layout_supported(N, K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
   if (n_mats > 16384 || max_items_per_matrix < 1) return SVQ_ERR_INVALID_ARG;
   if (x_mode != SVQ_X_F16 && x_mode != SVQ_X_SWIGLU_F32) return SVQ_ERR_INVALID_ARG;
@@ -315,7 +316,8 @@ int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int m
   char* b = reinterpret_cast<char*>(workspace);
   svq::MoeKParams p;
   p.mats = mats; p.n_mats = n_mats; p.N = N; p.K = K; p.max_b_d = max_b_d;
-  p.items = items; p.n_items = n_items; p.x = x; p.x_mode = x_mode; p.y = y; p.accumulate = accumulate ? 1 : 0;
+  p.items = items; p.n_items = n_items; p.x = x; p.x_mode = x_mode; p.n_x_rows = n_x_rows; p.y = y;
+  p.n_out_rows = n_out_rows; p.accumulate = accumulate ? 1 : 0;
   p.offsets = reinterpret_cast<int*>(b + w.offsets);
   p.cursor = reinterpret_cast<int*>(b + w.cursor);
   p.sorted = reinterpret_cast<int*>(b + w.sorted);
@@ -356,6 +358,8 @@ int svq_swiglu_permute(const float* gate, const float* up, int M, int I, const i
   if (perm && !aligned(perm, 4)) return SVQ_ERR_INVALID_ARG;
   return cuda_status(svq::launch_swiglu_permute(gate, up, M, I, perm, x, (cudaStream_t)stream));
 }
+
+unsigned svq_debug_set_wait_polls(unsigned polls) { return svq::set_wait_polls(polls); }
 
 int svq_get_device_status(svq_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SVQ_ERR_CUDA;

@@ -37,6 +37,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 
 #include "gemm_params.h"
@@ -84,7 +85,7 @@ __device__ __forceinline__ void record_timeout(const GemmKParams& p, Bars* bars)
 
 // Wait that gives up on timeout or when another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const GemmKParams& p, Bars* bars) {
-  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+  for (uint32_t i = 0; i < p.wait_polls; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 63 && *(volatile int*)&bars->abort_flag) return false;
   }
@@ -568,6 +569,12 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
+namespace {
+std::atomic<uint32_t> g_wait_polls{kWaitPolls};
+}  // namespace
+
+uint32_t set_wait_polls(uint32_t polls) { return g_wait_polls.exchange(polls); }
+
 GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   GemmPlan g{};
   g.BN = M >= 256 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : (M > 16 ? 32 : 16)));
@@ -635,6 +642,7 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.y_f32 = d.y_f32;
   p.partial = g.S > 1 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
   p.status = status;
+  p.wait_polls = g_wait_polls.load(std::memory_order_relaxed);
   cudaError_t e = d.x_bf16 ? launch_typed<true>(g.BN, tm, p, g.grid, st) : launch_typed<false>(g.BN, tm, p, g.grid, st);
   if (e != cudaSuccess || g.S == 1) return e;
   const long long mn = (long long)d.M * d.N;

@@ -19,6 +19,7 @@ struct GemmKParams {
   int y_f32;
   float* partial;       // [S][M][N] when S > 1
   int* status;          // device status word (bounded-wait timeouts)
+  uint32_t wait_polls;  // polls before a bounded wait gives up (svq_debug_set_wait_polls)
 };
 
 struct GemmPlan {
@@ -40,6 +41,9 @@ struct GemmMatDesc {
 };
 
 GemmPlan plan_gemm(int N, int K, int M, int num_sms);
+// Poll bound of the GEMM's bounded waits for subsequent launches (tests set 0
+// to make a wait give up at once); returns the previous value.
+uint32_t set_wait_polls(uint32_t polls);
 cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* status, cudaStream_t st);
 
 }  // namespace svq

@@ -308,24 +308,37 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint16_t* xg = g.x;
   if constexpr (kXS) {
-    // stage x (natural order, M rows) in shared memory: coalesced copy
+    // stage x (natural order, M rows) in shared memory: coalesced copy, four
+    // loads in flight per thread before their stores (one round trip for a
+    // token of up to 4 * 16 * blockDim columns)
     const bool vec = (reinterpret_cast<uintptr_t>(xg) & 15) == 0;
-    const int per_row = K / 8;
-    for (int i = threadIdx.x; i < MT * per_row; i += blockDim.x) {
-      const int m = i / per_row, j = i - m * per_row;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (m < M) {
-        if (vec) {
-          v = ldg_keep_v4(reinterpret_cast<const uint4*>(xg + (size_t)m * K) + j, pol_keep);
-        } else {
-          uint16_t h[8];
+    const int per_row = K / 8, total = MT * per_row;
+    for (int i0 = threadIdx.x; i0 < total; i0 += 4 * blockDim.x) {
+      uint4 v[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) h[k] = ldg_keep_u16(xg + (size_t)m * K + 8 * j + k, pol_keep);
-          v = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16), h[4] | ((uint32_t)h[5] << 16),
-                         h[6] | ((uint32_t)h[7] << 16));
+      for (int k = 0; k < 4; ++k) {
+        const int i = i0 + k * blockDim.x;
+        v[k] = make_uint4(0, 0, 0, 0);
+        if (i < total) {
+          const int m = i / per_row, j = i - m * per_row;
+          if (m < M) {
+            if (vec) {
+              v[k] = ldg_keep_v4(reinterpret_cast<const uint4*>(xg + (size_t)m * K) + j, pol_keep);
+            } else {
+              uint16_t h[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) h[e] = ldg_keep_u16(xg + (size_t)m * K + 8 * j + e, pol_keep);
+              v[k] = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16),
+                                h[4] | ((uint32_t)h[5] << 16), h[6] | ((uint32_t)h[7] << 16));
+            }
+          }
         }
       }
-      *reinterpret_cast<uint4*>(xn + ((size_t)m * K + 8 * j) * 2) = v;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int i = i0 + k * blockDim.x;
+        if (i < total) *reinterpret_cast<uint4*>(xn + (size_t)i * 16) = v[k];
+      }
     }
   }
   // Let the next kernel in the stream start its own weight-only prologue as this

@@ -20,7 +20,11 @@
 //      projection, fp16(silu(gate) * up) computed on the fly from an fp32
 //      [gate | up] row;
 //   3. combine_kernel (when accumulating): y[r] = sum of the items with
-//      out_row r, in item order (deterministic).
+//      out_row r, in item order (deterministic); one CTA per output row
+//      compacts its row's item list in item order, linear in the items.
+// Item fields are range-checked on the device: an input row outside x is read
+// as zeros, an output row outside y is not written, and either sets the device
+// status word to SVQ_ERR_INVALID_ARG (svq_get_device_status).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -170,8 +174,15 @@ __device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W
                                         int nc, unsigned char* xs, uint64_t pol_keep) {
   const int K = p.K;
   int xrow[MT];
+  bool xok[MT];
 #pragma unroll
-  for (int c = 0; c < MT; ++c) xrow[c] = c < nc ? p.items[sorted[i0 + c]].x_row : 0;
+  for (int c = 0; c < MT; ++c) {
+    xrow[c] = c < nc ? p.items[sorted[i0 + c]].x_row : 0;
+    // an input row outside x is reported (status word) and read as zeros
+    xok[c] = xrow[c] >= 0 && xrow[c] < p.n_x_rows;
+    if (c < nc && !xok[c] && threadIdx.x == 0) atomicExch(p.status, SVQ_ERR_INVALID_ARG);
+    if (!xok[c]) xrow[c] = 0;
+  }
   for (int j8 = threadIdx.x * 8; j8 < K; j8 += blockDim.x * 8) {
     int pj[8];
 #pragma unroll
@@ -179,8 +190,10 @@ __device__ __forceinline__ void stage_x(const MoeKParams& p, const svq_matrix& W
 #pragma unroll
     for (int c = 0; c < MT; ++c) {
       if (c >= nc) break;
-      uint32_t h[8];
-      if (p.x_mode == 0) {
+      uint32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (!xok[c]) {
+        // zeros (the item was reported as invalid)
+      } else if (p.x_mode == 0) {
         const uint16_t* xr = reinterpret_cast<const uint16_t*>(p.x) + (size_t)xrow[c] * K;
 #pragma unroll
         for (int k = 0; k < 8; ++k) h[k] = ldg_keep_u16(xr + pj[k], pol_keep);
@@ -280,8 +293,13 @@ __device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& 
     const svq_group_item it = p.items[item];
     const int n = t * kTileRows + nl;
     v *= it.out_scale;
-    if (p.accumulate) p.item_out[(size_t)item * N + n] = v;
-    else p.y[(size_t)it.out_row * N + n] = v;
+    if (p.accumulate) {
+      p.item_out[(size_t)item * N + n] = v;
+    } else if (it.out_row >= 0 && it.out_row < p.n_out_rows) {
+      p.y[(size_t)it.out_row * N + n] = v;
+    } else if (e == threadIdx.x) {
+      atomicExch(p.status, SVQ_ERR_INVALID_ARG);     // an output row outside y: reported, not written
+    }
   }
   __syncthreads();                                   // red is reused by the next unit
 }
@@ -462,19 +480,49 @@ __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_con
 }
 
 // y[r][n] = sum over items i with out_row r (ascending i) of item_out[i][n].
-__global__ void combine_kernel(const MoeKParams p, int n_out_rows) {
-  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (long long)n_out_rows * p.N) return;
-  const int r = (int)(e / p.N), n = (int)(e - (long long)r * p.N);
-  float s = 0.f;
-  bool any = false;
-  for (int i = 0; i < p.n_items; ++i) {
-    if (p.items[i].out_row == r) {
-      s += p.item_out[(size_t)i * p.N + n];
-      any = true;
+// One CTA per output row: the CTA scans the item list once and compacts the
+// indices of its row's items in item order (warp ballots, then a prefix over
+// the warps), so the work is linear in the number of items per row; rows with
+// more items than the shared list holds fall back to a scan per column.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineList = 2048;
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const MoeKParams p) {
+  __shared__ int list[kCombineList];
+  __shared__ int s_warp[kCombineThreads / 32];
+  __shared__ int s_count;
+  const int r = blockIdx.x, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (threadIdx.x == 0) s_count = 0;
+  __syncthreads();
+  for (int base = 0; base < p.n_items; base += kCombineThreads) {
+    const int i = base + threadIdx.x;
+    const bool hit = i < p.n_items && p.items[i].out_row == r;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
+    if (lane == 0) s_warp[wid] = __popc(bal);
+    __syncthreads();
+    int before = s_count;
+    for (int w = 0; w < wid; ++w) before += s_warp[w];
+    const int pos = before + __popc(bal & ((1u << lane) - 1u));
+    if (hit && pos < kCombineList) list[pos] = i;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int add = 0;
+      for (int w = 0; w < kCombineThreads / 32; ++w) add += s_warp[w];
+      s_count += add;
     }
+    __syncthreads();
   }
-  if (any) p.y[(size_t)r * p.N + n] = s;
+  const int cnt = s_count;
+  if (cnt == 0) return;                              // rows with no item are left untouched
+  for (int n = threadIdx.x; n < p.N; n += kCombineThreads) {
+    float s = 0.f;
+    if (cnt <= kCombineList) {
+      for (int k = 0; k < cnt; ++k) s += p.item_out[(size_t)list[k] * p.N + n];
+    } else {
+      for (int i = 0; i < p.n_items; ++i)
+        if (p.items[i].out_row == r) s += p.item_out[(size_t)i * p.N + n];
+    }
+    p.y[(size_t)r * p.N + n] = s;
+  }
 }
 
 template <int MT>
@@ -528,8 +576,7 @@ cudaError_t launch_moe(MoeKParams p, int mt, int n_out_rows, int num_sms, cudaSt
   }
   if (e != cudaSuccess) return e;
   if (p.accumulate) {
-    const long long work = (long long)n_out_rows * p.N;
-    combine_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(p, n_out_rows);
+    combine_kernel<<<(unsigned)n_out_rows, kCombineThreads, 0, st>>>(p);
     e = cudaGetLastError();
   }
   return e;

@@ -16,7 +16,9 @@ struct MoeKParams {
   int n_items;
   const void* x;                   // x_mode 0: fp16 [*][K]; 1: fp32 [*][2K] (gate | up)
   int x_mode;
+  int n_x_rows;                    // rows of x (items' x_row must be below)
   float* y;                        // [n_out_rows][N]
+  int n_out_rows;
   int accumulate;
   int* offsets;                    // workspace: item offsets per matrix [n_mats + 1]
   int* cursor;                     // [n_mats]

@@ -231,9 +231,16 @@ SVQ_API int svq_linear_gemm(const svq_matrix* W /* host */, const uint16_t* x, i
  *   accumulate == 0:   y[out_row_i] = v_i          (out rows must be distinct)
  *   accumulate == 1:   y[r] = sum of v_i over the items with out_row == r, in
  *                      item order (rows with no item are left untouched)
- * in(row): x_mode SVQ_X_F16 -> x is fp16 [*][K], in(row) = x[row];
- *          x_mode SVQ_X_SWIGLU_F32 -> x is fp32 [*][2K] holding [gate | up],
+ * in(row): x_mode SVQ_X_F16 -> x is fp16 [n_x_rows][K], in(row) = x[row];
+ *          x_mode SVQ_X_SWIGLU_F32 -> x is fp32 [n_x_rows][2K] holding [gate | up],
  *          in(row) = fp16(silu(gate) * up) computed per element in fp32.
+ * Item fields are checked on the device: an item whose x_row lies outside
+ *   0..n_x_rows-1 reads zeros, one whose out_row lies outside 0..n_out_rows-1
+ *   (accumulate == 0) is not written, an item whose matrix lies outside
+ *   0..n_mats-1 is skipped; each of these sets the device status word to
+ *   SVQ_ERR_INVALID_ARG (svq_get_device_status).  With accumulate == 1 the
+ *   items of one output row are summed in item order by one CTA per row, linear
+ *   in the number of items.
  * mats: DEVICE array of n_mats descriptors (same layout as svq_matrix), every
  *   one N x K with b_d <= max_b_d; the host cannot read them, so the caller
  *   guarantees them (the host checks N, K, max_b_d and the pointers it sees).
@@ -258,7 +265,7 @@ enum svq_x_mode { SVQ_X_F16 = 0, SVQ_X_SWIGLU_F32 = 1 };
 SVQ_API int svq_moe_grouped_gemv_workspace_size(int n_mats, int n_items, int N, int accumulate, size_t* bytes);
 SVQ_API int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int max_b_d,
                                  const svq_group_item* items, int n_items, int max_items_per_matrix,
-                                 const void* x, int x_mode, float* y, int n_out_rows, int accumulate,
+                                 const void* x, int x_mode, int n_x_rows, float* y, int n_out_rows, int accumulate,
                                  void* workspace, size_t workspace_bytes, svq_stream_t stream);
 
 /*
@@ -301,9 +308,22 @@ SVQ_API int svq_swiglu_permute(const float* gate, const float* up, int M, int I,
 
 /*
  * Synchronising read-and-clear of the device status word that kernels set
- * when a bounded wait runs out (SVQ_OK or SVQ_ERR_TIMEOUT).  Tests only.
+ * when a bounded wait runs out (SVQ_ERR_TIMEOUT) or a device-side argument
+ * check fails (SVQ_ERR_INVALID_ARG); SVQ_OK when neither happened.  Tests only.
  */
 SVQ_API int svq_get_device_status(svq_stream_t stream);
+
+/*
+ * Test aid for the failure path of the bounded waits (no counterpart in the
+ * paper).  Every wait of svq_linear_gemm on a pipeline barrier polls at most
+ * `polls` times (default 2^21) before it gives up: the kernel then sets the
+ * status word to SVQ_ERR_TIMEOUT, lets the copies it already issued land,
+ * releases its tensor memory and returns (no trap, no hang).  polls == 0 makes
+ * the first wait give up at once.  Applies to launches enqueued after the
+ * call, process-wide; returns the previous bound.  Restore the default before
+ * relying on results.
+ */
+SVQ_API unsigned svq_debug_set_wait_polls(unsigned polls);
 
 #ifdef __cplusplus
 }
