@@ -38,14 +38,18 @@ size_t up256(size_t b) { return (b + 255) / 256 * 256; }
 // CTA of unit q when T units are split into G contiguous ranges [c*T/G, (c+1)*T/G).
 long long cta_of(long long q, long long T, long long G) { return ((q + 1) * G - 1) / T; }
 
-// codebook replicas + two x slots per warp + per-warp partial sums of npw tiles
-// + 36 ints (warp range boundaries and first tiles) + one completion counter per tile of a CTA's
-// range (at most ntc tiles)
-size_t cta_smem(int b_d, int mt, int npw, int ntc, int K, int x_smem) {
+// codebook replicas + x (x_smem 2: natural order and, with a permutation, stored
+// order; 1: natural order; 0: none) + two x slots per warp (x_smem < 2) +
+// per-warp partial sums of npw tiles + 36 ints (warp range boundaries and first
+// tiles) + one completion counter per tile of a CTA's range (at most ntc tiles)
+size_t cta_smem(int b_d, int mt, int npw, int ntc, int K, int x_smem, bool perm) {
   const int R = gemv_cb_replicas(b_d);
   const int W = gemv_warps(mt);
-  return ((size_t)16 * R << b_d) + (x_smem ? (size_t)mt * K * 2 : 0) + (size_t)W * 2 * mt * kBlockCols * 2 +
-         (size_t)W * npw * mt * kTileRows * sizeof(float) + 144 + ((size_t)ntc * 4 + 15) / 16 * 16;
+  const size_t xcopy = (size_t)mt * K * 2;
+  const size_t x = x_smem == 2 ? xcopy * (perm ? 2 : 1) : (x_smem == 1 ? xcopy : 0);
+  const size_t slots = x_smem == 2 ? 0 : (size_t)W * 2 * mt * kBlockCols * 2;
+  return ((size_t)16 * R << b_d) + x + slots + (size_t)W * npw * mt * kTileRows * sizeof(float) + 144 +
+         ((size_t)ntc * 4 + 15) / 16 * 16;
 }
 
 }  // namespace
@@ -98,7 +102,7 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
       ++used;
     }
     size_t smem = 0, off = kGemvCounterBytes;
-    int total = 0, counters = 0;
+    int total = 0, counters = 0, x_smem = 2;
     for (int i = 0; i < n_mats; ++i) {
       GemvPlanMat& pm = plan->m[i];
       const long long Gi = ctas[i], Ui = U[i];
@@ -126,10 +130,27 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
       }
       total += pm.ctas;
       const int ntc = (int)((cta_len + tu - 2) / tu + 2);
-      // stage x in shared memory when it fits beside the rest (the gathers
-      // from shared memory cost far fewer L1 wavefronts than scattered global loads)
-      pm.x_smem = cta_smem(mats[i].b_d, mt, pm.npw, ntc, mats[i].K, 1) <= kGemvSmemMax ? 1 : 0;
-      smem = std::max(smem, cta_smem(mats[i].b_d, mt, pm.npw, ntc, mats[i].K, pm.x_smem));
+      // stage x in shared memory when it fits beside the rest: preferably in
+      // stored order as well (the decode then reads it with no per-unit
+      // gathers), else in natural order (gathers from shared memory cost far
+      // fewer L1 wavefronts than scattered global loads)
+      // (one choice for the whole launch: the kernel is compiled per choice).
+      // A stored-order copy costs the prologue one permuting pass over all K
+      // columns; it pays when there is no permutation (the copy is x itself) or
+      // when every CTA's range covers a full tile row of units, i.e. would
+      // gather each column at least once anyway.
+      pm.ntc = ntc;
+      const bool perm = mats[i].perm != nullptr;
+      const bool pays = !perm || Ui / Gi >= tu;
+      int fit = 0;
+      for (int xm = pays ? 2 : 1; xm >= 1 && fit == 0; --xm)
+        if (cta_smem(mats[i].b_d, mt, pm.npw, ntc, mats[i].K, xm, perm) <= kGemvSmemMax) fit = xm;
+      x_smem = std::min(x_smem, fit);
+    }
+    for (int i = 0; i < n_mats; ++i) {
+      GemvPlanMat& pm = plan->m[i];
+      pm.x_smem = x_smem;
+      smem = std::max(smem, cta_smem(mats[i].b_d, mt, pm.npw, pm.ntc, mats[i].K, x_smem, mats[i].perm != nullptr));
     }
     if (counters > kGemvMaxCounters) return false;
     if (counters == 0) off = 0;

@@ -3,14 +3,18 @@
 // decode-and-multiply (shared by the grouped GEMV and the MoE kernels):
 // cache-policy loads, lane-block loads and the per-block decode + dot product.
 //
-// A lane owns 4 rows x 16 subvectors of a block (layout.cuh).  For each
-// subvector: idx and radius code come out of the payload word with one shift
-// and one mask each; the fp16 codeword is gathered from the lane's replica of
-// the shared-memory codebook (conflict free); the subvector's sign bits are
-// XORed onto the fp16 sign bits (the shifted sign word puts each pair's two
-// signs on bits 15 and 31); 8 products are summed in fp16x2 and the radius
-// r = offset + scale * code ("SAGE", arXiv 2610.14745, Figure 2 caption: signs,
-// direction index, quantized radius) scales the sum in fp32.
+// Two decodes, one per arrangement of a block (layout.cuh):
+//  * fragment decode (full 128-row tiles, the hot path): per round of 128
+//    subvectors, ldmatrix gathers the fp16 codewords into tensor-core A
+//    fragments, the sign bits are XORed onto their fp16 sign bits, four
+//    mma.m16n8k16 form the eight-element dot products in fp32, and each is
+//    scaled by its radius and accumulated in fp32;
+//  * owner decode (a partial last tile): a lane owns 4 rows x 16 subvectors;
+//    per subvector the codeword is gathered with one 16-byte shared-memory
+//    load, signed by XOR, multiplied by x in fp16x2, the 8 products summed in
+//    fp32 and scaled by the radius in fp32.
+// The radius is r = offset + scale * code ("SAGE", arXiv 2610.14745, Figure 2
+// caption: signs, direction index, quantized radius).
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -155,11 +159,13 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
       cw.w ^= (S << (4 * r + 3)) & 0x80008000u;
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        __half2 p = __hmul2(as_h2(cw.x), as_h2(xv[m].x));
-        p = __hfma2(as_h2(cw.y), as_h2(xv[m].y), p);
-        p = __hfma2(as_h2(cw.z), as_h2(xv[m].z), p);
-        p = __hfma2(as_h2(cw.w), as_h2(xv[m].w), p);
-        dsum[r][m] = __half2float(__hadd(__low2half(p), __high2half(p)));
+        // products in fp16 (|c| <= 1, so a product never exceeds |x|), summed in fp32
+        const float2 p0 = __half22float2(__hmul2(as_h2(cw.x), as_h2(xv[m].x)));
+        const float2 p1 = __half22float2(__hmul2(as_h2(cw.y), as_h2(xv[m].y)));
+        const float2 p2 = __half22float2(__hmul2(as_h2(cw.z), as_h2(xv[m].z)));
+        const float2 p3 = __half22float2(__hmul2(as_h2(cw.w), as_h2(xv[m].w)));
+        const float2 q = __fadd2_rn(__fadd2_rn(p0, p1), __fadd2_rn(p2, p3));
+        dsum[r][m] = q.x + q.y;
       }
     }
     // radius r = scp * v + ofp and accumulation, two rows per packed fp32x2 FMA

@@ -11,27 +11,28 @@
 //
 // B200 mapping:
 //   * one CTA per SM; each matrix of the group gets SMs in proportion to its
-//     blocks, and each CTA a contiguous range of the matrix's blocks (128-row
-//     tile x 128 columns, in storage order, crossing tile boundaries), so all
-//     SMs stream about the same number of bytes;
-//   * the warps of a CTA split its range contiguously again; each lane owns 4
-//     complete rows of the current tile, so a row's partial sum never leaves
-//     its thread in the hot loop;
+//     work, and each CTA a contiguous range of the matrix's units (a quarter
+//     block -- 128 rows x 4 subvector groups -- in full tiles, a whole block in
+//     a partial last tile), in storage order and crossing tile boundaries, so
+//     all SMs stream about the same number of bytes;
+//   * the warps of a CTA split its range contiguously again; in a full tile
+//     lane T accumulates rows 4T..4T+3, so a row's partial sum never leaves its
+//     thread in the hot loop;
 //   * packed codes stream from HBM with 16-byte coalesced loads
-//     (ld.global.nc.L1::no_allocate, L2 evict-first), one block (9 loads per
-//     lane) ahead of the decode;
+//     (ld.global.nc.L1::no_allocate, L2 evict-first), one unit ahead of the
+//     decode, plus an L2 prefetch of the next block;
 //   * the fp16 codebook sits in shared memory as 8 replicas (4 for 1024
-//     entries), entry e of replica q at 16-byte slot 8e + q, and lane l reads
-//     replica l % 8: the 8 lanes of each quarter-warp phase of an LDS.128 hit 8
-//     different bank groups whatever the indices, so the random gather is
-//     conflict free;
-//   * each warp gathers x[perm] for its blocks itself, software-pipelined: the
-//     permutation of block b+2 and the activations of block b+1 are loaded
-//     while block b is decoded, into the other of two small shared-memory
-//     slots that the lanes read with broadcast loads;
-//   * signs are applied by XOR on fp16 sign bits; the eight products of a
-//     subvector are summed in fp16x2, then scaled by the radius and
-//     accumulated across subvectors in fp32;
+//     entries), entry e of replica q at 16-byte slot 8e + q; ldmatrix gathers
+//     the codewords straight into tensor-core A fragments, the eight lanes of
+//     each 8x8 matrix reading eight different replicas (conflict free);
+//   * signs are applied by XOR on the fp16 sign bits of the A fragments, the
+//     eight-element dot products run as mma.m16n8k16 with fp32 accumulation,
+//     and each product is scaled by its radius and accumulated in fp32
+//     (gemv_device.cuh, fragment decode);
+//   * x: staged in shared memory by the prologue, either in stored order as
+//     well (the decode reads its B operands from there) or in natural order
+//     only, each warp then gathering x[perm] for its next unit into a small
+//     double-buffered slot while it decodes the current one;
 //   * when a warp's range leaves a tile it parks that tile's sums in shared
 //     memory; the last warp of the CTA to leave the tile (a shared-memory
 //     counter) adds the parked sums in range order, so tiles complete while
@@ -42,6 +43,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <type_traits>
 
@@ -196,9 +198,18 @@ struct QRegs {
 
 // One CTA = one contiguous range of one matrix's units.  kPerm: the matrix has
 // a permutation (x is gathered through it); without one, x is already in stored
-// column order.
-template <int MT, bool kPerm, bool kXS>
+// column order.  kXM: where the decode reads x from --
+//   2: shared memory, all K columns in stored order, written once by the CTA's
+//      prologue (natural-order copy, then one permuting pass); the hot loop
+//      reads its operands straight from there;
+//   1: a natural-order copy in shared memory, gathered unit by unit into small
+//      per-warp slots (when a stored-order copy as well does not fit);
+//   0: global memory, gathered unit by unit into the slots.
+template <int MT, bool kPerm, int kXM>
 __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char* smem, int y_f32, uint32_t one) {
+  constexpr bool kXS = kXM >= 1;                       // x staged in shared memory (natural order)
+  constexpr bool kXP = kXM == 2;                       // ... and read by the decode in stored order
+  constexpr bool kXPerm = kXP && kPerm;                // a separate stored-order copy is built
   constexpr int W = gemv_warps(MT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BD = g.b_d, BR = 10 - BD;
@@ -222,17 +233,22 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   const int uf = min(u1, un.ufull);                      // full-tile units [u0, uf), partial-tile blocks [max(u0, ufull), u1)
   const int nfull = max(0, uf - u0);
 
-  // Shared memory: codebook replicas, then (x_smem) x in natural order [MT][K],
-  // then per warp two x slots (double buffer) of MT rows x 128 columns fp16 (a
-  // full-tile unit uses its first 32 columns), then [W][npw][MT][128] parked
-  // sums, the W + 1 range boundaries and the W ranges' first tiles (36 ints), and
-  // one completion counter per tile of the CTA's range.
+  // Shared memory: codebook replicas, then (kXS) x in natural order [MT][K],
+  // then (kXPerm) x in stored order [MT][K], then (kXM < 2) per warp two x slots
+  // (double buffer) of MT rows x 128 columns fp16 (a full-tile unit uses its
+  // first 32 columns), then [W][npw][MT][128] parked sums, the W + 1 range
+  // boundaries and the W ranges' first tiles (36 ints), and one completion
+  // counter per tile of the CTA's range.
   uint4* cbs = reinterpret_cast<uint4*>(smem);
   constexpr int kXSlot = MT * kBlockCols * 2;          // bytes per x slot
-  constexpr int kXStride = kBlockCols * 2;             // token stride inside a slot
-  unsigned char* xn = smem + ((size_t)16 * R << BD);   // x in natural column order (x_smem)
-  unsigned char* xs = xn + (kXS ? (size_t)MT * K * 2 : 0) + (size_t)warp * 2 * kXSlot;
-  float* red = reinterpret_cast<float*>(xn + (kXS ? (size_t)MT * K * 2 : 0) + (size_t)W * 2 * kXSlot);
+  const size_t xbytes = (size_t)MT * K * 2;            // one staged copy of x
+  unsigned char* xn = smem + ((size_t)16 * R << BD);   // x in natural column order (kXS)
+  unsigned char* xp = kXPerm ? xn + xbytes : xn;       // x in stored column order (kXP)
+  unsigned char* xs_all = xn + (kXS ? xbytes : 0) + (kXPerm ? xbytes : 0);
+  unsigned char* xs = xs_all + (kXP ? 0 : (size_t)warp * 2 * kXSlot);
+  // token stride of the x operand the decode reads: a slot row, or a staged row of K columns
+  const int xstride = kXP ? 2 * K : kBlockCols * 2;
+  float* red = reinterpret_cast<float*>(xs_all + (kXP ? 0 : (size_t)W * 2 * kXSlot));
   int* rbt = reinterpret_cast<int*>(red + (size_t)W * npw * MT * kTileRows);
   int* tcnt = rbt + 36;
   for (int i = threadIdx.x; i <= tb - ta; i += blockDim.x) tcnt[i] = 0;
@@ -296,12 +312,35 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   }
   const int col0 = nfull > 0 ? 32 * (u0 - 4 * B * t) + lane : 0;
   int pj0 = 0, pj1 = 0;                                // x index of units u0 and u0+1
-  if constexpr (kPerm) {
-    if (nfull > 0) pj0 = ldg_keep_i32(g.perm + col0, pol_keep);
-    if (nfull > 1) pj1 = ldg_keep_i32(g.perm + col1, pol_keep);
-  } else {
-    pj0 = col0;
-    pj1 = col1;
+  if constexpr (!kXP) {
+    if constexpr (kPerm) {
+      if (nfull > 0) pj0 = ldg_keep_i32(g.perm + col0, pol_keep);
+      if (nfull > 1) pj1 = ldg_keep_i32(g.perm + col1, pol_keep);
+    } else {
+      pj0 = col0;
+      pj1 = col1;
+    }
+  }
+  // Stored-order staging (kXPerm): the permutation is weight data, so its first
+  // kPP groups of four entries per thread are loaded before the dependency wait.
+  constexpr int kPP = 8;
+  const int nq = K >> 2;                               // groups of four columns
+  const bool pvec = (reinterpret_cast<uintptr_t>(g.perm) & 15) == 0;
+  auto load_perm4 = [&](int i) -> int4 {
+    if (pvec) {
+      const uint4 v = ldg_keep_v4(reinterpret_cast<const uint4*>(g.perm) + i, pol_keep);
+      return make_int4((int)v.x, (int)v.y, (int)v.z, (int)v.w);
+    }
+    return make_int4(ldg_keep_i32(g.perm + 4 * i, pol_keep), ldg_keep_i32(g.perm + 4 * i + 1, pol_keep),
+                     ldg_keep_i32(g.perm + 4 * i + 2, pol_keep), ldg_keep_i32(g.perm + 4 * i + 3, pol_keep));
+  };
+  int4 pv[kXPerm ? kPP : 1];
+  if constexpr (kXPerm) {
+#pragma unroll
+    for (int k = 0; k < kPP; ++k) {
+      const int i = threadIdx.x + k * blockDim.x;
+      pv[k] = i < nq ? load_perm4(i) : make_int4(0, 0, 0, 0);
+    }
   }
   // The activations may be written by the previous kernel in the stream
   // (programmatic dependent launch): wait for it before reading x.
@@ -367,6 +406,30 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       for (int q = 0; q < R; ++q) cbs[e * R + ((q + e) & (R - 1))] = cbv[k];
   }
   __syncthreads();
+  if constexpr (kXPerm) {
+    // x in stored order: column j of token m is x[m][perm[j]] (an entry outside
+    // 0..K-1, which a permutation never holds, reads column 0)
+    auto permute4 = [&](int i, int4 p) {
+      const uint32_t ku = (uint32_t)K;
+      const int j0 = (uint32_t)p.x < ku ? p.x : 0, j1 = (uint32_t)p.y < ku ? p.y : 0;
+      const int j2 = (uint32_t)p.z < ku ? p.z : 0, j3 = (uint32_t)p.w < ku ? p.w : 0;
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint16_t* xr = reinterpret_cast<const uint16_t*>(xn + (size_t)m * K * 2);
+        uint2 w;
+        w.x = (uint32_t)xr[j0] | ((uint32_t)xr[j1] << 16);
+        w.y = (uint32_t)xr[j2] | ((uint32_t)xr[j3] << 16);
+        *reinterpret_cast<uint2*>(xp + (size_t)m * K * 2 + 8 * (size_t)i) = w;
+      }
+    };
+#pragma unroll
+    for (int k = 0; k < kPP; ++k) {
+      const int i = threadIdx.x + k * blockDim.x;
+      if (i < nq) permute4(i, pv[k]);
+    }
+    for (int i = threadIdx.x + kPP * blockDim.x; i < nq; i += blockDim.x) permute4(i, load_perm4(i));
+    __syncthreads();
+  }
   // activations of one x column for every token: from the staged copy or global memory
   auto gather_x = [&](int pj, uint16_t (&h)[MT]) {
 #pragma unroll
@@ -377,9 +440,9 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   };
   auto put_x = [&](unsigned char* slot, const uint16_t (&h)[MT]) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m) reinterpret_cast<uint16_t*>(slot + m * kXStride)[lane] = h[m];
+    for (int m = 0; m < MT; ++m) reinterpret_cast<uint16_t*>(slot + m * xstride)[lane] = h[m];
   };
-  if (nfull > 0) {
+  if (!kXP && nfull > 0) {
     uint16_t h0[MT];
     gather_x(pj0, h0);
     put_x(xs, h0);
@@ -416,6 +479,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       for (int h = 0; h < 2; ++h) bm[i][h] = ((lane >> 3) == i && ((lane >> 2) & 1) == h) ? 0xFFFFFFFFu : 0u;
     const uint32_t xw_off = 16u * ((lane >> 2) & 1) + 4u * (lane & 3);
     int tile_end = un.tile_u1(t);                      // first unit of the next tile
+    uint32_t xo = 64u * (uint32_t)(u0 - un.tile_u0(t)); // (kXP) byte offset of unit i's 32 columns in x
     if (nfull > 4) {                                   // L2 prefetch of the second block of the range
       const uint8_t* pb = g.packed + (size_t)((u0 >> 2) + 1) * 4608;
       prefetch_l2(pb + lane * 128);
@@ -427,7 +491,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       constexpr bool kMore = decltype(more_tag)::value;
       const int u = u0 + i;
       const bool new_block = ((u + 1) & 3) == 0, new_tile = u + 1 == tile_end;
-      int pj2 = 0;                                     // x index of unit i+2
+      [[maybe_unused]] int pj2 = 0;                    // x index of unit i+2 (kXM < 2)
       if constexpr (kMore) {
         load_unit(nxt, u + 1);
         if (new_block) {
@@ -440,14 +504,17 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
           }
         }
         if (new_tile) load_radius(t + 1);
-        if (i + 2 < nfull) {
-          if constexpr (kPerm) pj2 = ldg_keep_i32(g.perm + col2, pol_keep);
-          else pj2 = col2;
+        if constexpr (!kXP) {
+          if (i + 2 < nfull) {
+            if constexpr (kPerm) pj2 = ldg_keep_i32(g.perm + col2, pol_keep);
+            else pj2 = col2;
+          }
         }
       }
       const int A = u & 3;
       const uint32_t p5 = A == 0 ? c8.x : (A == 1 ? c8.y : (A == 2 ? c8.z : c8.w));
-      frag_quarter<MT>(cur.s, cur.p, p5, xs + (i & 1) * kXSlot, kXStride, cb_base_q, fk, bm, xw_off, scp, ofp, acc);
+      const unsigned char* xq = kXP ? xp + xo : xs + (i & 1) * kXSlot;
+      frag_quarter<MT>(cur.s, cur.p, p5, xq, xstride, cb_base_q, fk, bm, xw_off, scp, ofp, acc);
       if constexpr (kMore) {
         if (new_tile) {
           park(t);
@@ -455,13 +522,17 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
           tile_end = un.tile_u1(t);
           radius_pairs(sc, of);
         }
-        uint16_t h[MT];
-        gather_x(pj1, h);
-        __syncwarp();                                  // all lanes done reading the slot about to be reused
-        put_x(xs + ((i + 1) & 1) * kXSlot, h);
-        __syncwarp();
-        pj1 = pj2;
-        col2 = col2 + 32 < K ? col2 + 32 : col2 + 32 - K;
+        if constexpr (kXP) {
+          xo = new_tile ? 0u : xo + 64u;
+        } else {
+          uint16_t h[MT];
+          gather_x(pj1, h);
+          __syncwarp();                                // all lanes done reading the slot about to be reused
+          put_x(xs + ((i + 1) & 1) * kXSlot, h);
+          __syncwarp();
+          pj1 = pj2;
+          col2 = col2 + 32 < K ? col2 + 32 : col2 + 32 - K;
+        }
         if (new_block) c8 = c8n;
       } else {
         park(t);
@@ -499,18 +570,21 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
     if (lane < L) load_block(d0, tbase + (size_t)kb0 * L * kLaneBlockBytes, L, lane, pol_stream);
     for (int k2 = kb0; k2 < kb1; ++k2) {
       if (k2 + 1 < kb1 && lane < L) load_block(d1, tbase + (size_t)(k2 + 1) * L * kLaneBlockBytes, L, lane, pol_stream);
-      __syncwarp();
+      if constexpr (!kXP) {
+        __syncwarp();
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int col = k2 * kBlockCols + lane + 32 * j;
-        const int pc = kPerm ? ldg_keep_i32(g.perm + col, pol_keep) : col;
-        uint16_t h[MT];
-        gather_x(pc, h);
+        for (int j = 0; j < 4; ++j) {
+          const int col = k2 * kBlockCols + lane + 32 * j;
+          const int pc = kPerm ? ldg_keep_i32(g.perm + col, pol_keep) : col;
+          uint16_t h[MT];
+          gather_x(pc, h);
 #pragma unroll
-        for (int m = 0; m < MT; ++m) reinterpret_cast<uint16_t*>(xs + m * kXStride)[lane + 32 * j] = h[m];
+          for (int m = 0; m < MT; ++m) reinterpret_cast<uint16_t*>(xs + m * xstride)[lane + 32 * j] = h[m];
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      if (lane < L) process_block<MT>(d0, xs, kXStride, cbb, q16, cs_, CODEM, scp, ofp, acc);
+      const unsigned char* xb = kXP ? xp + (size_t)k2 * kBlockCols * 2 : xs;
+      if (lane < L) process_block<MT>(d0, xb, xstride, cbb, q16, cs_, CODEM, scp, ofp, acc);
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     }
@@ -519,9 +593,10 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 }
 
 // PM: 1 = every matrix of the launch has a permutation, 0 = none has, 2 = mixed
-// (each CTA follows its own matrix).  The uniform cases get kernels of their own
-// so each is compiled (registers, schedule) for one path only.
-template <int MT, int PM>
+// (each CTA follows its own matrix).  XM: where every CTA of the launch keeps x
+// (kXM of gemv_cta).  The uniform cases get kernels of their own so each is
+// compiled (registers, schedule) for one path only.
+template <int MT, int PM, int XM>
 __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
 gemv_kernel(const __grid_constant__ GemvKParams P) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -529,36 +604,23 @@ gemv_kernel(const __grid_constant__ GemvKParams P) {
   while (mi + 1 < P.n_mats && (int)blockIdx.x >= P.mats[mi + 1].cta_begin) ++mi;
   const GemvKMat& g = P.mats[mi];
   const int c = (int)blockIdx.x - g.cta_begin;
-  // x staged in shared memory (every matrix of a launch decides alike unless
-  // shared memory ran short for one of them)
-  if constexpr (PM == 1) {
-    if (g.x_smem) gemv_cta<MT, true, true>(g, c, smem, P.y_f32, P.one);
-    else gemv_cta<MT, true, false>(g, c, smem, P.y_f32, P.one);
-  } else if constexpr (PM == 0) {
-    if (g.x_smem) gemv_cta<MT, false, true>(g, c, smem, P.y_f32, P.one);
-    else gemv_cta<MT, false, false>(g, c, smem, P.y_f32, P.one);
-  } else {
-    if (g.perm) {
-      if (g.x_smem) gemv_cta<MT, true, true>(g, c, smem, P.y_f32, P.one);
-      else gemv_cta<MT, true, false>(g, c, smem, P.y_f32, P.one);
-    } else {
-      if (g.x_smem) gemv_cta<MT, false, true>(g, c, smem, P.y_f32, P.one);
-      else gemv_cta<MT, false, false>(g, c, smem, P.y_f32, P.one);
-    }
-  }
+  if constexpr (PM == 1) gemv_cta<MT, true, XM>(g, c, smem, P.y_f32, P.one);
+  else if constexpr (PM == 0) gemv_cta<MT, false, XM>(g, c, smem, P.y_f32, P.one);
+  else if (g.perm) gemv_cta<MT, true, XM>(g, c, smem, P.y_f32, P.one);
+  else gemv_cta<MT, false, XM>(g, c, smem, P.y_f32, P.one);
 }
 
-template <int MT, int PM>
+template <int MT, int PM, int XM>
 cudaError_t launch_gemv_pm(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
-  static unsigned long long attr_set = 0;       // one bit per device
+  static std::atomic<unsigned long long> attr_set{0};   // one bit per device (setting it twice is harmless)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 64 || !((attr_set >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(gemv_kernel<MT, PM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (dev >= 64 || !((attr_set.load(std::memory_order_acquire) >> dev) & 1ull)) {
+    e = cudaFuncSetAttribute(gemv_kernel<MT, PM, XM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kGemvSmemMax);
     if (e != cudaSuccess) return e;
-    if (dev < 64) attr_set |= 1ull << dev;
+    if (dev < 64) attr_set.fetch_or(1ull << dev, std::memory_order_release);
   }
   // Programmatic dependent launch: the kernel's weight-only prologue may overlap
   // the tail of the previous kernel in the stream (it waits for that kernel
@@ -573,20 +635,31 @@ cudaError_t launch_gemv_pm(const GemvKParams& p, int grid, size_t smem, cudaStre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT, PM>, p);
+  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT, PM, XM>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
-template <int MT>
-cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
+template <int MT, int XM>
+cudaError_t launch_gemv_xm(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
   int with = 0;
   for (int i = 0; i < p.n_mats; ++i) with += p.mats[i].perm != nullptr;
-  if (with == p.n_mats) return launch_gemv_pm<MT, 1>(p, grid, smem, st);
-  if (with == 0) return launch_gemv_pm<MT, 0>(p, grid, smem, st);
-  return launch_gemv_pm<MT, 2>(p, grid, smem, st);
+  if (with == p.n_mats) return launch_gemv_pm<MT, 1, XM>(p, grid, smem, st);
+  if (with == 0) return launch_gemv_pm<MT, 0, XM>(p, grid, smem, st);
+  return launch_gemv_pm<MT, 2, XM>(p, grid, smem, st);
+}
+
+template <int MT>
+cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
+  // every matrix of a launch keeps x alike (the planner makes it so)
+  const int xm = p.mats[0].x_smem;
+  for (int i = 1; i < p.n_mats; ++i)
+    if (p.mats[i].x_smem != xm) return cudaErrorInvalidValue;
+  if (xm == 2) return launch_gemv_xm<MT, 2>(p, grid, smem, st);
+  if (xm == 1) return launch_gemv_xm<MT, 1>(p, grid, smem, st);
+  return launch_gemv_xm<MT, 0>(p, grid, smem, st);
 }
 
 }  // namespace svq

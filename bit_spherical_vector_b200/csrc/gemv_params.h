@@ -22,7 +22,8 @@ struct GemvKMat {
   unsigned* counters;     // [n_tiles]
   int N, K, b_d, M;
   int ctas, cta_begin, kmax, npw;
-  int x_smem;             // 1: the CTA stages x (natural order, MT rows) in shared memory
+  int x_smem;             // where a CTA keeps x: 2 shared memory, natural and stored order
+                          // (the decode reads the stored order); 1 natural order only; 0 none
 };
 
 struct GemvKParams {

@@ -63,7 +63,9 @@ struct GemvPlanMat {
   int npw;                               // most tiles that one warp's range touches
   int counter0;                          // first counter of this matrix's tiles
   size_t part_offset, part_bytes;        // partial sums [n_tiles][kmax][mt][128] (kmax > 1)
-  int x_smem;                            // x staged in shared memory by every CTA of the matrix
+  int x_smem;                            // x in shared memory: 2 natural + stored order, 1 natural, 0 none
+                                         // (the same for every matrix of a launch)
+  int ntc;                               // most tiles that one CTA's range touches
 };
 
 struct GemvPlan {

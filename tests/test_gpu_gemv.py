@@ -197,3 +197,25 @@ def test_lm_head_sized_matrix_sampled_rows():
                               m.perm)
         y_ref, den = oracle.linear(sub, x)
         assert rel_err(y[:, r0:r0 + 4], y_ref, den) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 2, 5])
+@pytest.mark.parametrize("N", [9728, 9660])
+def test_grouped_stored_order_staging(N, M):
+    """Two N x 2560 matrices with permutations in one grouped call: every CTA's range covers more than
+    one 128-row tile of units, so each CTA stages x in stored order once and the decode reads its
+    operands from that copy (N = 9660 adds a 60-row last tile).  Every output against the oracle."""
+    need_gpu()
+    K = 2560
+    mats = [synth.make_matrix(68, i + N % 7, N, K, 7 + i) for i in range(2)]
+    xs = [synth.make_x(68, 20 + i, M, K) for i in range(2)]
+    Ws = [svq.SvqWeight.from_synth(m) for m in mats]
+    nb = svq.svq_linear_gemv_batched_workspace_size(Ws, M)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+    svq.svq_workspace_init(ws)
+    ys = [torch.empty((M, N), dtype=torch.float32, device="cuda") for _ in mats]
+    svq.svq_linear_gemv_batched(Ws, [x_f16(x) for x in xs], ys, ws)
+    torch.cuda.synchronize()
+    for m, x, y in zip(mats, xs, ys):
+        y_ref, den = oracle.linear(m, x)
+        assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL

@@ -59,3 +59,37 @@ def test_noalloc_rejects_scratch_beyond_limit():
     assert svq.lib().svq_linear_gemv_workspace_size(ctypes.byref(desc), 8, ctypes.byref(n)) == svq.SVQ_OK
     assert n.value > LIMIT
     assert _noalloc(desc, 0x60000, 8, 0x70000) == svq.SVQ_ERR_WORKSPACE
+
+
+def _ptr_y(y):
+    return svq.SVQ_F16 if y.dtype == torch.float16 else svq.SVQ_F32
+
+
+@pytest.mark.parametrize("stored", [False, True])
+def test_noalloc_against_oracle_m12_fp16_out(stored):
+    """9728 x 2560, M = 12 (two passes of 8 and 4 tokens), fp16 output, against the oracle; with
+    stored=True the matrix is called with perm NULL and x already in stored column order."""
+    need_gpu()
+    import oracle
+    N, K, M, b_d = 9728, 2560, 12, 7
+    m = synth.make_matrix(98, 12, N, K, b_d)
+    W = svq.SvqWeight.from_synth(m)
+    x_bits = synth.make_x(98, 13, M, K)
+    x = x_f16(x_bits)
+    if stored:
+        W = W.without_perm()
+        x = x[:, torch.from_numpy(m.perm.astype(np.int64)).cuda()].contiguous()
+    nb = svq.svq_linear_gemv_workspace_size(W, M)
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+    rc = svq.lib().svq_linear_gemv_noalloc(ctypes.byref(W.desc), ctypes.c_void_p(x.data_ptr()), M,
+                                           ctypes.c_void_p(y.data_ptr()), _ptr_y(y),
+                                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if nb > LIMIT:
+        assert rc == svq.SVQ_ERR_WORKSPACE
+        return
+    assert rc == svq.SVQ_OK
+    torch.cuda.synchronize()
+    y_ref, den = oracle.linear(m, x_bits)
+    got = y.float().cpu().numpy().astype(np.float64)
+    # fp16 output: add the output rounding (half an ulp of |y_ref|, 2^-11 relative) to the bound
+    assert np.all(np.abs(got - y_ref) <= TOL * den + np.abs(y_ref) * 2.0 ** -11)
