@@ -22,7 +22,10 @@ readings taken here (each the plainest one the captions support):
   brute-force encoder picks; the first candidate wins a tie;
 * radius grid (an input to ABS, not fixed by the pages, which optimise the
   radius levels blockwise): uniform between the smallest and largest subvector
-  norm of each row, scale and offset rounded to fp16.
+  norm of each row, scale and offset rounded to fp16;
+* sums whose order the pages leave open (channel energies over calibration
+  rows, a subvector's squared norm over its elements) run in ascending index
+  order in fp64, one rounding per operation.
 """
 from __future__ import annotations
 
@@ -34,9 +37,17 @@ from . import decode_exact, encode, f64_to_h_rne, h2f, pack
 
 
 def channel_energy(x_cal) -> np.ndarray:
-    """e_k = (1/T) sum_t x[t][k]^2 in fp64 for calibration activations x_cal [T][K] (float values)."""
+    """e_k = (1/T) sum_t x[t][k]^2 in fp64 for calibration activations x_cal [T][K] (float values).
+
+    The sum runs over t in ascending order, one rounding per addition, then one
+    division by T: a fixed order, so that another implementation can reproduce
+    the value exactly."""
     x = np.asarray(x_cal, np.float64)
-    return np.mean(x * x, axis=0)
+    T = x.shape[0]
+    s = x[0] * x[0]
+    for t in range(1, T):
+        s = s + x[t] * x[t]
+    return s / float(T)
 
 
 def esg_weights(energy, gamma: float) -> np.ndarray:
@@ -62,7 +73,12 @@ def radius_grid(W_stored, b_d: int):
     """Per-row uniform radius grid over the row's subvector norms: fp16 (scale, offset) bit patterns [N]."""
     W = np.asarray(W_stored, np.float64)
     N, K = W.shape
-    norms = np.sqrt((W.reshape(N, K // 8, 8) ** 2).sum(axis=2))
+    sub = W.reshape(N, K // 8, 8)
+    # squared norm summed over the eight elements in element order (fixed order, see channel_energy)
+    sq = sub[:, :, 0] * sub[:, :, 0]
+    for i in range(1, 8):
+        sq = sq + sub[:, :, i] * sub[:, :, i]
+    norms = np.sqrt(sq)
     lo, hi = norms.min(axis=1), norms.max(axis=1)
     levels = (1 << (10 - b_d)) - 1
     scale = (hi - lo) / levels if levels > 0 else np.zeros(N)
