@@ -75,6 +75,10 @@ def lib():
         "svq_rmsnorm_permute": ([P, I, P, ctypes.c_float, I, I, ctypes.POINTER(P), ctypes.POINTER(P), I, P], I),
         "svq_swiglu_permute": ([P, P, I, I, P, P, P], I),
         "svq_get_device_status": ([P], I),
+        "svq_esg": ([P, I, I, ctypes.c_double, P, P, P, P], I),
+        "svq_radius_grid": ([P, I, I, P, I, P, P, P], I),
+        "svq_encode": ([P, I, I, I, P, P, P, P, P, P, P, P], I),
+        "svq_abs_select": ([P, I, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -308,6 +312,37 @@ def svq_swiglu_permute(gate, up, perm, x, stream=None):
     M, I = gate.shape
     _check(lib().svq_swiglu_permute(_ptr(gate), _ptr(up), M, I, _ptr(perm), _ptr(x), _stream(stream)),
            "svq_swiglu_permute")
+
+
+# ------------------------------------------------------------------ calibration (ESG, radius grid, encoder, ABS)
+def svq_esg(x_cal, gamma, energy, perm, weights=None, stream=None):
+    """Channel energies (fp64 [K]), the ESG permutation (int32 [K]) and fitting weights e^gamma (fp32 [K] or None)
+    from calibration activations x_cal (fp32 [T][K])."""
+    T, K = x_cal.shape
+    _check(lib().svq_esg(_ptr(x_cal), T, K, float(gamma), _ptr(energy), _ptr(perm), _ptr(weights), _stream(stream)),
+           "svq_esg")
+
+
+def svq_radius_grid(W, perm, b_d, scale, offset, stream=None):
+    """Per-row uniform radius grid (fp16 bit patterns scale/offset [N], as int16/uint16 tensors) of W (fp32 [N][K])."""
+    N, K = W.shape
+    _check(lib().svq_radius_grid(_ptr(W), N, K, _ptr(perm), int(b_d), _ptr(scale), _ptr(offset), _stream(stream)),
+           "svq_radius_grid")
+
+
+def svq_encode(W, b_d, perm, weights, codebook, scale, offset, canonical, row_err=None, stream=None):
+    """Activation-weighted SVQ encoding of W (fp32 [N][K], natural column order) into the canonical stream
+    (uint8 [N][row_bytes]); row_err (fp64 [N]) receives each row's weighted reconstruction error."""
+    N, K = W.shape
+    _check(lib().svq_encode(_ptr(W), N, K, int(b_d), _ptr(perm), _ptr(weights), _ptr(codebook), _ptr(scale),
+                            _ptr(offset), _ptr(canonical), _ptr(row_err), _stream(stream)), "svq_encode")
+
+
+def svq_abs_select(row_err, totals, best, stream=None):
+    """ABS: totals[k] = sum of row_err[k] (fp64 [n_cand][N]) and best[0] = the first least total (int32)."""
+    n_cand, N = row_err.shape
+    _check(lib().svq_abs_select(_ptr(row_err), n_cand, N, _ptr(totals), _ptr(best), _stream(stream)),
+           "svq_abs_select")
 
 
 def svq_get_device_status(stream=None) -> int:

@@ -359,6 +359,44 @@ int svq_swiglu_permute(const float* gate, const float* up, int M, int I, const i
   return cuda_status(svq::launch_swiglu_permute(gate, up, M, I, perm, x, (cudaStream_t)stream));
 }
 
+int svq_esg(const float* x_cal, int T, int K, double gamma, double* energy, int32_t* perm, float* weights,
+            svq_stream_t stream) {
+  if (T < 1 || K < 8 || K % 8 != 0) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!x_cal || !energy || !perm) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(x_cal, 4) || !aligned(energy, 8) || !aligned(perm, 4) || (weights && !aligned(weights, 4)))
+    return SVQ_ERR_INVALID_ARG;
+  if (!(gamma == gamma)) return SVQ_ERR_INVALID_ARG;               // NaN exponent
+  return cuda_status(svq::launch_esg(x_cal, T, K, gamma, energy, perm, weights, (cudaStream_t)stream));
+}
+
+int svq_radius_grid(const float* W, int N, int K, const int32_t* perm, int b_d, uint16_t* scale, uint16_t* offset,
+                    svq_stream_t stream) {
+  if (N < 1 || K < 8 || K % 8 != 0 || b_d < 1 || b_d > 10) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!W || !scale || !offset) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(scale, 2) || !aligned(offset, 2) || (perm && !aligned(perm, 4)))
+    return SVQ_ERR_INVALID_ARG;
+  return cuda_status(svq::launch_radius_grid(W, N, K, perm, b_d, scale, offset, (cudaStream_t)stream));
+}
+
+int svq_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
+               const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset, uint8_t* canonical,
+               double* row_err, svq_stream_t stream) {
+  if (N < 1 || K < 8 || K % 8 != 0 || b_d < 1 || b_d > 10) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!W || !codebook || !scale || !offset || !canonical) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(codebook, 2) || !aligned(scale, 2) || !aligned(offset, 2) ||
+      (perm && !aligned(perm, 4)) || (weights && !aligned(weights, 4)) || (row_err && !aligned(row_err, 8)))
+    return SVQ_ERR_INVALID_ARG;
+  return cuda_status(svq::launch_encode(W, N, K, b_d, perm, weights, codebook, scale, offset, canonical, row_err,
+                                        (cudaStream_t)stream));
+}
+
+int svq_abs_select(const double* row_err, int n_cand, int N, double* totals, int32_t* best, svq_stream_t stream) {
+  if (n_cand < 1 || n_cand > svq::kAbsMaxCandidates || N < 1) return SVQ_ERR_INVALID_ARG;
+  if (!row_err || !best || !aligned(row_err, 8) || !aligned(best, 4) || (totals && !aligned(totals, 8)))
+    return SVQ_ERR_INVALID_ARG;
+  return cuda_status(svq::launch_abs_select(row_err, n_cand, N, totals, best, (cudaStream_t)stream));
+}
+
 unsigned svq_debug_set_wait_polls(unsigned polls) { return svq::set_wait_polls(polls); }
 
 int svq_get_device_status(svq_stream_t stream) {

@@ -311,6 +311,66 @@ SVQ_API int svq_swiglu_permute(const float* gate, const float* up, int M, int I,
                                svq_stream_t stream);
 
 /*
+ * Calibration side (offline, before svq_repack): Energy-Stratified Grouping,
+ * the per-row radius grid, the activation-weighted encoder and Adaptive Bit
+ * Split ("SAGE", abstract; Figure 2 caption: signs, direction index and
+ * quantized radius fitted under activation-energy weights; Figure 4(a): the
+ * energy exponent gamma).  The pages give no formulas; the readings are stated
+ * with each call.  Every integer result (permutation, signs, direction indices,
+ * radius codes, the chosen split) is decided from fp64 values computed with one
+ * rounding per operation in a fixed order, so it is reproducible bit for bit.
+ * Inputs must be finite.  All pointers are device pointers; nothing is
+ * allocated; every call is asynchronous on `stream`.
+ *
+ * svq_esg -- channel energies e_k = (sum_t x_cal[t][k]^2) / T (fp64, t
+ * ascending), the ESG permutation and the fitting weights.  The channels are
+ * ordered by energy, highest first (equal energies: lower index first) and cut
+ * into 8 tiers of K/8; stored column 8g + t takes the g-th channel of tier t:
+ * perm[8g + t] = order[t * K/8 + g].  weights[k] = (float) pow(e_k, gamma)
+ * (NULL: not written; pow is CUDA's, within 2 ulp in fp64).
+ * x_cal: fp32 [T][K], 4-byte aligned; energy: fp64 [K] out, 8-byte aligned;
+ * perm: int32 [K] out; weights: fp32 [K] out or NULL.  T >= 1, K a multiple of
+ * 8.  Cost O(K^2) comparisons (ranking).
+ *
+ * svq_radius_grid -- per-row uniform radius grid: with the row's subvector
+ * norms in stored order (W[n][perm[8g..8g+7]], squares summed in element order,
+ * correctly rounded sqrt) and their minimum lo and maximum hi,
+ * offset[n] = fp16(lo) and scale[n] = fp16((hi - lo) / (2^b_r - 1)) (0 when
+ * b_r = 0), each rounded once to nearest even.  W: fp32 [N][K], natural column
+ * order; perm: [K] or NULL (identity).
+ *
+ * svq_encode -- encodes W (fp32 [N][K], natural column order) as the
+ * canonical stream of an SVQ matrix with stored column j = perm[j] (identity
+ * when perm is NULL).  Per subvector (stored columns 8g..8g+7, w = those
+ * weights, e = weights[perm[...]], all 1 when weights is NULL): sign bit
+ * s_i = (w_i < 0); (idx, code) minimises
+ *   X = sum_i e_i (|w_i| - r_code c_idx,i)^2,  r_code = fma(scale[n], code, offset[n]) (fp32)
+ * evaluated term by term in fp64 (i ascending), ties to the lowest idx, then
+ * the lowest code -- the brute-force choice, reached without evaluating every
+ * pair (a filter with a proven error bound skips pairs that cannot win).
+ * codebook: fp16 [2^b_d][8]; scale, offset: fp16 [N]; canonical: [N][row
+ * bytes of svq_canonical_bytes] out, pad bits zero; row_err: fp64 [N] out or
+ * NULL: sum_j e_j (W[n][perm[j]] - What[n][j])^2 over the row (What the exact
+ * decoded weight), per subvector in element order, then in a fixed tree over
+ * each 32 subvectors and in order over those chunks.  1 <= b_d <= 10, K a
+ * multiple of 8.
+ *
+ * svq_abs_select -- Adaptive Bit Split: totals[k] = sum_n row_err[k][n] (fixed
+ * order) for n_cand (1..64) candidate encodings of one matrix (row_err: fp64
+ * [n_cand][N], each written by svq_encode under one split), and *best = the
+ * first candidate with the least total.  totals may be NULL; best: int32 [1].
+ */
+SVQ_API int svq_esg(const float* x_cal, int T, int K, double gamma, double* energy, int32_t* perm, float* weights,
+                    svq_stream_t stream);
+SVQ_API int svq_radius_grid(const float* W, int N, int K, const int32_t* perm, int b_d, uint16_t* scale,
+                            uint16_t* offset, svq_stream_t stream);
+SVQ_API int svq_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
+                       const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset, uint8_t* canonical,
+                       double* row_err, svq_stream_t stream);
+SVQ_API int svq_abs_select(const double* row_err, int n_cand, int N, double* totals, int32_t* best,
+                           svq_stream_t stream);
+
+/*
  * Synchronising read-and-clear of the device status word that kernels set
  * when a bounded wait runs out (SVQ_ERR_TIMEOUT) or a device-side argument
  * check fails (SVQ_ERR_INVALID_ARG); SVQ_OK when neither happened.  Tests only.
