@@ -148,36 +148,43 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
   const uint8_t* cbq = cbs + (lane & (rep - 1)) * 16;
   const int cb_stride = rep * 16;                      // bytes per codebook entry (all replicas)
   // Fields of the lane's subvectors (row 4 * lane + r, group j) of this block:
-  // sign byte, direction index, radius code.
-  uint32_t sgn[2], pidx[2], pcode[2];
+  // sign masks of the four element pairs (bits 15 and 31, ready to XOR onto a
+  // 16-bit pair), direction index, radius code.
+  uint32_t smk[2][4], pidx[2], pcode[2];
   if (L == 32) {
-    // fragment arrangement (full tile): signs from the four sign-holder lanes of
-    // the lane's quad, the index from its address lane, the code from itself
-    auto wordl = [&](int l, int wi) -> uint32_t {
-      return *reinterpret_cast<const uint32_t*>(pk + word_offset_in_block(32, l, wi));
-    };
-    auto slot = [&](int l, int u, int k) -> uint32_t {
-      const int pb = frag_slot_bit(u, k);
-      uint32_t P[2];
-      P[0] = wordl(l, frag_payload_word(pb >> 5));
-      P[1] = (pb & 31) > 22 ? wordl(l, frag_payload_word((pb >> 5) + 1)) : 0u;
-      return payload_field(P, pb & 31);
-    };
+    // fragment arrangement (full tile).  The warp's two rows r0, r0 + 1 of
+    // group j belong to one round u of quarter A = j / 4; every field it needs
+    // sits in two places per lane: the round's sign word S_u and the 40 payload
+    // bits of round u (quarter bits [40 (u % 4), 40 (u % 4) + 40), inside the
+    // quarter's payload words w0 and w0 + 1).  Each lane loads its own three
+    // words; the sign holders' words and the address lanes' payload come by
+    // warp shuffles (all 32 lanes take part, also past L).
+    const int u = frag_round(r0, j);
+    const int A = j >> 2, ub = u & 3;
+    const int w0 = (5 * ub) >> 2;                       // 40 * ub / 32
+    const int sh0 = 40 * ub - 32 * w0;                  // bit of the round's field 0 in (P[w0], P[w0+1])
+    const uint32_t Sown = *reinterpret_cast<const uint32_t*>(pk + word_offset_in_block(32, lane, frag_sign_word(u)));
+    const uint32_t Plo = *reinterpret_cast<const uint32_t*>(
+        pk + word_offset_in_block(32, lane, frag_payload_word(5 * A + w0)));
+    const uint32_t Phi = *reinterpret_cast<const uint32_t*>(
+        pk + word_offset_in_block(32, lane, frag_payload_word(5 * A + w0 + 1)));
+    const unsigned long long Pown = ((unsigned long long)Phi << 32) | Plo;
+    uint32_t Sq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) Sq[q] = __shfl_sync(0xFFFFFFFFu, Sown, frag_sign_lane(lane, q));
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int r = r0 + rr;
-      const int u = frag_round(r, j);
-      pcode[rr] = (slot(lane, u, frag_code_slot(r, j)) >> bd) & cmask;
-      pidx[rr] = slot(frag_addr_lane(lane, r, j), u, frag_addr_slot(lane)) & imask;
+      const int la = frag_addr_lane(lane, r, j);
+      const uint32_t alo = __shfl_sync(0xFFFFFFFFu, Plo, la), ahi = __shfl_sync(0xFFFFFFFFu, Phi, la);
+      const unsigned long long Pa = ((unsigned long long)ahi << 32) | alo;
+      pcode[rr] = ((uint32_t)(Pown >> (sh0 + 10 * frag_code_slot(r, j))) >> bd) & cmask;
+      pidx[rr] = (uint32_t)(Pa >> (sh0 + 10 * frag_addr_slot(lane))) & imask;
+      // the sign holder's word shifted left by the subvector's position puts the
+      // pair's two signs on bits 15 and 31
       const int ww = frag_sign_pos(lane, r, j);
-      uint32_t sg = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t S = wordl(frag_sign_lane(lane, q), frag_sign_word(u));
-        sg |= ((S >> (15 - ww)) & 1u) << (2 * q);
-        sg |= ((S >> (31 - ww)) & 1u) << (2 * q + 1);
-      }
-      sgn[rr] = sg;
+      for (int q = 0; q < 4; ++q) smk[rr][q] = (Sq[q] << ww) & 0x80008000u;
     }
   } else {
     // owner arrangement (partial tile): everything in the lane's own words
@@ -213,14 +220,8 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
       }
       pidx[rr] = pay & imask;
       pcode[rr] = (pay >> bd) & cmask;
-      uint32_t sg = 0;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int t = 4 * r + q;
-        sg |= ((S >> (15 - t)) & 1u) << (2 * q);
-        sg |= ((S >> (31 - t)) & 1u) << (2 * q + 1);
-      }
-      sgn[rr] = sg;
+      for (int q = 0; q < 4; ++q) smk[rr][q] = (S << (4 * r + q)) & 0x80008000u;
     }
   }
 #pragma unroll
@@ -238,8 +239,7 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
     for (int q = 0; q < 4; ++q) {
       const float2 cf = __half22float2(*reinterpret_cast<const __half2*>(&c4[q]));
       const float2 pr = __fmul2_rn(rad2, cf);               // binary32 products r * c
-      const uint32_t sm = (((sgn[rr] >> (2 * q)) & 1u) << 15) | (((sgn[rr] >> (2 * q + 1)) & 1u) << 31);
-      o4[q] = pack2<BF16>(pr.x, pr.y) ^ sm;
+      o4[q] = pack2<BF16>(pr.x, pr.y) ^ smk[rr][q];
     }
     const int rho = lane + 32 * r;                       // A-tile row of weight row 4 * lane + r
     uint8_t* dst = a_tile + (rho >> 3) * 1024 + (rho & 7) * 128 + ((kc ^ (rho & 7)) << 4);
@@ -448,14 +448,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c0, v);
         tmem_ld_wait();
-        const int nl = 4 * lane + q;         // weight row of TMEM lane 32q + lane
+        // weight row 4 * lane + q (TMEM lane 32q + lane) is staged at position
+        // 4 * lane + (q ^ x), x = (lane / 8) % 4: the lanes of a store that
+        // share a bank (lane, lane + 8, ...) get different offsets, so the
+        // stores are conflict free; the reader undoes the swizzle in registers
+        const int xs = (lane >> 3) & 3;
+        const int nl = 4 * lane + (q ^ xs);
 #pragma unroll
         for (int i = 0; i < 32; ++i) stg[i * 128 + nl] = __uint_as_float(v[i]);
         named_bar_sync(1, kNumEpi * 32);
         for (int i = e * 8; i < e * 8 + 8; ++i) {
           const int m = w.mt * BN + c0 + i;
           if (m >= p.M || 4 * lane >= rows) continue;
-          const float4 val = *reinterpret_cast<const float4*>(stg + i * 128 + 4 * lane);
+          const float4 raw = *reinterpret_cast<const float4*>(stg + i * 128 + 4 * lane);
+          const float rv[4] = {raw.x, raw.y, raw.z, raw.w};
+          auto pick = [&](int t) -> float {                // rv[t ^ xs] without dynamic indexing
+            const int k = t ^ xs;
+            return k == 0 ? rv[0] : (k == 1 ? rv[1] : (k == 2 ? rv[2] : rv[3]));
+          };
+          const float4 val = make_float4(pick(0), pick(1), pick(2), pick(3));
           const int n = n0 + 4 * lane;
           if (split) {
             float* dst = p.partial + ((size_t)w.s * p.M + m) * p.N + n;
