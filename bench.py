@@ -486,7 +486,7 @@ def run_gpu(args, world, rank, local):
     if world == 1 and not args.no_secondary:
         del g_all, g_one
         line["secondary"] = {"sweep_8192": run_sweep(args, quiet=True), "prefill": run_prefill(args, quiet=True),
-                             "moe": run_moe(args, quiet=True)}
+                             "moe": run_moe(args, quiet=True), "calibration": run_calib(args, quiet=True)}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -650,6 +650,59 @@ def run_moe(args, quiet=False):
     return recs if quiet else 0
 
 
+def run_calib(args, quiet=False):
+    """Calibration side on one gate-projection-shaped matrix (9728 x 2560): ESG from 512 calibration rows,
+    then for each candidate split b_d 6..9 the radius grid and the activation-weighted encode, then ABS.
+    Each step timed with CUDA events (median of 3)."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    N, K, T = 9728, 2560, 512
+    rng = np.random.default_rng(7)
+    W = torch.from_numpy((rng.standard_normal((N, K)) * 0.02).astype(np.float32)).cuda()
+    x = torch.from_numpy((rng.standard_normal((T, K)) * rng.lognormal(0.0, 1.0, K)[None, :]).astype(np.float32)).cuda()
+    energy = torch.empty(K, dtype=torch.float64, device="cuda")
+    perm = torch.empty(K, dtype=torch.int32, device="cuda")
+    wts = torch.empty(K, dtype=torch.float32, device="cuda")
+    splits = (6, 7, 8, 9)
+    cbs = [torch.from_numpy(synth.make_codebook(synth.rng(7, b, synth.F_CODEBOOK), b).view(np.int16)).cuda()
+           for b in splits]
+    sc = [torch.empty(N, dtype=torch.int16, device="cuda") for _ in splits]
+    of = [torch.empty(N, dtype=torch.int16, device="cuda") for _ in splits]
+    canon = [torch.empty((N, synth.canonical_row_bytes(K)), dtype=torch.uint8, device="cuda") for _ in splits]
+    row_err = torch.empty((len(splits), N), dtype=torch.float64, device="cuda")
+    totals = torch.empty(len(splits), dtype=torch.float64, device="cuda")
+    best = torch.empty(1, dtype=torch.int32, device="cuda")
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        out = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1) * 1e3)
+        return float(np.median(out))
+
+    rec = {"workload": "calibration 9728x2560 (gate shape), 512 calibration rows, splits b_d 6..9",
+           "esg_us": round(timed(lambda: svq.svq_esg(x, 0.5, energy, perm, wts)), 1), "splits": []}
+    nsub = N * K // 8
+    for i, b in enumerate(splits):
+        g_us = timed(lambda: svq.svq_radius_grid(W, perm, b, sc[i], of[i]))
+        e_us = timed(lambda: svq.svq_encode(W, b, perm, wts, cbs[i], sc[i], of[i], canon[i], row_err[i]))
+        rec["splits"].append({"b_d": b, "radius_grid_us": round(g_us, 1), "encode_us": round(e_us, 1),
+                              "encode_Msubvectors_per_s": round(nsub / e_us, 1)})
+    rec["abs_select_us"] = round(timed(lambda: svq.svq_abs_select(row_err, totals, best)), 1)
+    rec["abs_choice_b_d"] = splits[int(best.item())]
+    rec["total_ms"] = round((rec["esg_us"] + sum(d["radius_grid_us"] + d["encode_us"] for d in rec["splits"])
+                             + rec["abs_select_us"]) / 1e3, 2)
+    if not quiet:
+        print(json.dumps(rec), flush=True)
+    return [rec] if quiet else 0
+
+
 def run_chain(args):
     """Qwen3-4B decoder-layer chain at batch 1 and 4: the layer's linears in dependency order with their
     producers (norm -> q|k|v, o, norm -> gate|up, SiLU-gated product -> down; attention itself is not part of
@@ -739,12 +792,13 @@ def main():
     ap.add_argument("--impl", default="svq", choices=["svq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the sweep / prefill / MoE measurements added to the headline line")
-    ap.add_argument("--workload", default="layer", choices=["layer", "sweep", "prefill", "moe", "chain"],
+                    help="skip the sweep / prefill / MoE / calibration measurements added to the headline line")
+    ap.add_argument("--workload", default="layer", choices=["layer", "sweep", "prefill", "moe", "chain", "calib"],
                     help="layer = the headline line; the others print one JSON line per configuration")
     args = ap.parse_args()
     if args.workload != "layer":
-        return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe, "chain": run_chain}[args.workload](args)
+        return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe, "chain": run_chain,
+                "calib": run_calib}[args.workload](args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_init() if args.impl == "svq" else (int(os.environ.get("WORLD_SIZE", "1")),
