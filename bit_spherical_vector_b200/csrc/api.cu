@@ -13,6 +13,7 @@
 #include "gemm_params.h"
 #include "moe_params.h"
 #include "svq_internal.h"
+#include "calib.h"
 
 namespace {
 

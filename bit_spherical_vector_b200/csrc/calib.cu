@@ -28,7 +28,7 @@
 #include <cmath>
 #include <cstdint>
 
-#include "svq_internal.h"
+#include "calib.h"
 
 namespace svq {
 namespace {

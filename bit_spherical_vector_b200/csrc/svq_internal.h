@@ -23,18 +23,6 @@ cudaError_t launch_rmsnorm_permute(const uint16_t* h, int h_bf16, const uint16_t
 cudaError_t launch_swiglu_permute(const float* gate, const float* up, int M, int I, const int32_t* perm,
                                   uint16_t* out, cudaStream_t st);
 
-// ---------------------------------------------------------------- calibration (ESG, radius grid, encoder, ABS)
-constexpr int kAbsMaxCandidates = 64;
-cudaError_t launch_esg(const float* x, int T, int K, double gamma, double* energy, int32_t* perm, float* weights,
-                       cudaStream_t st);
-cudaError_t launch_radius_grid(const float* W, int N, int K, const int32_t* perm, int b_d, uint16_t* scale,
-                               uint16_t* offset, cudaStream_t st);
-cudaError_t launch_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
-                          const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset,
-                          uint8_t* canonical, double* row_err, cudaStream_t st);
-cudaError_t launch_abs_select(const double* row_err, int n_cand, int N, double* totals, int32_t* best,
-                              cudaStream_t st);
-
 // ---------------------------------------------------------------- GEMV
 constexpr int kGemvMaxMats = 8;
 constexpr int kGemvMaxTokens = 8;        // tokens per pass (more are split into passes)
