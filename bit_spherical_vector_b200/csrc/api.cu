@@ -329,7 +329,6 @@ int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int m
   p.local_route = svq::moe_local_route(n_mats, n_items) ? 1 : 0;
   p.item_out = accumulate ? reinterpret_cast<float*>(b + w.item_out) : nullptr;
   p.status = status;
-  p.one = 1u;
   return cuda_status(svq::launch_moe(p, mt, n_out_rows, sms, (cudaStream_t)stream));
 }
 

@@ -151,43 +151,8 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
   // sign masks of the four element pairs (bits 15 and 31, ready to XOR onto a
   // 16-bit pair), direction index, radius code.
   uint32_t smk[2][4], pidx[2], pcode[2];
-  if (L == 32) {
-    // fragment arrangement (full tile).  The warp's two rows r0, r0 + 1 of
-    // group j belong to one round u of quarter A = j / 4; every field it needs
-    // sits in two places per lane: the round's sign word S_u and the 40 payload
-    // bits of round u (quarter bits [40 (u % 4), 40 (u % 4) + 40), inside the
-    // quarter's payload words w0 and w0 + 1).  Each lane loads its own three
-    // words; the sign holders' words and the address lanes' payload come by
-    // warp shuffles (all 32 lanes take part, also past L).
-    const int u = frag_round(r0, j);
-    const int A = j >> 2, ub = u & 3;
-    const int w0 = (5 * ub) >> 2;                       // 40 * ub / 32
-    const int sh0 = 40 * ub - 32 * w0;                  // bit of the round's field 0 in (P[w0], P[w0+1])
-    const uint32_t Sown = *reinterpret_cast<const uint32_t*>(pk + word_offset_in_block(32, lane, frag_sign_word(u)));
-    const uint32_t Plo = *reinterpret_cast<const uint32_t*>(
-        pk + word_offset_in_block(32, lane, frag_payload_word(5 * A + w0)));
-    const uint32_t Phi = *reinterpret_cast<const uint32_t*>(
-        pk + word_offset_in_block(32, lane, frag_payload_word(5 * A + w0 + 1)));
-    const unsigned long long Pown = ((unsigned long long)Phi << 32) | Plo;
-    uint32_t Sq[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) Sq[q] = __shfl_sync(0xFFFFFFFFu, Sown, frag_sign_lane(lane, q));
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int r = r0 + rr;
-      const int la = frag_addr_lane(lane, r, j);
-      const uint32_t alo = __shfl_sync(0xFFFFFFFFu, Plo, la), ahi = __shfl_sync(0xFFFFFFFFu, Phi, la);
-      const unsigned long long Pa = ((unsigned long long)ahi << 32) | alo;
-      pcode[rr] = ((uint32_t)(Pown >> (sh0 + 10 * frag_code_slot(r, j))) >> bd) & cmask;
-      pidx[rr] = (uint32_t)(Pa >> (sh0 + 10 * frag_addr_slot(lane))) & imask;
-      // the sign holder's word shifted left by the subvector's position puts the
-      // pair's two signs on bits 15 and 31
-      const int ww = frag_sign_pos(lane, r, j);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) smk[rr][q] = (Sq[q] << ww) & 0x80008000u;
-    }
-  } else {
-    // owner arrangement (partial tile): everything in the lane's own words
+  {
+    // everything in the lane's own words (owner arrangement)
     const uint32_t S = word(j);
     uint32_t top[2] = {0u, 0u};
     if (j == 15) {

@@ -8,16 +8,15 @@
 // (Figure 6 caption); weights are reconstructed on demand, never stored dense
 // (Figures 1 and 5).
 //
-// Work split: one CTA per SM.  A matrix's work is cut into units -- a quarter
-// block (128 rows x 4 subvector groups) in full 128-row tiles, a whole block
-// in a partial last tile -- numbered in storage order (tile-major).  Each
-// matrix gets a number of CTAs by a greedy min-max over the estimated time of
-// its slowest CTA (units per warp), each CTA a contiguous range of its units
-// (crossing tile boundaries), and the warps of a CTA contiguous sub-ranges.
-// Partial sums are combined in a fixed order: warps of a CTA in shared memory
-// (the last warp to leave a tile adds them in range order), CTAs sharing a tile
-// through the workspace (the last CTA to finish the tile sums the slots in CTA
-// order).
+// Work split: one CTA per SM.  Each matrix gets a number of CTAs by a greedy
+// min-max over the estimated time of its slowest CTA (rounds of blocks per
+// warp, plus the cross-CTA hand-off when it cannot overlap other work), and
+// each of its CTAs a contiguous range of its blocks in
+// storage order (tile-major), which may cross tile boundaries.  Inside a CTA
+// the warps split the range again contiguously.  Partial sums are combined in
+// a fixed order: warps of a CTA in shared memory (the last warp to leave a tile
+// adds them in range order), CTAs sharing a tile through the workspace (the
+// last CTA to finish the tile sums the slots in CTA order).
 // The workspace starts with a fixed region of completion counters, then the
 // partial sums of the matrices that have tiles shared by several CTAs.
 
@@ -35,21 +34,17 @@ namespace {
 
 size_t up256(size_t b) { return (b + 255) / 256 * 256; }
 
-// CTA of unit q when T units are split into G contiguous ranges [c*T/G, (c+1)*T/G).
+// CTA of block q when T blocks are split into G contiguous ranges [c*T/G, (c+1)*T/G).
 long long cta_of(long long q, long long T, long long G) { return ((q + 1) * G - 1) / T; }
 
-// codebook replicas + x (x_smem 2: natural order and, with a permutation, stored
-// order; 1: natural order; 0: none) + two x slots per warp (x_smem < 2) +
-// per-warp partial sums of npw tiles + 36 ints (warp range boundaries and first
-// tiles) + one completion counter per tile of a CTA's range (at most ntc tiles)
-size_t cta_smem(int b_d, int mt, int npw, int ntc, int K, int x_smem, bool perm) {
+// codebook replicas + two x slots per warp + per-warp partial sums of npw tiles
+// + 36 ints (warp range boundaries and first tiles) + one completion counter per tile of a CTA's
+// range (at most ntc tiles)
+size_t cta_smem(int b_d, int mt, int npw, int ntc) {
   const int R = gemv_cb_replicas(b_d);
   const int W = gemv_warps(mt);
-  const size_t xcopy = (size_t)mt * K * 2;
-  const size_t x = x_smem == 2 ? xcopy * (perm ? 2 : 1) : (x_smem == 1 ? xcopy : 0);
-  const size_t slots = x_smem == 2 ? 0 : (size_t)W * 2 * mt * kBlockCols * 2;
-  return ((size_t)16 * R << b_d) + x + slots + (size_t)W * npw * mt * kTileRows * sizeof(float) + 144 +
-         ((size_t)ntc * 4 + 15) / 16 * 16;
+  return ((size_t)16 * R << b_d) + (size_t)W * 2 * mt * kBlockCols * 2 +
+         (size_t)W * npw * mt * kTileRows * sizeof(float) + 144 + ((size_t)ntc * 4 + 15) / 16 * 16;
 }
 
 }  // namespace
@@ -61,40 +56,40 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
   plan->n_mats = n_mats;
   plan->M = M;
   plan->mt = mt;
-  // Units (gemv_impl.cuh): a quarter block in full 128-row tiles, a whole
-  // block in a partial last tile (worth about four quarters of work).
-  long long U[kGemvMaxMats], work[kGemvMaxMats], total_units = 0;
-  int B[kGemvMaxMats], full[kGemvMaxMats];
+  long long T[kGemvMaxMats], total_blocks = 0;
+  int B[kGemvMaxMats];
   for (int i = 0; i < n_mats; ++i) {
     B[i] = mats[i].K / kBlockCols;
-    full[i] = mats[i].N / kTileRows;
-    const bool partial = mats[i].N % kTileRows != 0;
-    U[i] = 4LL * B[i] * full[i] + (partial ? B[i] : 0);
-    work[i] = 4LL * B[i] * (full[i] + (partial ? 1 : 0));
-    if (U[i] < 1 || U[i] > (1LL << 30)) return false;
-    total_units += U[i];
+    T[i] = (long long)num_tiles(mats[i].N) * B[i];
+    if (T[i] < 1 || T[i] > (1LL << 30)) return false;
+    total_blocks += T[i];
   }
   // One wave of one CTA per SM if the partial-sum buffers fit in shared memory,
   // else more (shorter) ranges.
   for (int mult = 1; mult <= 64; mult *= 2) {
-    const long long G = std::min<long long>((long long)num_sms * mult, total_units);
+    const long long G = std::min<long long>((long long)num_sms * mult, total_blocks);
     if (G < n_mats) return false;
     int ctas[kGemvMaxMats];
     long long used = 0;
     for (int i = 0; i < n_mats; ++i) { ctas[i] = 1; ++used; }
-    // Estimated time of a matrix's slowest CTA, in unit times of one warp: the
-    // units its busiest warp runs.  Greedy min-max: the next CTA goes to the
-    // matrix with the largest estimate (ties: more work per CTA).
+    // Estimated time of a matrix's slowest CTA, in block times of one warp: the
+    // rounds of blocks its warps run (range length / W, rounded up), plus about
+    // 0.6 when the CTA range holds no whole row tile besides the ones it shares
+    // at its ends, so the cross-CTA hand-off of those tiles ends the CTA instead
+    // of overlapping its other work.  Greedy min-max: the next CTA goes to the
+    // matrix with the largest estimate (ties: more blocks per CTA).
     auto est = [&](int i) -> double {
-      const double per_cta = (double)work[i] / ctas[i];
-      return std::ceil(std::ceil(per_cta) / W);
+      const long long n = (T[i] + ctas[i] - 1) / ctas[i];
+      const double rounds = (double)((n + W - 1) / W);
+      const bool exposed = ctas[i] > 1 && 2LL * B[i] > n;
+      return rounds + (exposed ? 0.6 : 0.0);
     };
     while (used < G) {
       int best = -1;
       double worst = -1.0, worst_per = 0.0;
       for (int i = 0; i < n_mats; ++i) {
-        if (ctas[i] >= U[i]) continue;
-        const double e = est(i), per = (double)work[i] / ctas[i];
+        if (ctas[i] >= T[i]) continue;
+        const double e = est(i), per = (double)T[i] / ctas[i];
         if (e > worst + 1e-9 || (e > worst - 1e-9 && per > worst_per)) { worst = e; worst_per = per; best = i; }
       }
       if (best < 0) break;
@@ -102,21 +97,18 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
       ++used;
     }
     size_t smem = 0, off = kGemvCounterBytes;
-    int total = 0, counters = 0, x_smem = 2;
+    int total = 0, counters = 0;
     for (int i = 0; i < n_mats; ++i) {
       GemvPlanMat& pm = plan->m[i];
-      const long long Gi = ctas[i], Ui = U[i];
-      const long long cta_len = (Ui + Gi - 1) / Gi;                // longest CTA range (units)
+      const long long Gi = ctas[i], Ti = T[i];
+      const long long cta_len = (Ti + Gi - 1) / Gi;                // longest CTA range
       const long long warp_len = (cta_len + W - 1) / W;            // longest warp range
-      const long long tu = 4LL * B[i];                             // units of a full tile
       pm.ctas = ctas[i];
       pm.n_tiles = num_tiles(mats[i].N);
-      pm.npw = (int)((warp_len + tu - 2) / tu + 2);
+      pm.npw = (int)((warp_len - 1 + B[i] - 1) / B[i] + 1);
       int kmax = 1;
       for (int t = 0; t < pm.n_tiles; ++t) {
-        const long long q0 = t < full[i] ? tu * t : tu * full[i];
-        const long long q1 = t < full[i] ? tu * (t + 1) : Ui;
-        const long long c0 = cta_of(q0, Ui, Gi), c1 = cta_of(q1 - 1, Ui, Gi);
+        const long long c0 = cta_of((long long)t * B[i], Ti, Gi), c1 = cta_of((long long)(t + 1) * B[i] - 1, Ti, Gi);
         kmax = std::max<int>(kmax, (int)(c1 - c0 + 1));
       }
       pm.kmax = kmax;
@@ -129,28 +121,8 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
         off += pm.part_bytes;
       }
       total += pm.ctas;
-      const int ntc = (int)((cta_len + tu - 2) / tu + 2);
-      // stage x in shared memory when it fits beside the rest: preferably in
-      // stored order as well (the decode then reads it with no per-unit
-      // gathers), else in natural order (gathers from shared memory cost far
-      // fewer L1 wavefronts than scattered global loads)
-      // (one choice for the whole launch: the kernel is compiled per choice).
-      // A stored-order copy costs the prologue one permuting pass over all K
-      // columns; it pays when there is no permutation (the copy is x itself) or
-      // when every CTA's range covers a full tile row of units, i.e. would
-      // gather each column at least once anyway.
-      pm.ntc = ntc;
-      const bool perm = mats[i].perm != nullptr;
-      const bool pays = !perm || Ui / Gi >= tu;
-      int fit = 0;
-      for (int xm = pays ? 2 : 1; xm >= 1 && fit == 0; --xm)
-        if (cta_smem(mats[i].b_d, mt, pm.npw, ntc, mats[i].K, xm, perm) <= kGemvSmemMax) fit = xm;
-      x_smem = std::min(x_smem, fit);
-    }
-    for (int i = 0; i < n_mats; ++i) {
-      GemvPlanMat& pm = plan->m[i];
-      pm.x_smem = x_smem;
-      smem = std::max(smem, cta_smem(mats[i].b_d, mt, pm.npw, pm.ntc, mats[i].K, x_smem, mats[i].perm != nullptr));
+      const int ntc = (int)((cta_len - 1 + B[i] - 1) / B[i] + 1);
+      smem = std::max(smem, cta_smem(mats[i].b_d, mt, pm.npw, ntc));
     }
     if (counters > kGemvMaxCounters) return false;
     if (counters == 0) off = 0;
@@ -172,7 +144,6 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
     GemvKParams kp{};
     kp.n_mats = plan.n_mats;
     kp.y_f32 = y_f32;
-    kp.one = 1u;
     int cta = 0;
     for (int i = 0; i < plan.n_mats; ++i) {
       const GemvMatDesc& d = mats[i];
@@ -193,7 +164,7 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
         g.counters = nullptr;
       }
       g.N = d.N; g.K = d.K; g.b_d = d.b_d; g.M = Mp;
-      g.ctas = pm.ctas; g.cta_begin = cta; g.kmax = pm.kmax; g.npw = pm.npw; g.x_smem = pm.x_smem;
+      g.ctas = pm.ctas; g.cta_begin = cta; g.kmax = pm.kmax; g.npw = pm.npw;
       cta += pm.ctas;
     }
     const size_t smem = plan.smem;

@@ -22,15 +22,12 @@ struct GemvKMat {
   unsigned* counters;     // [n_tiles]
   int N, K, b_d, M;
   int ctas, cta_begin, kmax, npw;
-  int x_smem;             // where a CTA keeps x: 2 shared memory, natural and stored order
-                          // (the decode reads the stored order); 1 natural order only; 0 none
 };
 
 struct GemvKParams {
   GemvKMat mats[kGemvMaxMats];
   int n_mats;
   int y_f32;
-  uint32_t one;           // always 1: shift amounts derived from it stay opaque to the compiler
 };
 
 constexpr size_t kGemvSmemMax = 220 * 1024;

@@ -257,22 +257,9 @@ __device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& 
       ofp[0] = make_float2(op[0], op[1]); ofp[1] = make_float2(op[2], op[3]);
     }
     const uint32_t q16 = (uint32_t)(lane % RR) * 16;
-    // full tiles: fragment decode on the tensor cores (gemv_device.cuh)
-    const FragK fk = frag_consts(p.one, BD, RR);
-    const uint32_t cb_base_q = (uint32_t)__cvta_generic_to_shared(cbs) + q16;
-    uint32_t bm[4][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) bm[i][h] = ((lane >> 3) == i && ((lane >> 2) & 1) == h) ? 0xFFFFFFFFu : 0u;
-    const uint32_t xw_off = 16u * ((lane >> 2) & 1) + 4u * (lane & 3);
     for (int b = 0; b < nb; ++b) {
       if (b + 1 < nb) load_block(d1, tile_base + (size_t)(wb0 + b + 1) * blk_bytes, L, lane, pol_stream);
-      if (L == 32)
-        process_block_frag<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cb_base_q, fk, bm, xw_off, scp,
-                               ofp, acc);
-      else
-        process_block<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cbs, q16, cs, CODEM, scp, ofp, acc);
+      process_block<NC>(d0, xs + (size_t)(wb0 + b) * kBlockCols * 2, K * 2, cbs, q16, cs, CODEM, scp, ofp, acc);
 #pragma unroll
       for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     }
@@ -480,7 +467,7 @@ __global__ void __launch_bounds__(kMoeWarps * 32, 1) moe_kernel(const __grid_con
 }
 
 // y[r][n] = sum over items i with out_row r (ascending i) of item_out[i][n].
-// One CTA per output row: the CTA scans the item list once and compacts the
+// One CTA per (output row, 256-column chunk): the CTA scans the item list once and compacts the
 // indices of its row's items in item order (warp ballots, then a prefix over
 // the warps), so the work is linear in the number of items per row; rows with
 // more items than the shared list holds fall back to a scan per column.
@@ -513,7 +500,9 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const MoeKPara
   }
   const int cnt = s_count;
   if (cnt == 0) return;                              // rows with no item are left untouched
-  for (int n = threadIdx.x; n < p.N; n += kCombineThreads) {
+  // this CTA's columns: chunk blockIdx.y of kCombineThreads columns
+  for (int n = blockIdx.y * kCombineThreads + threadIdx.x; n < min(p.N, (int)(blockIdx.y + 1) * kCombineThreads);
+       n += kCombineThreads) {
     float s = 0.f;
     if (cnt <= kCombineList) {
       for (int k = 0; k < cnt; ++k) s += p.item_out[(size_t)list[k] * p.N + n];
@@ -576,7 +565,8 @@ cudaError_t launch_moe(MoeKParams p, int mt, int n_out_rows, int num_sms, cudaSt
   }
   if (e != cudaSuccess) return e;
   if (p.accumulate) {
-    combine_kernel<<<(unsigned)n_out_rows, kCombineThreads, 0, st>>>(p);
+    const dim3 grid((unsigned)n_out_rows, (unsigned)((p.N + kCombineThreads - 1) / kCombineThreads));
+    combine_kernel<<<grid, kCombineThreads, 0, st>>>(p);
     e = cudaGetLastError();
   }
   return e;

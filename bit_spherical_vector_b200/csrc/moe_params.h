@@ -30,7 +30,6 @@ struct MoeKParams {
   int local_route;                 // 1: every CTA builds the routing tables in shared memory
   float* item_out;                 // [n_items][N] (accumulate only)
   int* status;                     // device status word
-  uint32_t one;                    // always 1 (shift amounts derived from it stay opaque to the compiler)
 };
 
 struct MoeWorkspace {

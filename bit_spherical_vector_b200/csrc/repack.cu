@@ -1,11 +1,9 @@
 // repack.cu -- canonical stream -> device layout, its inverse (field export)
 // and the bit-exact dense dequantisation.
 //
-// One thread builds (or reads) one lane-block (144 bytes); see layout.cuh for
-// the two arrangements (fragment order in full 128-row tiles, owner order in a
-// partial last tile).  These kernels run once per matrix (repack) or in tests
-// and exports (unpack, dequantize), so they favour plainness over speed: each
-// field is located through the arrangement's index functions.
+// One thread owns one lane-block (4 rows x 16 subvectors, 144 bytes); see
+// layout.cuh.  These kernels run once per matrix (repack) or in tests and
+// exports (unpack, dequantize), so they favour plainness over speed.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -117,52 +115,20 @@ __global__ void repack_kernel(const uint8_t* __restrict__ canon, int N, int K, i
   const LaneBlockId lb = lane_block_id(N, K, id);
   if (!lb.valid) return;
   const size_t rb = (size_t)K * 9 / 32;               // canonical row bytes (K % 128 == 0)
-  uint32_t w[kWords];
-  if (tile_lanes(N, lb.t) == 32) {
-    // fragment arrangement: every word is built from the subvectors this lane's
-    // roles need (sign holder, codebook address, owner), read straight from the
-    // canonical stream
-    auto code_of = [&](int row, int grp) -> uint32_t {
-      const uint8_t* seg = canon + (size_t)(lb.t * kTileRows + row) * rb + (size_t)lb.b * 36;
-      return read_code(seg, grp);
-    };
-    const int q = lb.l & 3;
-    uint32_t P[21];
-    for (int k = 0; k < 21; ++k) P[k] = 0;
-    for (int u = 0; u < 16; ++u) {
-      uint32_t S = 0;
-      for (int ww = 0; ww < 16; ++ww) {
-        const uint32_t c = code_of(frag_sign_row(lb.l, u, ww), frag_sign_group(u, ww));
-        S |= ((c >> (2 * q)) & 1u) << (15 - ww);
-        S |= ((c >> (2 * q + 1)) & 1u) << (31 - ww);
-      }
-      w[frag_sign_word(u)] = S;
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t ci = code_of(frag_addr_row(lb.l, u, k), frag_addr_group(lb.l, u));
-        const uint32_t cc = code_of(frag_code_row(lb.l, u, k), frag_code_group(u, k));
-        const uint32_t idx = (ci >> 8) & ((1u << b_d) - 1u);
-        const uint32_t code = (cc >> 8) >> b_d;
-        const uint32_t slot = idx | (code << b_d);
-        const int p = frag_slot_bit(u, k);
-        P[p >> 5] |= slot << (p & 31);
-        if ((p & 31) > 22) P[(p >> 5) + 1] |= slot >> (32 - (p & 31));
-      }
+  uint8_t s[16][4];
+  uint32_t p[16][4];
+  for (int r = 0; r < 4; ++r) {
+    const int n = lb.t * kTileRows + 4 * lb.l + r;
+    const uint8_t* seg = canon + (size_t)n * rb + (size_t)lb.b * 36;   // 16 codes = 36 bytes
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t code = read_code(seg, j);
+      s[j][r] = (uint8_t)(code & 0xFFu);
+      p[j][r] = code >> 8;                              // idx | radius << b_d
     }
-    for (int i = 0; i < 20; ++i) w[frag_payload_word(i)] = P[i];
-  } else {
-    uint8_t s[16][4];
-    uint32_t p[16][4];
-    for (int r = 0; r < 4; ++r) {
-      const int n = lb.t * kTileRows + 4 * lb.l + r;
-      const uint8_t* seg = canon + (size_t)n * rb + (size_t)lb.b * 36;   // 16 codes = 36 bytes
-      for (int j = 0; j < 16; ++j) {
-        const uint32_t code = read_code(seg, j);
-        s[j][r] = (uint8_t)(code & 0xFFu);
-        p[j][r] = code >> 8;                              // idx | radius << b_d
-      }
-    }
-    build_words(s, p, w);
   }
+  (void)b_d;
+  uint32_t w[kWords];
+  build_words(s, p, w);
   for (int c = 0; c < kChunks; ++c) {
     uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
     *reinterpret_cast<uint4*>(out + chunk_offset(N, K, lb.t, lb.b, c, lb.l)) = v;
@@ -180,47 +146,6 @@ __device__ void load_words(const uint8_t* packed, int N, int K, const LaneBlockI
   }
 }
 
-// Fields of lane lb.l's own 4 rows x 16 subvectors: s[j][r] sign byte, p[j][r]
-// payload (idx | code << b_d).  Partial tiles: read from the lane's own words;
-// full tiles: each field from the lane that holds it in the fragment arrangement.
-__device__ void lane_fields(const uint8_t* packed, int N, int K, int b_d, const LaneBlockId& lb, uint8_t s[16][4],
-                            uint32_t p[16][4]) {
-  if (tile_lanes(N, lb.t) != 32) {
-    uint32_t w[kWords];
-    load_words(packed, N, K, lb, w);
-    split_words(w, s, p);
-    return;
-  }
-  const uint8_t* blk = packed + tile_offset(K, lb.t) + (size_t)lb.b * 32 * kLaneBlockBytes;
-  auto word = [&](int lane, int wi) -> uint32_t {
-    return *reinterpret_cast<const uint32_t*>(blk + word_offset_in_block(32, lane, wi));
-  };
-  auto slot = [&](int lane, int u, int k) -> uint32_t {
-    const int pb = frag_slot_bit(u, k);
-    uint32_t P[2];
-    P[0] = word(lane, frag_payload_word(pb >> 5));
-    P[1] = (pb & 31) > 22 ? word(lane, frag_payload_word((pb >> 5) + 1)) : 0u;
-    return payload_field(P, pb & 31);
-  };
-  const int T = lb.l;
-  const uint32_t imask = (1u << b_d) - 1u;
-  for (int r = 0; r < 4; ++r)
-    for (int j = 0; j < 16; ++j) {
-      const int u = frag_round(r, j);
-      const uint32_t code = slot(T, u, frag_code_slot(r, j)) >> b_d;
-      const uint32_t idx = slot(frag_addr_lane(T, r, j), u, frag_addr_slot(T)) & imask;
-      const int ww = frag_sign_pos(T, r, j);
-      uint32_t sg = 0;
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t S = word(frag_sign_lane(T, q), frag_sign_word(u));
-        sg |= ((S >> (15 - ww)) & 1u) << (2 * q);
-        sg |= ((S >> (31 - ww)) & 1u) << (2 * q + 1);
-      }
-      s[j][r] = (uint8_t)sg;
-      p[j][r] = idx | (code << b_d);
-    }
-}
-
 __global__ void unpack_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d,
                               uint8_t* __restrict__ signs, uint16_t* __restrict__ idx,
                               uint16_t* __restrict__ code) {
@@ -228,9 +153,11 @@ __global__ void unpack_kernel(const uint8_t* __restrict__ packed, int N, int K, 
   if (id >= num_lane_blocks(N, K)) return;
   const LaneBlockId lb = lane_block_id(N, K, id);
   if (!lb.valid) return;
+  uint32_t w[kWords];
+  load_words(packed, N, K, lb, w);
   uint8_t s[16][4];
   uint32_t p[16][4];
-  lane_fields(packed, N, K, b_d, lb, s, p);
+  split_words(w, s, p);
   const int G = K / 8;
   const uint32_t imask = (1u << b_d) - 1u;
   for (int r = 0; r < 4; ++r) {
@@ -254,9 +181,11 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, int N, int K,
   if (id >= num_lane_blocks(N, K)) return;
   const LaneBlockId lb = lane_block_id(N, K, id);
   if (!lb.valid) return;
+  uint32_t w[kWords];
+  load_words(packed, N, K, lb, w);
   uint8_t s[16][4];
   uint32_t p[16][4];
-  lane_fields(packed, N, K, b_d, lb, s, p);
+  split_words(w, s, p);
   const uint32_t imask = (1u << b_d) - 1u;
   for (int r = 0; r < 4; ++r) {
     const int n = lb.t * kTileRows + 4 * lb.l + r;

@@ -46,9 +46,8 @@ struct GemvMatDesc {                      // host-side description of one matrix
   void* y;                               // [M][N]
 };
 
-// A matrix's work units (a quarter of a 128-row x 128-column block in full
-// tiles, a whole block in a partial last tile) are numbered in storage order;
-// its ctas CTAs take equal contiguous ranges of them.
+// A matrix's blocks (128-row tile t, 128-column block kb) are numbered
+// q = t * (K / 128) + kb.  Its ctas CTAs take equal contiguous ranges of q.
 // Workspace of a GEMV launch: completion counters (one per shared-capable row
 // tile) in a fixed region at its start, then the partial sums of each matrix.
 // The counter region never moves, so counters left at zero by one call are
@@ -57,15 +56,12 @@ constexpr size_t kGemvCounterBytes = 64 * 1024;
 constexpr int kGemvMaxCounters = (int)(kGemvCounterBytes / sizeof(unsigned));
 
 struct GemvPlanMat {
-  int ctas;                              // CTA c covers units [c*U/ctas, (c+1)*U/ctas)
+  int ctas;                              // CTA c covers q in [c*T/ctas, (c+1)*T/ctas), T = blocks
   int n_tiles;                           // 128-row tiles
   int kmax;                              // most CTAs sharing one tile (1: no cross-CTA sums)
   int npw;                               // most tiles that one warp's range touches
   int counter0;                          // first counter of this matrix's tiles
   size_t part_offset, part_bytes;        // partial sums [n_tiles][kmax][mt][128] (kmax > 1)
-  int x_smem;                            // x in shared memory: 2 natural + stored order, 1 natural, 0 none
-                                         // (the same for every matrix of a launch)
-  int ntc;                               // most tiles that one CTA's range touches
 };
 
 struct GemvPlan {
