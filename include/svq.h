@@ -142,11 +142,10 @@ SVQ_API int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t strea
  * x: fp16 [M][K] (natural input order; the kernel applies perm, Figure 6;
  * stored order when perm is NULL).
  * y: [M][N] of y_dtype SVQ_F16 or SVQ_F32.  Each subvector's eight products
- * of fp16 codeword entries and fp16 activations are summed in fp32 (in full
- * 128-row tiles on the tensor cores; in a partial last tile each product is
- * first rounded to fp16, never exceeding |x| since codeword entries are at most
- * 1), scaled by the radius and accumulated across subvectors in fp32, so any
- * finite fp16 x is safe from overflow.
+ * of fp16 codeword entries and fp16 activations are formed exactly and
+ * accumulated in fp32 (one rounding per addition), scaled by the radius and
+ * accumulated across subvectors in fp32, so any finite fp16 x is safe from
+ * overflow.
  * Error bound used by the tests: |y - y_ref| <= 1e-3 * sum_j |W[n][j]||x[m][perm[j]]|.
  * Launch: the kernel is launched as a programmatic dependent of the previous
  * kernel on `stream`; it reads x only after that kernel has completed, but may

@@ -201,10 +201,10 @@ def test_lm_head_sized_matrix_sampled_rows():
 
 @pytest.mark.parametrize("M", [1, 2, 5])
 @pytest.mark.parametrize("N", [9728, 9660])
-def test_grouped_stored_order_staging(N, M):
-    """Two N x 2560 matrices with permutations in one grouped call: every CTA's range covers more than
-    one 128-row tile of units, so each CTA stages x in stored order once and the decode reads its
-    operands from that copy (N = 9660 adds a 60-row last tile).  Every output against the oracle."""
+def test_grouped_two_permuted_gate_shaped_matrices(N, M):
+    """Two N x 2560 matrices with permutations and different b_d in one grouped call, CTA ranges
+    spanning more than one row tile (N = 9660 adds a 60-row last tile).  Every output against the
+    oracle."""
     need_gpu()
     K = 2560
     mats = [synth.make_matrix(68, i + N % 7, N, K, 7 + i) for i in range(2)]
