@@ -65,9 +65,11 @@ constexpr int kStgBytes = kStageCols * 128 * 4;
 template <int NS>
 __host__ __device__ constexpr int p_slots() { return NS + 3 <= 8 ? NS + 3 : 8; }
 
-template <int BN, int NS>
+// DENSE (pre-decoded weights): no packed-code ring and no codebook, so the
+// A/B ring can be deeper.
+template <int BN, int NS, bool DENSE>
 __host__ __device__ constexpr uint32_t smem_bytes() {
-  return NS * kATileBytes + NS * BN * 128 + p_slots<NS>() * kPTileBytes + kCbBytes + kStgBytes +
+  return NS * kATileBytes + NS * BN * 128 + (DENSE ? 0 : p_slots<NS>() * kPTileBytes + kCbBytes) + kStgBytes +
          1024 /* barriers */ + 1024 /* align */;
 }
 
@@ -212,17 +214,18 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
   }
 }
 
-template <int BN, int NS, bool BF16>
+template <int BN, int NS, bool BF16, bool DENSE>
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmKParams p) {
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+            const __grid_constant__ GemmKParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* a_st = base;
   uint8_t* b_st = a_st + NS * kATileBytes;
   constexpr int NP = p_slots<NS>();
-  uint8_t* p_st = b_st + NS * BN * 128;             // packed-code ring (NP slots)
-  uint8_t* cbs = p_st + NP * kPTileBytes;
-  float* stg = reinterpret_cast<float*>(cbs + kCbBytes);
+  uint8_t* p_st = b_st + NS * BN * 128;             // packed-code ring (NP slots; none when DENSE)
+  uint8_t* cbs = p_st + (DENSE ? 0 : NP * kPTileBytes);
+  float* stg = reinterpret_cast<float*>(cbs + (DENSE ? 0 : kCbBytes));
   Bars* bars = reinterpret_cast<Bars*>(reinterpret_cast<uint8_t*>(stg) + kStgBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -231,7 +234,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&bars->full_a[s], kNumDec);
+      mbar_init(&bars->full_a[s], DENSE ? 1 : kNumDec);   // TMA bytes, or the decoders
       mbar_init(&bars->full_b[s], 1);
       mbar_init(&bars->empty[s], 1);
     }
@@ -247,13 +250,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) prefetch_tmap(&tmap_x);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmap_x);
+    if (DENSE) prefetch_tmap(&tmap_w);
+  }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
   }
   // Codebook replicas: entry e, replica q at 16-byte slot e * rep + q.
-  {
+  if constexpr (!DENSE) {
     const int rep = p.cb_replicas;
     const int n = (1 << p.b_d) * rep;
     for (int i = threadIdx.x; i < n; i += kThreads)
@@ -290,7 +296,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       int itb = 0, itp = 0;
       bool ok = true;
       while (ok && cb_.u < n_units) {
-        while (cp_.u < n_units && itp < itb + NP - 2) {
+        while (!DENSE && cp_.u < n_units && itp < itb + NP - 2) {
           const int s = itp % NP;
           const uint32_t ph = (itp / NP) & 1;
           if (itp >= NP && !wait_bar(&bars->empty_p[s], ph ^ 1, p, bars)) { ok = false; break; }
@@ -306,6 +312,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         const int s = itb % NS;
         const uint32_t ph = (itb / NS) & 1;
         if (itb >= NS && !wait_bar(&bars->empty[s], ph ^ 1, p, bars)) { ok = false; break; }
+        if constexpr (DENSE) {
+          // pre-decoded weights: the 128 x 64 tile of rows nt*128.. straight from the workspace
+          mbar_arrive_expect_tx(&bars->full_a[s], kATileBytes);
+          tma_load_2d(a_st + s * kATileBytes, &tmap_w, &bars->full_a[s], cb_.kb * 64, cb_.w.nt * kTileRows);
+        }
         mbar_arrive_expect_tx(&bars->full_b[s], BN * 128);
         tma_load_2d(b_st + s * BN * 128, &tmap_x, &bars->full_b[s], cb_.kb * 64, cb_.w.mt * BN);
         advance(cb_);
@@ -313,7 +324,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       }
       if (!ok) {
         // Let copies already issued land before the CTA exits.
-        for (int k = std::max(0, itb - NS); k < itb; ++k) mbar_wait(&bars->full_b[k % NS], (k / NS) & 1);
+        for (int k = std::max(0, itb - NS); k < itb; ++k) {
+          mbar_wait(&bars->full_b[k % NS], (k / NS) & 1);
+          if (DENSE) mbar_wait(&bars->full_a[k % NS], (k / NS) & 1);
+        }
         for (int k = std::max(0, itp - NP); k < itp; ++k) mbar_wait(&bars->full_p[k % NP], (k / NP) & 1);
       }
     }
@@ -358,7 +372,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     // phases could alias an mbarrier parity).
     const int d = warp - kDecWarp0;
     int it = 0;
-    bool ok = true;
+    bool ok = !DENSE;                        // pre-decoded weights: the decoders have nothing to do
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);
       // radius parameters of this lane's 4 rows of the unit's row tile
@@ -413,12 +427,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c0, v);
         tmem_ld_wait();
-        // weight row 4 * lane + q (TMEM lane 32q + lane) is staged at position
-        // 4 * lane + (q ^ x), x = (lane / 8) % 4: the lanes of a store that
-        // share a bank (lane, lane + 8, ...) get different offsets, so the
-        // stores are conflict free; the reader undoes the swizzle in registers
-        const int xs = (lane >> 3) & 3;
-        const int nl = 4 * lane + (q ^ xs);
+        // Weight row `row` of the tile is staged at position 4 L + ((row % 4) ^
+        // x(L)), L = row / 4, x(L) = (L / 8) % 4: the reader lane L takes rows
+        // 4L..4L+3 with one 16-byte load and undoes the swizzle in registers.
+        // For decoded tiles (weight row 4 * lane + q in TMEM lane 32q + lane)
+        // the lanes of a store that would share a bank (lane, lane + 8, ...)
+        // get different offsets; pre-decoded tiles (row 32q + lane) store 32
+        // distinct banks either way.
+        const int row = DENSE ? 32 * q + lane : 4 * lane + q;
+        const int rl = row >> 2;
+        const int nl = 4 * rl + ((row & 3) ^ ((rl >> 3) & 3));
+        const int xs = (lane >> 3) & 3;                // the reader's swizzle (rows 4 * lane ..)
 #pragma unroll
         for (int i = 0; i < 32; ++i) stg[i * 128 + nl] = __uint_as_float(v[i]);
         named_bar_sync(1, kNumEpi * 32);
@@ -505,24 +524,27 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ partial, int S, l
   }
 }
 
-template <int BN, int NS, bool BF16>
-cudaError_t launch_bn(const CUtensorMap& tm, const GemmKParams& p, int grid, cudaStream_t st) {
-  constexpr uint32_t smem = smem_bytes<BN, NS>();
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, NS, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+template <int BN, int NS, bool BF16, bool DENSE = false>
+cudaError_t launch_bn(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid, cudaStream_t st) {
+  constexpr uint32_t smem = smem_bytes<BN, NS, DENSE>();
+  static_assert(smem <= 227 * 1024, "shared memory");
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, NS, BF16, DENSE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gemm_kernel<BN, NS, BF16><<<grid, kThreads, smem, st>>>(tm, p);
+  gemm_kernel<BN, NS, BF16, DENSE><<<grid, kThreads, smem, st>>>(tm, tw, p);
   return cudaGetLastError();
 }
 
 template <bool BF16>
-cudaError_t launch_typed(int BN, const CUtensorMap& tm, const GemmKParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_typed(int BN, const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid,
+                         cudaStream_t st) {
   switch (BN) {
-    case 16: return launch_bn<16, 6, BF16>(tm, p, grid, st);
-    case 32: return launch_bn<32, 6, BF16>(tm, p, grid, st);
-    case 64: return launch_bn<64, 5, BF16>(tm, p, grid, st);
-    case 128: return launch_bn<128, 4, BF16>(tm, p, grid, st);
-    default: return launch_bn<256, 3, BF16>(tm, p, grid, st);
+    case 16: return launch_bn<16, 6, BF16>(tm, tw, p, grid, st);
+    case 32: return launch_bn<32, 6, BF16>(tm, tw, p, grid, st);
+    case 64: return launch_bn<64, 5, BF16>(tm, tw, p, grid, st);
+    case 128: return launch_bn<128, 4, BF16>(tm, tw, p, grid, st);
+    default:
+      return p.dense ? launch_bn<256, 4, BF16, true>(tm, tw, p, grid, st) : launch_bn<256, 3, BF16>(tm, tw, p, grid, st);
   }
 }
 
@@ -573,11 +595,18 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
     }
   }
   g.grid = std::min(T * g.S, num_sms);
+  // From four token tiles on, the matrix is decoded once into the workspace
+  // (N x K 16-bit values, the activations' type) and the kernel loads weight
+  // tiles by TMA instead of decoding every stage once per token tile; below
+  // that the decode pass costs more than the repeated on-chip decodes.
+  g.dense = g.m_tiles >= 4 ? 1 : 0;
   const size_t xp = ((size_t)M * K * 2 + 255) / 256 * 256;
+  const size_t wdec = g.dense ? ((size_t)N * K * 2 + 255) / 256 * 256 : 0;
   g.xp_offset = 0;
-  g.partial_offset = xp;
+  g.wdec_offset = xp;
+  g.partial_offset = xp + wdec;
   const size_t part = g.S > 1 ? ((size_t)g.S * M * N * 4 + 255) / 256 * 256 : 0;
-  g.ws_bytes = xp + part;
+  g.ws_bytes = xp + wdec + part;
   return g;
 }
 
@@ -606,6 +635,21 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
                          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // pre-decoded weights (dense plan): the matrix decoded once, in the stored
+  // column order and the activations' 16-bit type, tiles of 128 rows x 64 columns
+  CUtensorMap tw = tm;
+  if (g.dense) {
+    uint16_t* wdec = reinterpret_cast<uint16_t*>(wsb + g.wdec_offset);
+    cudaError_t e = launch_dequant(d.packed, d.N, d.K, d.b_d, d.codebook, d.scale, d.offset, d.x_bf16, wdec, st);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t wdims[2] = {(cuuint64_t)d.K, (cuuint64_t)d.N};
+    const cuuint32_t wbox[2] = {64, (cuuint32_t)kTileRows};
+    const CUresult rw = enc(&tw, d.x_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                            wdec, wdims, strides, wbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (rw != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  }
   GemmKParams p{};
   p.packed = reinterpret_cast<const uint8_t*>(d.packed);
   p.codebook = reinterpret_cast<const uint4*>(d.codebook);
@@ -619,7 +663,9 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.partial = g.S > 1 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
   p.status = status;
   p.wait_polls = g_wait_polls.load(std::memory_order_relaxed);
-  cudaError_t e = d.x_bf16 ? launch_typed<true>(g.BN, tm, p, g.grid, st) : launch_typed<false>(g.BN, tm, p, g.grid, st);
+  p.dense = g.dense;
+  cudaError_t e = d.x_bf16 ? launch_typed<true>(g.BN, tm, tw, p, g.grid, st)
+                           : launch_typed<false>(g.BN, tm, tw, p, g.grid, st);
   if (e != cudaSuccess || g.S == 1) return e;
   const long long mn = (long long)d.M * d.N;
   const long long blocks = std::min<long long>((mn / 4 + 255) / 256, 148LL * 8);

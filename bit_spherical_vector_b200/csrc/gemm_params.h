@@ -20,11 +20,13 @@ struct GemmKParams {
   float* partial;       // [S][M][N] when S > 1
   int* status;          // device status word (bounded-wait timeouts)
   uint32_t wait_polls;  // polls before a bounded wait gives up (svq_debug_set_wait_polls)
+  int dense;            // 1: weight tiles come pre-decoded from the workspace by TMA (decoders idle)
 };
 
 struct GemmPlan {
   int BN, m_tiles, n_tiles, S, grid;
-  size_t xp_offset, partial_offset, ws_bytes;
+  int dense;            // decode the whole matrix once into the workspace, then a dense GEMM
+  size_t xp_offset, wdec_offset, partial_offset, ws_bytes;
 };
 
 struct GemmMatDesc {

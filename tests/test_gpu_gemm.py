@@ -119,3 +119,22 @@ def test_gemm_metamorphic_permutation():
     y1, _, _ = _gemm(svq.SvqWeight.from_synth(m), x)
     y2, _, _ = _gemm(svq.SvqWeight.from_synth(mid), np.ascontiguousarray(x[:, m.perm]))
     assert torch.equal(y1, y2)
+
+
+@pytest.mark.parametrize("x_dtype", ["bf16", "f16"])
+def test_gemm_pre_decoded_plan_matches_decoded_tiles(x_dtype):
+    """Four or more 256-token tiles switch the GEMM to weights decoded once into the workspace and
+    loaded by TMA; one tile decodes on chip.  Both place the same 16-bit weights in the MMA (the export
+    reading), so the first 256 tokens of a 1100-token call equal a 256-token call bit for bit (K = 512:
+    no K split in either plan), and every output is within the bound of the oracle.  N = 1028 ends in a
+    4-row tile (rows past N read as zeros by the TMA box)."""
+    need_gpu()
+    N, K = 1028, 512
+    m = synth.make_matrix(76, 1 if x_dtype == "f16" else 0, N, K, 7)
+    x = synth.make_x(76, 2, 1100, K, dtype=x_dtype)
+    W = svq.SvqWeight.from_synth(m)
+    yb, _, _ = _gemm(W, x, kind=x_dtype)
+    y256, _, _ = _gemm(W, np.ascontiguousarray(x[:256]), kind=x_dtype)
+    assert torch.equal(yb[:256], y256)
+    y_ref, den = oracle.linear(m, x, x_dtype)
+    assert rel_err(yb.cpu().numpy(), y_ref, den) <= TOL
