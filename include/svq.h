@@ -11,7 +11,8 @@
  *   - Figure 6 caption: the kernel multiplies each decoded subvector by eight
  *     reordered activations (the ESG input-channel permutation).
  *   - Figures 1 and 5 captions: weights are reconstructed on demand; no dense
- *     copy of W is kept.
+ *     copy of W is kept (svq_linear_gemm from 4 tiles of 256 tokens on decodes
+ *     the matrix into its caller-owned workspace for the duration of the call).
  *
  * Conventions for every entry point:
  *   - All data pointers are DEVICE pointers owned by the caller, except where
