@@ -72,13 +72,13 @@ def _load():
         lib.svqref_unpack.restype = None
         lib.svqref_radius.argtypes = [ctypes.c_uint16, ctypes.c_uint16, ctypes.c_uint32]
         lib.svqref_radius.restype = ctypes.c_float
-        lib.svqref_decode_exact.argtypes = [i32, i32, i32, P, P, P, P, P]
+        lib.svqref_decode_exact.argtypes = [i32, i32, i32, P, P, P, P, P, P]
         lib.svqref_decode_exact.restype = None
-        lib.svqref_dequant.argtypes = [i32, i32, i32, P, P, P, P, i32, P]
+        lib.svqref_dequant.argtypes = [i32, i32, i32, P, P, P, P, P, i32, P]
         lib.svqref_dequant.restype = None
-        lib.svqref_linear.argtypes = [i32, i32, i32, P, P, P, P, P, P, i32, i32, P, P]
+        lib.svqref_linear.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, i32, i32, P, P]
         lib.svqref_linear.restype = None
-        lib.svqref_encode.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
+        lib.svqref_encode.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P, P]
         lib.svqref_encode.restype = None
         lib.svqref_num_threads.argtypes = []
         lib.svqref_num_threads.restype = i32
@@ -154,21 +154,38 @@ def unpack(N, K, b_d, canon):
 
 
 # --------------------------------------------------------------------------- decode
+def _radius_arrays(m):
+    """(scale, offset, lut) contiguous arrays of an SvqMatrix-like object: a per-row level table when it
+    has one (m.lut [N][2^b_r] fp16 bits) and no affine pair, else the affine pair and no table.  The
+    caller keeps the arrays alive across the C call."""
+    lut = getattr(m, "lut", None)
+    if lut is not None:
+        lut = _c(lut, np.uint16)
+        assert lut.shape == (m.N, 1 << (10 - m.b_d))
+        return None, None, lut
+    return _c(m.scale, np.uint16), _c(m.offset, np.uint16), None
+
+
+def _optr(a):
+    return None if a is None else _ptr(a)
+
+
 def decode_exact(m) -> np.ndarray:
     """Exact fp64 weights [N][K] (stored column order) of an SvqMatrix-like object."""
     W = np.empty((m.N, m.K), np.float64)
+    sc, of, lt = _radius_arrays(m)
     _load().svqref_decode_exact(m.N, m.K, m.b_d, _ptr(_c(m.canonical, np.uint8)),
-                                _ptr(_c(m.codebook, np.uint16)), _ptr(_c(m.scale, np.uint16)),
-                                _ptr(_c(m.offset, np.uint16)), _ptr(W))
+                                _ptr(_c(m.codebook, np.uint16)), _optr(sc), _optr(of), _optr(lt), _ptr(W))
     return W
 
 
 def dequant(m, kind: str = "f16") -> np.ndarray:
     """Bit patterns [N][K] of the exported fp16 ('f16') or bf16 ('bf16') weights."""
     out = np.empty((m.N, m.K), np.uint16)
+    sc, of, lt = _radius_arrays(m)
     _load().svqref_dequant(m.N, m.K, m.b_d, _ptr(_c(m.canonical, np.uint8)),
-                           _ptr(_c(m.codebook, np.uint16)), _ptr(_c(m.scale, np.uint16)),
-                           _ptr(_c(m.offset, np.uint16)), 0 if kind == "f16" else 1, _ptr(out))
+                           _ptr(_c(m.codebook, np.uint16)), _optr(sc), _optr(of), _optr(lt),
+                           0 if kind == "f16" else 1, _ptr(out))
     return out
 
 
@@ -183,23 +200,28 @@ def linear(m, x_bits, x_kind: str = "f16"):
     assert x_bits.shape[1] == m.K
     y = np.empty((M, m.N), np.float64)
     den = np.empty((M, m.N), np.float64)
+    sc, of, lt = _radius_arrays(m)
     _load().svqref_linear(m.N, m.K, m.b_d, _ptr(_c(m.canonical, np.uint8)),
-                          _ptr(_c(m.codebook, np.uint16)), _ptr(_c(m.scale, np.uint16)),
-                          _ptr(_c(m.offset, np.uint16)), _ptr(_c(m.perm, np.int32)),
+                          _ptr(_c(m.codebook, np.uint16)), _optr(sc), _optr(of), _optr(lt),
+                          _ptr(_c(m.perm, np.int32)),
                           _ptr(x_bits), 0 if x_kind == "f16" else 1, M, _ptr(y), _ptr(den))
     return y, den
 
 
-def encode(N, K, b_d, W, codebook, scale, offset, energy=None):
-    """Brute-force nearest-codeword encoder; returns (signs, idx, code) [N][K/8]."""
+def encode(N, K, b_d, W, codebook, scale, offset, energy=None, lut=None):
+    """Brute-force nearest-codeword encoder; returns (signs, idx, code) [N][K/8].  The radius levels of
+    row n are fma(scale[n], code, offset[n]), or lut[n][code] when a per-row table is given."""
     W = _c(W, np.float64)
     G = K // 8
     signs = np.empty((N, G), np.uint8)
     idx = np.empty((N, G), np.uint16)
     code = np.empty((N, G), np.uint16)
     e = None if energy is None else _c(energy, np.float64)
+    lt = None if lut is None else _c(lut, np.uint16)
     _load().svqref_encode(N, K, b_d, _ptr(W), _ptr(_c(codebook, np.uint16)),
-                          _ptr(_c(scale, np.uint16)), _ptr(_c(offset, np.uint16)),
+                          None if lt is not None else _ptr(_c(scale, np.uint16)),
+                          None if lt is not None else _ptr(_c(offset, np.uint16)),
+                          None if lt is None else _ptr(lt),
                           None if e is None else _ptr(e), _ptr(signs), _ptr(idx), _ptr(code))
     return signs, idx, code
 

@@ -216,11 +216,21 @@ float svqref_radius(uint16_t scale_h, uint16_t offset_h, uint32_t code) {
   return std::fmaf(svqref_h2f(scale_h), (float)code, svqref_h2f(offset_h));
 }
 
+// Radius of (row n, code) under either form of the quantized radius: the
+// affine pair above, or (lut != NULL) a per-row table of 2^b_r fp16 levels,
+// r = fp32(lut[n][code]) -- the levels the pages optimise ("SAGE", Figure 2
+// caption: a quantized radius; the pages fit the levels, not a formula).
+static float row_radius(const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int b_d, int n,
+                        uint32_t code) {
+  if (lut) return svqref_h2f(lut[((size_t)n << (10 - b_d)) + code]);
+  return svqref_radius(scale[n], offset[n], code);
+}
+
 // Exact decoded weights in fp64, W[n][j] in the stored (permuted) column
 // order: W[n][8g+i] = (-1)^{s_i} * r * c_{idx,i}.  The product of a binary32
 // radius and a binary16 codebook entry is exact in fp64.
 void svqref_decode_exact(int N, int K, int b_d, const uint8_t* canon, const uint16_t* codebook,
-                         const uint16_t* scale, const uint16_t* offset, double* W) {
+                         const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, double* W) {
   const int G = K / 8;
   std::vector<uint8_t> s((size_t)N * G);
   std::vector<uint16_t> id((size_t)N * G), cd((size_t)N * G);
@@ -230,7 +240,7 @@ void svqref_decode_exact(int N, int K, int b_d, const uint8_t* canon, const uint
   for (int n = 0; n < N; ++n) {
     for (int g = 0; g < G; ++g) {
       const int64_t f = (int64_t)n * G + g;
-      const double r = (double)svqref_radius(scale[n], offset[n], cd[f]);
+      const double r = (double)row_radius(scale, offset, lut, b_d, n, cd[f]);
       for (int i = 0; i < 8; ++i) {
         const double c = (double)svqref_h2f(codebook[(size_t)id[f] * 8 + i]);
         const double w = r * c;
@@ -246,7 +256,8 @@ void svqref_decode_exact(int N, int K, int b_d, const uint8_t* canon, const uint
 //   bf16: same, rounding the binary32 product to bfloat16.
 // out_kind: 0 = fp16, 1 = bf16.  Output bit patterns [N][K].
 void svqref_dequant(int N, int K, int b_d, const uint8_t* canon, const uint16_t* codebook,
-                    const uint16_t* scale, const uint16_t* offset, int out_kind, uint16_t* out) {
+                    const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_kind,
+                    uint16_t* out) {
   const int G = K / 8;
   std::vector<uint8_t> s((size_t)N * G);
   std::vector<uint16_t> id((size_t)N * G), cd((size_t)N * G);
@@ -254,7 +265,7 @@ void svqref_dequant(int N, int K, int b_d, const uint8_t* canon, const uint16_t*
   for (int n = 0; n < N; ++n) {
     for (int g = 0; g < G; ++g) {
       const int64_t f = (int64_t)n * G + g;
-      const float r = svqref_radius(scale[n], offset[n], cd[f]);
+      const float r = row_radius(scale, offset, lut, b_d, n, cd[f]);
       for (int i = 0; i < 8; ++i) {
         const float c = svqref_h2f(codebook[(size_t)id[f] * 8 + i]);
         const float p = r * c;                              // one binary32 rounding
@@ -274,10 +285,10 @@ void svqref_dequant(int N, int K, int b_d, const uint8_t* canon, const uint16_t*
 // x holds M rows of K 16-bit values; x_kind 0 = fp16, 1 = bf16.
 // ---------------------------------------------------------------------------
 void svqref_linear(int N, int K, int b_d, const uint8_t* canon, const uint16_t* codebook,
-                   const uint16_t* scale, const uint16_t* offset, const int32_t* perm,
+                   const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, const int32_t* perm,
                    const uint16_t* x, int x_kind, int M, double* y, double* den) {
   std::vector<double> W((size_t)N * K);
-  svqref_decode_exact(N, K, b_d, canon, codebook, scale, offset, W.data());
+  svqref_decode_exact(N, K, b_d, canon, codebook, scale, offset, lut, W.data());
   std::vector<double> xp((size_t)M * K);
   for (int m = 0; m < M; ++m)
     for (int j = 0; j < K; ++j) {
@@ -308,7 +319,7 @@ void svqref_linear(int N, int K, int b_d, const uint8_t* canon, const uint16_t* 
 // the lowest code.  energy may be NULL (all weights 1).
 // ---------------------------------------------------------------------------
 void svqref_encode(int N, int K, int b_d, const double* W, const uint16_t* codebook,
-                   const uint16_t* scale, const uint16_t* offset, const double* energy,
+                   const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, const double* energy,
                    uint8_t* signs, uint16_t* idx, uint16_t* code) {
   const int G = K / 8, b_r = 10 - b_d;
   const int n_dir = 1 << b_d, n_rad = 1 << b_r;
@@ -316,7 +327,7 @@ void svqref_encode(int N, int K, int b_d, const double* W, const uint16_t* codeb
   for (int e = 0; e < n_dir * 8; ++e) cb[e] = (double)svqref_h2f(codebook[e]);
   for (int n = 0; n < N; ++n) {
     std::vector<double> rad(n_rad);
-    for (int c = 0; c < n_rad; ++c) rad[c] = (double)svqref_radius(scale[n], offset[n], c);
+    for (int c = 0; c < n_rad; ++c) rad[c] = (double)row_radius(scale, offset, lut, b_d, n, c);
     for (int g = 0; g < G; ++g) {
       const double* w = W + (int64_t)n * K + 8 * g;
       const double* e = energy ? energy + 8 * g : nullptr;

@@ -22,6 +22,8 @@ Recipe (every stream is ``Generator(PCG64(SeedSequence([config, matrix, field]))
   field 9  router logits ~ N(0,1) (MoE case).
   field 10 per-matrix bit split choice (MoE case): a fair coin between
            (b_d, b_r) = (7, 3) and (8, 2).
+  field 11 per-row radius look-up tables: 0.5 + cumulative sums of 2^b_r
+           draws of U(1, 2) / 2^b_r per row (increasing levels), rounded to fp16.
 """
 from __future__ import annotations
 
@@ -29,7 +31,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-F_CODEBOOK, F_CODES, F_OFFSET, F_SCALE, F_PERM, F_X, F_ENERGY, F_ROUTER, F_SPLIT = 0, 1, 4, 5, 6, 7, 8, 9, 10
+F_CODEBOOK, F_CODES, F_OFFSET, F_SCALE, F_PERM, F_X, F_ENERGY, F_ROUTER, F_SPLIT, F_LUT = 0, 1, 4, 5, 6, 7, 8, 9, 10, 11
 
 
 def rng(config: int, matrix: int, fld: int) -> np.random.Generator:
@@ -50,6 +52,8 @@ class SvqMatrix:
     scale:     uint16 [N]             fp16 radius scale per row
     offset:    uint16 [N]             fp16 radius offset per row
     perm:      int32 [K]              stored column j multiplies x[perm[j]]
+    lut:       uint16 [N][2^b_r] or None   fp16 radius level of each code, per row
+                                           (replaces scale/offset when present)
     """
     N: int
     K: int
@@ -61,6 +65,7 @@ class SvqMatrix:
     perm: np.ndarray
     name: str = ""
     meta: dict = field(default_factory=dict)
+    lut: np.ndarray | None = None
 
     @property
     def b_r(self) -> int:
@@ -94,6 +99,15 @@ def make_matrix(config: int, matrix: int, N: int, K: int, b_d: int, name: str = 
     else:
         perm = rng(config, matrix, F_PERM).permutation(K).astype(np.int32)
     return SvqMatrix(N, K, b_d, codes, cb, scale, offset, perm, name)
+
+
+def make_lut(config: int, matrix: int, N: int, b_d: int) -> np.ndarray:
+    """Per-row radius levels [N][2^b_r] as fp16 bit patterns: 0.5 plus cumulative sums of U(1, 2) / 2^b_r
+    draws, so each row's levels increase (by at least 2^-b_r: distinct in fp16 for b_r <= 8) over about
+    [0.5, 2]."""
+    nr = 1 << (10 - b_d)
+    lv = 0.5 + np.cumsum(rng(config, matrix, F_LUT).uniform(1.0, 2.0, (N, nr)), axis=1) / nr
+    return lv.astype(np.float16).view(np.uint16)
 
 
 def make_x(config: int, matrix: int, M: int, K: int, dtype: str = "f16",
