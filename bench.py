@@ -486,7 +486,8 @@ def run_gpu(args, world, rank, local):
     if world == 1 and not args.no_secondary:
         del g_all, g_one
         line["secondary"] = {"sweep_8192": run_sweep(args, quiet=True), "prefill": run_prefill(args, quiet=True),
-                             "moe": run_moe(args, quiet=True), "calibration": run_calib(args, quiet=True)}
+                             "moe": run_moe(args, quiet=True), "calibration": run_calib(args, quiet=True),
+                             "layer_radius_tables": run_lut_layer(args, quiet=True)}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -650,6 +651,38 @@ def run_moe(args, quiet=False):
     return recs if quiet else 0
 
 
+def run_lut_layer(args, quiet=False):
+    """The headline decoder layer (one grouped launch, batch 1, 14 rotated copies) with every matrix
+    carrying a per-row radius table (2^b_r fp16 levels) instead of the affine scale/offset."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    stream = torch.cuda.Stream()
+    layers = []
+    for L in range(N_LAYERS):
+        mats = []
+        for i, (m, x) in enumerate(synth.qwen3_4b_layer(L)):
+            m.lut = synth.make_lut(500 + L, i, m.N, m.b_d)
+            mats.append((svq.SvqWeight.from_synth(m),
+                         torch.from_numpy(x.view(np.int16)).cuda().view(torch.float16)))
+        layers.append(mats)
+    ys = [[torch.empty((1, W.N), dtype=torch.float32, device="cuda") for W, _ in mats] for mats in layers]
+    Ws0 = [W for W, _ in layers[0]]
+    ws = torch.zeros(max(svq.svq_linear_gemv_batched_workspace_size(Ws0, 1), 256), dtype=torch.uint8, device="cuda")
+    calls = [svq.GemvBatchCall([W for W, _ in mats], [x for _, x in mats], y, ws) for mats, y in zip(layers, ys)]
+
+    def chain():
+        for c in calls:
+            c()
+    us = _time_graph(chain, 50, stream) / N_LAYERS
+    packed = sum(N * K * 9 // 32 for _, N, K in synth.QWEN3_4B_SHAPES)
+    tables = sum(N * 2 * (1 << (10 - b)) for (_, N, K), b in zip(synth.QWEN3_4B_SHAPES, synth.QWEN3_4B_SPLITS))
+    rec = {"workload": "qwen3-4b decoder layer, batch 1, per-row radius tables", "us_per_layer": round(us, 3),
+           "GBps_packed": round(packed / us / 1e3, 1), "table_bytes_per_layer": tables}
+    if not quiet:
+        print(json.dumps(rec), flush=True)
+    return [rec] if quiet else 0
+
+
 def run_calib(args, quiet=False):
     """Calibration side on one gate-projection-shaped matrix (9728 x 2560): ESG from 512 calibration rows,
     then for each candidate split b_d 6..9 the radius grid and the activation-weighted encode, then ABS.
@@ -793,12 +826,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the sweep / prefill / MoE / calibration measurements added to the headline line")
-    ap.add_argument("--workload", default="layer", choices=["layer", "sweep", "prefill", "moe", "chain", "calib"],
+    ap.add_argument("--workload", default="layer",
+                    choices=["layer", "sweep", "prefill", "moe", "chain", "calib", "lut"],
                     help="layer = the headline line; the others print one JSON line per configuration")
     args = ap.parse_args()
     if args.workload != "layer":
         return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe, "chain": run_chain,
-                "calib": run_calib}[args.workload](args)
+                "calib": run_calib, "lut": run_lut_layer}[args.workload](args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_init() if args.impl == "svq" else (int(os.environ.get("WORLD_SIZE", "1")),

@@ -30,7 +30,7 @@ class svq_matrix(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int32), ("K", ctypes.c_int32), ("b_d", ctypes.c_int32),
                 ("reserved", ctypes.c_int32), ("packed", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
                 ("radius_scale", ctypes.c_void_p), ("radius_offset", ctypes.c_void_p),
-                ("perm", ctypes.c_void_p)]
+                ("perm", ctypes.c_void_p), ("radius_lut", ctypes.c_void_p)]
 
 
 _lib = None
@@ -77,7 +77,7 @@ def lib():
         "svq_get_device_status": ([P], I),
         "svq_esg": ([P, I, I, ctypes.c_double, P, P, P, P], I),
         "svq_radius_grid": ([P, I, I, P, I, P, P, P], I),
-        "svq_encode": ([P, I, I, I, P, P, P, P, P, P, P, P], I),
+        "svq_encode": ([P, I, I, I, P, P, P, P, P, P, P, P, P], I),
         "svq_abs_select": ([P, I, I, P, P, P], I),
     }
     for name, (args, res) in sig.items():
@@ -134,23 +134,28 @@ def svq_unpack_fields(packed, N: int, K: int, b_d: int, signs, idx, code, stream
 
 
 class SvqWeight:
-    """Device-resident SVQ matrix (packed codes, codebook, radius params, perm) and its
-    C descriptor.  Built from canonical host arrays by ``from_canonical``.  ``perm``
-    None means x is supplied already in the stored column order."""
+    """Device-resident SVQ matrix (packed codes, codebook, radius params, perm, optional per-row radius
+    table) and its C descriptor.  Built from canonical host arrays by ``from_canonical``.  ``perm``
+    None means x is supplied already in the stored column order; ``lut`` (fp16 [N][2^b_r]) replaces the
+    affine radius when given."""
 
-    def __init__(self, N, K, b_d, packed, codebook, scale, offset, perm):
+    def __init__(self, N, K, b_d, packed, codebook, scale, offset, perm, lut=None):
         self.N, self.K, self.b_d = N, K, b_d
         self.packed, self.codebook, self.scale, self.offset, self.perm = packed, codebook, scale, offset, perm
-        self.desc = svq_matrix(N, K, b_d, 0, packed.data_ptr(), codebook.data_ptr(), scale.data_ptr(),
-                               offset.data_ptr(), 0 if perm is None else perm.data_ptr())
+        self.lut = lut
+        ptr = lambda t: 0 if t is None else t.data_ptr()
+        self.desc = svq_matrix(N, K, b_d, 0, packed.data_ptr(), codebook.data_ptr(), ptr(scale), ptr(offset),
+                               ptr(perm), ptr(lut))
 
     def without_perm(self):
         """The same device arrays with perm NULL: its calls take x in stored column order."""
-        return SvqWeight(self.N, self.K, self.b_d, self.packed, self.codebook, self.scale, self.offset, None)
+        return SvqWeight(self.N, self.K, self.b_d, self.packed, self.codebook, self.scale, self.offset, None,
+                         self.lut)
 
     @classmethod
-    def from_canonical(cls, N, K, b_d, canonical, codebook, scale, offset, perm, device="cuda", stream=None):
-        """canonical/codebook/scale/offset/perm: numpy arrays (uint8 / uint16 bit patterns / int32)."""
+    def from_canonical(cls, N, K, b_d, canonical, codebook, scale, offset, perm, device="cuda", stream=None,
+                       lut=None):
+        """canonical/codebook/scale/offset/perm/lut: numpy arrays (uint8 / uint16 bit patterns / int32)."""
         import numpy as np
         import torch
         dev = torch.device(device)
@@ -159,14 +164,15 @@ class SvqWeight:
         svq_repack(canon_d, N, K, b_d, packed, stream)
         to16 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.uint16).view(np.int16)).to(dev)
         w = cls(N, K, b_d, packed, to16(codebook), to16(scale), to16(offset),
-                torch.from_numpy(np.ascontiguousarray(perm, np.int32)).to(dev))
+                torch.from_numpy(np.ascontiguousarray(perm, np.int32)).to(dev),
+                None if lut is None else to16(lut))
         w._canon_d = canon_d   # keep alive until the repack has run
         return w
 
     @classmethod
     def from_synth(cls, m, device="cuda", stream=None):
         return cls.from_canonical(m.N, m.K, m.b_d, m.canonical, m.codebook, m.scale, m.offset, m.perm,
-                                  device, stream)
+                                  device, stream, getattr(m, "lut", None))
 
 
 def svq_dequantize(W: SvqWeight, out, stream=None):
@@ -330,12 +336,13 @@ def svq_radius_grid(W, perm, b_d, scale, offset, stream=None):
            "svq_radius_grid")
 
 
-def svq_encode(W, b_d, perm, weights, codebook, scale, offset, canonical, row_err=None, stream=None):
+def svq_encode(W, b_d, perm, weights, codebook, scale, offset, canonical, row_err=None, stream=None, lut=None):
     """Activation-weighted SVQ encoding of W (fp32 [N][K], natural column order) into the canonical stream
-    (uint8 [N][row_bytes]); row_err (fp64 [N]) receives each row's weighted reconstruction error."""
+    (uint8 [N][row_bytes]); row_err (fp64 [N]) receives each row's weighted reconstruction error.  lut
+    (fp16 [N][2^b_r]) gives per-row radius levels in place of scale/offset."""
     N, K = W.shape
     _check(lib().svq_encode(_ptr(W), N, K, int(b_d), _ptr(perm), _ptr(weights), _ptr(codebook), _ptr(scale),
-                            _ptr(offset), _ptr(canonical), _ptr(row_err), _stream(stream)), "svq_encode")
+                            _ptr(offset), _ptr(lut), _ptr(canonical), _ptr(row_err), _stream(stream)), "svq_encode")
 
 
 def svq_abs_select(row_err, totals, best, stream=None):

@@ -34,10 +34,16 @@ int check_matrix(const svq_matrix* W) {
   if (!W) return SVQ_ERR_INVALID_ARG;
   if (W->b_d < 1 || W->b_d > 10) return SVQ_ERR_UNSUPPORTED_SHAPE;
   if (W->K % 8 != 0 || !svq::layout_supported(W->N, W->K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
-  if (!W->packed || !W->codebook || !W->radius_scale || !W->radius_offset)
-    return SVQ_ERR_INVALID_ARG;
-  if (!aligned(W->packed, 16) || !aligned(W->codebook, 16) || !aligned(W->radius_scale, 2) ||
-      !aligned(W->radius_offset, 2) || (W->perm && !aligned(W->perm, 4)))
+  if (!W->packed || !W->codebook) return SVQ_ERR_INVALID_ARG;
+  if (W->radius_lut) {
+    // per-row radius table: at most 16 levels (b_r <= 4)
+    if (10 - W->b_d > svq::kLutMaxBits) return SVQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(W->radius_lut, 2)) return SVQ_ERR_INVALID_ARG;
+  } else {
+    if (!W->radius_scale || !W->radius_offset) return SVQ_ERR_INVALID_ARG;
+    if (!aligned(W->radius_scale, 2) || !aligned(W->radius_offset, 2)) return SVQ_ERR_INVALID_ARG;
+  }
+  if (!aligned(W->packed, 16) || !aligned(W->codebook, 16) || (W->perm && !aligned(W->perm, 4)))
     return SVQ_ERR_INVALID_ARG;
   return SVQ_OK;
 }
@@ -46,7 +52,7 @@ svq::GemvMatDesc desc_of(const svq_matrix& W, const uint16_t* x, void* y) {
   svq::GemvMatDesc d;
   d.N = W.N; d.K = W.K; d.b_d = W.b_d;
   d.packed = W.packed; d.codebook = W.codebook; d.scale = W.radius_scale; d.offset = W.radius_offset;
-  d.perm = W.perm; d.x = x; d.y = y;
+  d.perm = W.perm; d.lut = W.radius_lut; d.x = x; d.y = y;
   return d;
 }
 
@@ -57,6 +63,8 @@ int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
   for (int i = 0; i < n_mats; ++i) {
     const int st = check_matrix(&mats[i]);
     if (st != SVQ_OK) return st;
+    // one grouped launch: every matrix with a radius table, or none
+    if ((mats[i].radius_lut != nullptr) != (mats[0].radius_lut != nullptr)) return SVQ_ERR_INVALID_ARG;
     descs[i] = desc_of(mats[i], x ? x[i] : nullptr, y ? y[i] : nullptr);
   }
   const int sms = num_sms();
@@ -83,7 +91,9 @@ int plan_group(const svq_matrix* mats, int n_mats, int M, svq::GemvPlan* plan,
   Key key{};
   key.sms = sms; key.M = M; key.n = n_mats;
   for (int i = 0; i < n_mats; ++i) {
-    key.dims[3 * i] = mats[i].N; key.dims[3 * i + 1] = mats[i].K; key.dims[3 * i + 2] = mats[i].b_d;
+    // b_d, plus 16 when the matrix carries a radius table (its shared memory differs)
+    key.dims[3 * i] = mats[i].N; key.dims[3 * i + 1] = mats[i].K;
+    key.dims[3 * i + 2] = mats[i].b_d + (mats[i].radius_lut ? 16 : 0);
   }
   {
     std::lock_guard<std::mutex> lock(mu);
@@ -189,7 +199,7 @@ int svq_dequantize(const svq_matrix* W, int out_dtype, void* w_out, svq_stream_t
   if (!w_out || !aligned(w_out, 16)) return SVQ_ERR_INVALID_ARG;
   if (out_dtype != SVQ_F16 && out_dtype != SVQ_BF16) return SVQ_ERR_INVALID_ARG;
   return cuda_status(svq::launch_dequant(W->packed, W->N, W->K, W->b_d, W->codebook, W->radius_scale,
-                                         W->radius_offset, out_dtype == SVQ_BF16, (uint16_t*)w_out,
+                                         W->radius_offset, W->radius_lut, out_dtype == SVQ_BF16, (uint16_t*)w_out,
                                          (cudaStream_t)stream));
 }
 
@@ -286,6 +296,7 @@ int svq_linear_gemm(const svq_matrix* W, const uint16_t* x, int x_dtype, int M, 
   svq::GemmMatDesc d;
   d.N = W->N; d.K = W->K; d.b_d = W->b_d; d.M = M;
   d.packed = W->packed; d.codebook = W->codebook; d.scale = W->radius_scale; d.offset = W->radius_offset;
+  d.lut = W->radius_lut;
   d.perm = W->perm; d.x = x; d.x_bf16 = x_dtype == SVQ_BF16; d.y = y; d.y_f32 = y_dtype == SVQ_F32;
   return cuda_status(svq::launch_gemm(d, g, workspace, status, (cudaStream_t)stream));
 }
@@ -379,15 +390,17 @@ int svq_radius_grid(const float* W, int N, int K, const int32_t* perm, int b_d, 
 }
 
 int svq_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
-               const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset, uint8_t* canonical,
-               double* row_err, svq_stream_t stream) {
+               const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset, const uint16_t* radius_lut,
+               uint8_t* canonical, double* row_err, svq_stream_t stream) {
   if (N < 1 || K < 8 || K % 8 != 0 || b_d < 1 || b_d > 10) return SVQ_ERR_UNSUPPORTED_SHAPE;
-  if (!W || !codebook || !scale || !offset || !canonical) return SVQ_ERR_INVALID_ARG;
-  if (!aligned(W, 4) || !aligned(codebook, 2) || !aligned(scale, 2) || !aligned(offset, 2) ||
-      (perm && !aligned(perm, 4)) || (weights && !aligned(weights, 4)) || (row_err && !aligned(row_err, 8)))
+  if (radius_lut && 10 - b_d > svq::kLutMaxBits) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  if (!W || !codebook || !canonical || (!radius_lut && (!scale || !offset))) return SVQ_ERR_INVALID_ARG;
+  if (!aligned(W, 4) || !aligned(codebook, 2) || (scale && !aligned(scale, 2)) || (offset && !aligned(offset, 2)) ||
+      (radius_lut && !aligned(radius_lut, 2)) || (perm && !aligned(perm, 4)) || (weights && !aligned(weights, 4)) ||
+      (row_err && !aligned(row_err, 8)))
     return SVQ_ERR_INVALID_ARG;
-  return cuda_status(svq::launch_encode(W, N, K, b_d, perm, weights, codebook, scale, offset, canonical, row_err,
-                                        (cudaStream_t)stream));
+  return cuda_status(svq::launch_encode(W, N, K, b_d, perm, weights, codebook, scale, offset, radius_lut, canonical,
+                                        row_err, (cudaStream_t)stream));
 }
 
 int svq_abs_select(const double* row_err, int n_cand, int N, double* totals, int32_t* best, svq_stream_t stream) {

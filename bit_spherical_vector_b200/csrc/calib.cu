@@ -172,8 +172,9 @@ struct EncodeArgs {
   const int32_t* perm;         // [K] or null
   const float* weights;        // [K] natural order, or null (all 1)
   const uint16_t* codebook;    // fp16 [2^b_d][8]
-  const uint16_t* scale;       // fp16 [N]
+  const uint16_t* scale;       // fp16 [N] (affine radius), or
   const uint16_t* offset;      // fp16 [N]
+  const uint16_t* lut;         // fp16 [N][2^b_r] per-row radius table (when not null)
   uint8_t* canonical;          // [N][row_bytes]
   double* row_err;             // [N] or null
   int N, K, b_d;
@@ -200,23 +201,35 @@ __global__ void __launch_bounds__(kEncWarps * 32, 1) encode_kernel(const EncodeA
   const int n = blockIdx.x * kEncWarps + warp;
   if (n >= a.N) return;
   const int G = a.K / 8;
-  // radius levels of this row: r_c = fma(scale, c, offset) in fp32, widened exactly
-  const float scf = __half2float(__ushort_as_half(a.scale[n])), off = __half2float(__ushort_as_half(a.offset[n]));
+  // radius levels of this row: r_c = fma(scale, c, offset) in fp32, or the table
+  // level lut[n][c]; widened exactly
+  const uint16_t* lrow = a.lut ? a.lut + ((size_t)n << BR) : nullptr;
+  const float scf = lrow ? 0.f : __half2float(__ushort_as_half(a.scale[n]));
+  const float off = lrow ? 0.f : __half2float(__ushort_as_half(a.offset[n]));
+  auto level = [&](int c) -> double {
+    return lrow ? h2d(lrow[c]) : (double)__fmaf_rn(scf, (float)c, off);
+  };
   double rr[kRegR ? NR : 1];
   if constexpr (kRegR) {
 #pragma unroll
-    for (int c = 0; c < NR; ++c) rr[c] = (double)__fmaf_rn(scf, (float)c, off);
+    for (int c = 0; c < NR; ++c) rr[c] = level(c);
   } else {
-    for (int c = lane; c < NR; c += 32) rts[c] = (double)__fmaf_rn(scf, (float)c, off);
+    for (int c = lane; c < NR; c += 32) rts[c] = level(c);
     __syncwarp();
   }
   auto rad = [&](int c) -> double {
     if constexpr (kRegR) return rr[c];
     else return rts[c];
   };
-  // r_c is monotone in c, so the largest |r_c| is at an end
-  const double r_lo = (double)__fmaf_rn(scf, 0.f, off), r_hi = (double)__fmaf_rn(scf, (float)(NR - 1), off);
-  const double rmax2 = fmax(__dmul_rn(r_lo, r_lo), __dmul_rn(r_hi, r_hi)) * (1.0 + 0x1p-50);
+  // the largest r_c^2: at an end of the affine levels (monotone in c), over all table levels
+  double rm2 = 0.0;
+  if (lrow) {
+    for (int c = 0; c < NR; ++c) { const double v = level(c); rm2 = fmax(rm2, __dmul_rn(v, v)); }
+  } else {
+    const double r_lo = level(0), r_hi = level(NR - 1);
+    rm2 = fmax(__dmul_rn(r_lo, r_lo), __dmul_rn(r_hi, r_hi));
+  }
+  const double rmax2 = rm2 * (1.0 + 0x1p-50);
   const float* Wr = a.W + (size_t)n * a.K;
   double row_acc = 0.0;
   for (int g0 = 0; g0 < G; g0 += 32) {
@@ -375,9 +388,10 @@ cudaError_t launch_radius_grid(const float* W, int N, int K, const int32_t* perm
 
 cudaError_t launch_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
                           const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset,
-                          uint8_t* canonical, double* row_err, cudaStream_t st) {
+                          const uint16_t* lut, uint8_t* canonical, double* row_err, cudaStream_t st) {
   EncodeArgs a;
   a.W = W; a.perm = perm; a.weights = weights; a.codebook = codebook; a.scale = scale; a.offset = offset;
+  a.lut = lut;
   a.canonical = canonical; a.row_err = row_err; a.N = N; a.K = K; a.b_d = b_d;
   a.row_bytes = ((size_t)(K / 8) * 18 + 7) / 8;
   switch (10 - b_d) {

@@ -14,7 +14,7 @@ cudaError_t launch_radius_grid(const float* W, int N, int K, const int32_t* perm
                                uint16_t* offset, cudaStream_t st);
 cudaError_t launch_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
                           const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset,
-                          uint8_t* canonical, double* row_err, cudaStream_t st);
+                          const uint16_t* lut, uint8_t* canonical, double* row_err, cudaStream_t st);
 cudaError_t launch_abs_select(const double* row_err, int n_cand, int N, double* totals, int32_t* best,
                               cudaStream_t st);
 

@@ -132,7 +132,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 template <bool BF16>
 __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const uint8_t* pk, uint8_t* a_tile,
                                              const uint8_t* cbs, int lane, int dw, int L, const float (&sc)[4],
-                                             const float (&of)[4]) {
+                                             const float (&of)[4], int row_base) {
   if (lane >= L) return;
   const int kc = dw & 7;                               // 16-byte chunk within the 128-byte A row
   const int r0 = 2 * (dw >> 3);                        // this warp decodes rows r0, r0 + 1 of each lane
@@ -198,7 +198,9 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
     const uint32_t code = pcode[rr];
     const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
     const float scr = r0 == 0 ? sc[rr] : sc[2 + rr], ofr = r0 == 0 ? of[rr] : of[2 + rr];
-    const float rad = __fmaf_rn(scr, (float)code, ofr);
+    // the quantized radius: the row's table level (read through L1), or the affine form
+    const float rad = p.lut ? __half2float(__ushort_as_half(__ldg(p.lut + ((size_t)(row_base + r) << (10 - bd)) + code)))
+                            : __fmaf_rn(scr, (float)code, ofr);
     const float2 rad2 = make_float2(rad, rad);
     const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
     uint32_t o4[4];
@@ -378,7 +380,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       // radius parameters of this lane's 4 rows of the unit's row tile
       const int L = tile_lanes(p.N, w.nt);
       float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
-      if (lane < L) {
+      if (lane < L && !p.lut) {
         const int n0 = w.nt * kTileRows + 4 * lane;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -398,7 +400,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
         }
         good = __shfl_sync(0xFFFFFFFFu, good, 0);
         if (!good) { ok = false; break; }
-        decode_stage<BF16>(p, kb, p_st + sp * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d, L, sc, of);
+        decode_stage<BF16>(p, kb, p_st + sp * kPTileBytes, a_st + s * kATileBytes, cbs, lane, d, L, sc, of,
+                           w.nt * kTileRows + 4 * lane);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -640,7 +643,8 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   CUtensorMap tw = tm;
   if (g.dense) {
     uint16_t* wdec = reinterpret_cast<uint16_t*>(wsb + g.wdec_offset);
-    cudaError_t e = launch_dequant(d.packed, d.N, d.K, d.b_d, d.codebook, d.scale, d.offset, d.x_bf16, wdec, st);
+    cudaError_t e = launch_dequant(d.packed, d.N, d.K, d.b_d, d.codebook, d.scale, d.offset, d.lut, d.x_bf16, wdec,
+                                   st);
     if (e != cudaSuccess) return e;
     const cuuint64_t wdims[2] = {(cuuint64_t)d.K, (cuuint64_t)d.N};
     const cuuint32_t wbox[2] = {64, (cuuint32_t)kTileRows};
@@ -655,6 +659,7 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.codebook = reinterpret_cast<const uint4*>(d.codebook);
   p.scale = d.scale;
   p.offset = d.offset;
+  p.lut = d.lut;
   p.N = d.N; p.K = d.K; p.b_d = d.b_d; p.M = d.M;
   p.n_tiles = g.n_tiles; p.m_tiles = g.m_tiles; p.S = g.S;
   p.cb_replicas = d.b_d <= 8 ? 8 : (d.b_d == 9 ? 4 : 2);

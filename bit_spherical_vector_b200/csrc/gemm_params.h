@@ -12,6 +12,7 @@ struct GemmKParams {
   const uint4* codebook;
   const uint16_t* scale;
   const uint16_t* offset;
+  const uint16_t* lut;  // per-row radius table [N][2^b_r], or null (affine radius)
   int N, K, b_d, M;
   int n_tiles, m_tiles, S;
   int cb_replicas;
@@ -35,6 +36,7 @@ struct GemmMatDesc {
   const uint16_t* codebook;
   const uint16_t* scale;
   const uint16_t* offset;
+  const uint16_t* lut;  // per-row radius table or null
   const int32_t* perm;
   const uint16_t* x;    // [M][K], fp16 or bf16 (x_bf16)
   int x_bf16;

@@ -40,16 +40,21 @@ long long cta_of(long long q, long long T, long long G) { return ((q + 1) * G - 
 // codebook replicas + two x slots per warp + per-warp partial sums of npw tiles
 // + 36 ints (warp range boundaries and first tiles) + one completion counter per tile of a CTA's
 // range (at most ntc tiles)
-size_t cta_smem(int b_d, int mt, int npw, int ntc) {
+size_t cta_smem(int b_d, int mt, int npw, int ntc, bool lut) {
   const int R = gemv_cb_replicas(b_d);
   const int W = gemv_warps(mt);
+  // (lut) the radius levels of the CTA's tiles, fp32 [tile][code][4][32]
+  const size_t lut_bytes = lut ? ((size_t)ntc << (10 - b_d)) * kTileRows * sizeof(float) : 0;
   return ((size_t)16 * R << b_d) + (size_t)W * 2 * mt * kBlockCols * 2 +
-         (size_t)W * npw * mt * kTileRows * sizeof(float) + 144 + ((size_t)ntc * 4 + 15) / 16 * 16;
+         (size_t)W * npw * mt * kTileRows * sizeof(float) + 144 + ((size_t)ntc * 4 + 15) / 16 * 16 + lut_bytes;
 }
 
 }  // namespace
 
 bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan* plan) {
+  // a grouped launch either gives every matrix a radius table or none (one kernel per case)
+  for (int i = 1; i < n_mats; ++i)
+    if ((mats[i].lut != nullptr) != (mats[0].lut != nullptr)) return false;
   if (n_mats < 1 || n_mats > kGemvMaxMats || M < 1 || num_sms < 1) return false;
   const int mt = M >= 5 ? 8 : (M >= 3 ? 4 : M);
   const int W = gemv_warps(mt);
@@ -122,7 +127,7 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
       }
       total += pm.ctas;
       const int ntc = (int)((cta_len - 1 + B[i] - 1) / B[i] + 1);
-      smem = std::max(smem, cta_smem(mats[i].b_d, mt, pm.npw, ntc));
+      smem = std::max(smem, cta_smem(mats[i].b_d, mt, pm.npw, ntc, mats[i].lut != nullptr));
     }
     if (counters > kGemvMaxCounters) return false;
     if (counters == 0) off = 0;
@@ -154,6 +159,7 @@ cudaError_t launch_gemv(const GemvMatDesc* mats, const GemvPlan& plan, int y_f32
       g.scale = d.scale;
       g.offset = d.offset;
       g.perm = d.perm;
+      g.lut = d.lut;
       g.x = d.x + (size_t)m0 * d.K;
       g.y = reinterpret_cast<char*>(d.y) + (size_t)m0 * d.N * (y_f32 ? 4 : 2);
       if (pm.kmax > 1) {

@@ -123,11 +123,17 @@ __device__ __forceinline__ CbShift cb_shift(int b_d, int R) {
 
 __device__ __forceinline__ CbShift cb_shift(int b_d) { return cb_shift(b_d, cb_replicas(b_d)); }
 
-template <int MT>
+// kLut: the radius of row r (of the lane's 4) and code c is the table level
+// lut_lane[(c * 4 + r) * 32] (lut_lane = the tile's shared-memory table
+// [code][row of lane][lane] plus this lane; conflict free), instead of
+// scp * v + ofp.
+template <int MT, bool kLut = false>
 __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const unsigned char* xb,
                                               int xstride_bytes, const unsigned char* cbs, uint32_t q16,
                                               const CbShift& cs, uint32_t CODEM, const float2 (&scp)[2],
-                                              const float2 (&ofp)[2], float2 (&acc)[2][MT]) {
+                                              const float2 (&ofp)[2], float2 (&acc)[2][MT],
+                                              const float* lut_lane = nullptr, int bd = 0) {
+  const uint32_t cmask_l = kLut ? (1u << (10 - bd)) - 1u : 0u;
   uint32_t w[kWords];
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
@@ -141,6 +147,7 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
     const uint32_t S = w[j];
     float vf[4];
     float dsum[4][MT];
+    uint32_t cdl[4];                                 // (kLut) radius code of each row
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int v = 4 * j + r;
@@ -152,6 +159,7 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
           case 1: ia = (pw >> cs.r1) & cs.mask; vb = shl<3>(pw) & CODEM; break;
           default: ia = (pw >> cs.r2) & cs.mask; vb = shl<-7>(pw) & CODEM; break;
         }
+        if constexpr (kLut) cdl[r] = (pw >> (bd + 10 * (v % 3))) & cmask_l;
       } else {
         const int a = v - 60;
         const uint32_t pw = ((w[16 + 5 * a] >> 30) << 8) | ((w[17 + 5 * a] >> 30) << 6) |
@@ -159,6 +167,7 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
                             (w[20 + 5 * a] >> 30);
         ia = (pw << cs.l0) & cs.mask;
         vb = shl<13>(pw) & CODEM;
+        if constexpr (kLut) cdl[r] = (pw >> bd) & cmask_l;
       }
       // replica offset q16 (below bit l0) and the scaled index do not overlap: OR, not add
       uint4 cw = lds128(cbs, ia | q16);
@@ -177,9 +186,15 @@ __device__ __forceinline__ void process_block(const uint4 (&d)[kChunks], const u
         dsum[r][m] = s8;
       }
     }
-    // radius r = scp * v + ofp and accumulation, two rows per packed fp32x2 FMA
-    const float2 r01 = __ffma2_rn(scp[0], make_float2(vf[0], vf[1]), ofp[0]);
-    const float2 r23 = __ffma2_rn(scp[1], make_float2(vf[2], vf[3]), ofp[1]);
+    // radius r = scp * v + ofp (or the table level) and accumulation, two rows per packed fp32x2 FMA
+    float2 r01, r23;
+    if constexpr (kLut) {
+      r01 = make_float2(lut_lane[(cdl[0] * 4 + 0) * 32], lut_lane[(cdl[1] * 4 + 1) * 32]);
+      r23 = make_float2(lut_lane[(cdl[2] * 4 + 2) * 32], lut_lane[(cdl[3] * 4 + 3) * 32]);
+    } else {
+      r01 = __ffma2_rn(scp[0], make_float2(vf[0], vf[1]), ofp[0]);
+      r23 = __ffma2_rn(scp[1], make_float2(vf[2], vf[3]), ofp[1]);
+    }
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       acc[0][m] = __ffma2_rn(r01, make_float2(dsum[0][m], dsum[1][m]), acc[0][m]);

@@ -155,7 +155,9 @@ __device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, co
 // One CTA = one contiguous range of one matrix's blocks.  kPerm: the matrix has
 // a permutation (x is gathered through it); without one, x is already in stored
 // column order and lane l reads columns l, l+32, l+64, l+96 of each block.
-template <int MT, bool kPerm>
+// kLut: the matrix carries a per-row radius table (g.lut): the levels of the
+// CTA's row tiles are staged in shared memory by the prologue.
+template <int MT, bool kPerm, bool kLut>
 __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char* smem, int y_f32) {
   constexpr int W = gemv_warps(MT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,6 +199,9 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   float* red = reinterpret_cast<float*>(smem + ((size_t)16 * R << BD) + (size_t)W * 2 * kXSlot);
   int* rbt = reinterpret_cast<int*>(red + (size_t)W * npw * MT * kTileRows);
   int* tcnt = rbt + 36;
+  // (kLut) radius levels of tiles ta..tb as fp32, [tile][code][row of lane][lane]
+  float* lutsm = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(tcnt) +
+                                          ((size_t)(tb - ta + 1) * 4 + 15) / 16 * 16);
   for (int i = threadIdx.x; i <= tb - ta; i += blockDim.x) tcnt[i] = 0;
   if (threadIdx.x <= W) rbt[threadIdx.x] = range_begin(threadIdx.x);
   if (threadIdx.x < W) rbt[W + 1 + threadIdx.x] = range_begin(threadIdx.x) / B;   // first tile of range
@@ -232,7 +237,31 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   // (kept as raw fp16 bits until they are needed, so the loads stay in flight
   // through the rest of the prologue)
   uint16_t sc[4] = {0, 0, 0, 0}, of[4] = {0, 0, 0, 0};
-  if (nb > 0 && lane < L_cur) {
+  if constexpr (kLut) {
+    // the per-row radius tables of the CTA's tiles: eight loads in flight per
+    // thread before their stores (weights: read before the dependency wait)
+    const int nrl = 1 << BR, per_tile = kTileRows << BR, total = (tb - ta + 1) * per_tile;
+    for (int i0 = threadIdx.x; i0 < total; i0 += 8 * blockDim.x) {
+      uint16_t hv[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = i0 + k * blockDim.x;
+        const int tt = i / per_tile, rem = i - tt * per_tile;
+        const int n = (ta + tt) * kTileRows + (rem >> BR);
+        hv[k] = (i < total && n < N) ? ldg_keep_u16(g.lut + (size_t)n * nrl + (rem & (nrl - 1)), pol_keep)
+                                     : (uint16_t)0;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int i = i0 + k * blockDim.x;
+        if (i >= total) break;
+        const int tt = i / per_tile, rem = i - tt * per_tile;
+        const int row = rem >> BR, code = rem & (nrl - 1);
+        lutsm[((tt * nrl + code) * 4 + (row & 3)) * 32 + (row >> 2)] = __half2float(__ushort_as_half(hv[k]));
+      }
+    }
+  }
+  if (!kLut && nb > 0 && lane < L_cur) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       sc[r] = ldg_keep_u16(g.scale + t_cur * kTileRows + 4 * lane + r, pol_keep);
@@ -329,7 +358,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
       L_next = tile_lanes(N, t_next);
       if (lane < L_next) {
         load_block(d1, block_ptr(qn, L_next), L_next, lane, pol_stream);
-        if (t_next != t_cur) {
+        if (!kLut && t_next != t_cur) {
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             sc[r] = ldg_keep_u16(g.scale + t_next * kTileRows + 4 * lane + r, pol_keep);
@@ -338,7 +367,9 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
         }
       }
     }
-    if (lane < L_cur) process_block<MT>(d0, xs + (b & 1) * kXSlot, kBlockCols * 2, cbb, q16, cs, CODEM, scp, ofp, acc);
+    if (lane < L_cur)
+      process_block<MT, kLut>(d0, xs + (b & 1) * kXSlot, kBlockCols * 2, cbb, q16, cs, CODEM, scp, ofp, acc,
+                              lutsm + ((size_t)(t_cur - ta) << BR) * kTileRows + lane, BD);
 #pragma unroll
     for (int k = 0; k < kChunks; ++k) d0[k] = d1[k];
     if (b + 1 == nb || t_next != t_cur) {
@@ -373,7 +404,8 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 // PM: 1 = every matrix of the launch has a permutation, 0 = none has, 2 = mixed
 // (each CTA follows its own matrix).  The uniform cases get kernels of their own
 // so each is compiled (registers, schedule) for one path only.
-template <int MT, int PM>
+// LM: every matrix of the launch carries a per-row radius table (or none does).
+template <int MT, int PM, bool LM>
 __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
 gemv_kernel(const __grid_constant__ GemvKParams P) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -382,23 +414,23 @@ gemv_kernel(const __grid_constant__ GemvKParams P) {
   const GemvKMat& g = P.mats[mi];
   const int c = (int)blockIdx.x - g.cta_begin;
   if constexpr (PM == 1) {
-    gemv_cta<MT, true>(g, c, smem, P.y_f32);
+    gemv_cta<MT, true, LM>(g, c, smem, P.y_f32);
   } else if constexpr (PM == 0) {
-    gemv_cta<MT, false>(g, c, smem, P.y_f32);
+    gemv_cta<MT, false, LM>(g, c, smem, P.y_f32);
   } else {
-    if (g.perm) gemv_cta<MT, true>(g, c, smem, P.y_f32);
-    else gemv_cta<MT, false>(g, c, smem, P.y_f32);
+    if (g.perm) gemv_cta<MT, true, LM>(g, c, smem, P.y_f32);
+    else gemv_cta<MT, false, LM>(g, c, smem, P.y_f32);
   }
 }
 
-template <int MT, int PM>
+template <int MT, int PM, bool LM>
 cudaError_t launch_gemv_pm(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
   static std::atomic<unsigned long long> attr_set{0};   // one bit per device (setting it twice is harmless)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !((attr_set.load(std::memory_order_acquire) >> dev) & 1ull)) {
-    e = cudaFuncSetAttribute(gemv_kernel<MT, PM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(gemv_kernel<MT, PM, LM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kGemvSmemMax);
     if (e != cudaSuccess) return e;
     if (dev < 64) attr_set.fetch_or(1ull << dev, std::memory_order_release);
@@ -416,20 +448,29 @@ cudaError_t launch_gemv_pm(const GemvKParams& p, int grid, size_t smem, cudaStre
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT, PM>, p);
+  e = cudaLaunchKernelEx(&cfg, gemv_kernel<MT, PM, LM>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
+template <int MT, bool LM>
+cudaError_t launch_gemv_lm(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
+  int with = 0;
+  for (int i = 0; i < p.n_mats; ++i) with += p.mats[i].perm != nullptr;
+  if (with == p.n_mats) return launch_gemv_pm<MT, 1, LM>(p, grid, smem, st);
+  if (with == 0) return launch_gemv_pm<MT, 0, LM>(p, grid, smem, st);
+  return launch_gemv_pm<MT, 2, LM>(p, grid, smem, st);
+}
+
 template <int MT>
 cudaError_t launch_gemv_mt(const GemvKParams& p, int grid, size_t smem, cudaStream_t st) {
   int with = 0;
-  for (int i = 0; i < p.n_mats; ++i) with += p.mats[i].perm != nullptr;
-  if (with == p.n_mats) return launch_gemv_pm<MT, 1>(p, grid, smem, st);
-  if (with == 0) return launch_gemv_pm<MT, 0>(p, grid, smem, st);
-  return launch_gemv_pm<MT, 2>(p, grid, smem, st);
+  for (int i = 0; i < p.n_mats; ++i) with += p.mats[i].lut != nullptr;
+  if (with == p.n_mats) return launch_gemv_lm<MT, true>(p, grid, smem, st);
+  if (with == 0) return launch_gemv_lm<MT, false>(p, grid, smem, st);
+  return cudaErrorInvalidValue;                        // mixed: refused by the planner already
 }
 
 }  // namespace svq

@@ -16,6 +16,7 @@ struct GemvKMat {
   const uint16_t* scale;
   const uint16_t* offset;
   const int32_t* perm;    // [K]
+  const uint16_t* lut;    // per-row radius table [N][2^b_r], or null
   const uint16_t* x;      // fp16 [M][K], natural input order
   void* y;                // [M][N]
   float* partial;         // [n_tiles][kmax][MT][128] when kmax > 1

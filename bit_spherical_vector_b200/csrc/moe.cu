@@ -226,7 +226,10 @@ __device__ __forceinline__ void moe_tile(const MoeKParams& p, const svq_matrix& 
   const uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
   const int wb0 = (B * warp) / kMoeWarps, wb1 = (B * (warp + 1)) / kMoeWarps, nb = wb1 - wb0;
   const int L = tile_lanes(N, t);
-  const bool on = lane < L;
+  // matrices with a per-row radius table are not taken here: reported, decoded as zeros
+  const bool lut_refused = W.radius_lut != nullptr;
+  if (lut_refused && threadIdx.x == 0) atomicExch(p.status, SVQ_ERR_INVALID_ARG);
+  const bool on = lane < L && !lut_refused;
   const int row0 = t * kTileRows + 4 * lane;
   const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
   const uint8_t* tile_base = reinterpret_cast<const uint8_t*>(W.packed) + tile_offset(K, t);

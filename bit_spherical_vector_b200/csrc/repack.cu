@@ -176,7 +176,7 @@ __global__ void unpack_kernel(const uint8_t* __restrict__ packed, int N, int K, 
 __global__ void dequant_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d,
                                const uint16_t* __restrict__ codebook,
                                const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-                               int out_bf16, uint16_t* __restrict__ out) {
+                               const uint16_t* __restrict__ lut, int out_bf16, uint16_t* __restrict__ out) {
   const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= num_lane_blocks(N, K)) return;
   const LaneBlockId lb = lane_block_id(N, K, id);
@@ -189,12 +189,14 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, int N, int K,
   const uint32_t imask = (1u << b_d) - 1u;
   for (int r = 0; r < 4; ++r) {
     const int n = lb.t * kTileRows + 4 * lb.l + r;
-    const float sc = __half2float(__ushort_as_half(scale[n]));
-    const float of = __half2float(__ushort_as_half(offset[n]));
+    const float sc = lut ? 0.f : __half2float(__ushort_as_half(scale[n]));
+    const float of = lut ? 0.f : __half2float(__ushort_as_half(offset[n]));
     for (int j = 0; j < 16; ++j) {
       const uint32_t id_ = p[j][r] & imask;
       const uint32_t cd = p[j][r] >> b_d;
-      const float rad = __fmaf_rn(sc, (float)cd, of);
+      // the quantized radius: per-row table level, or the affine form
+      const float rad = lut ? __half2float(__ushort_as_half(lut[((size_t)n << (10 - b_d)) + cd]))
+                            : __fmaf_rn(sc, (float)cd, of);
       uint16_t vals[8];
       for (int i = 0; i < 8; ++i) {
         const float c = __half2float(__ushort_as_half(codebook[id_ * 8 + i]));
@@ -234,11 +236,11 @@ cudaError_t launch_unpack(const void* packed, int N, int K, int b_d, uint8_t* si
 }
 
 cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
-                           const uint16_t* scale, const uint16_t* offset, int out_bf16, uint16_t* out,
-                           cudaStream_t st) {
+                           const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
+                           uint16_t* out, cudaStream_t st) {
   const long long work = (long long)(N / kRowsPerLane) * (K / kBlockCols);
   dequant_kernel<<<grid_for(work, 128), 128, 0, st>>>((const uint8_t*)packed, N, K, b_d, codebook, scale,
-                                                      offset, out_bf16, out);
+                                                      offset, lut, out_bf16, out);
   return cudaGetLastError();
 }
 

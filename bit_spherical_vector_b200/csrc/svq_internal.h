@@ -11,9 +11,12 @@ namespace svq {
 cudaError_t launch_repack(const uint8_t* canon, int N, int K, int b_d, void* out, cudaStream_t st);
 cudaError_t launch_unpack(const void* packed, int N, int K, int b_d, uint8_t* signs, uint16_t* idx,
                           uint16_t* code, cudaStream_t st);
+// Per-row radius tables (svq_matrix.radius_lut): at most 2^kLutMaxBits levels.
+constexpr int kLutMaxBits = 4;
+
 cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
-                           const uint16_t* scale, const uint16_t* offset, int out_bf16, uint16_t* out,
-                           cudaStream_t st);
+                           const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
+                           uint16_t* out, cudaStream_t st);
 
 // ---------------------------------------------------------------- producers
 constexpr int kMaxProducerOuts = 8;
@@ -42,6 +45,7 @@ struct GemvMatDesc {                      // host-side description of one matrix
   const uint16_t* scale;
   const uint16_t* offset;
   const int32_t* perm;
+  const uint16_t* lut;                   // per-row radius table [N][2^b_r] or null
   const uint16_t* x;                     // fp16 [M][K]
   void* y;                               // [M][N]
 };

@@ -62,7 +62,13 @@ enum svq_dtype { SVQ_F16 = 1, SVQ_BF16 = 2, SVQ_F32 = 3 };
  * order (the producer of x applied the permutation, as a decoder layer does
  * when the previous kernel writes its output permuted), every call below reads
  * x[m][j] for column j, and the permutation pass of svq_linear_gemm is
- * skipped. */
+ * skipped.
+ * The quantized radius (Figure 2 caption) of row n and radius code c is
+ *   r = fmaf(radius_scale[n], c, radius_offset[n])  (fp32, affine form), or,
+ *   when radius_lut is not NULL, r = radius_lut[n][c] (a per-row table of
+ *   2^b_r fp16 levels: levels fitted freely, as the pages optimise them; then
+ *   radius_scale and radius_offset are not read and may be NULL).  The table
+ *   form needs b_r <= 4 (b_d >= 6); svq_moe_grouped_gemv does not take it. */
 typedef struct svq_matrix {
   int32_t N;                      /* output features (rows of W)                            */
   int32_t K;                      /* input features                                         */
@@ -73,6 +79,7 @@ typedef struct svq_matrix {
   const uint16_t* radius_scale;   /* fp16 [N]                                               */
   const uint16_t* radius_offset;  /* fp16 [N]                                               */
   const int32_t* perm;            /* [K], a permutation of 0..K-1, 4-byte aligned, or NULL  */
+  const uint16_t* radius_lut;     /* fp16 [N][1 << (10 - b_d)], 2-byte aligned, or NULL      */
 } svq_matrix;
 
 /* Message for a status code (static string). */
@@ -351,6 +358,8 @@ SVQ_API int svq_swiglu_permute(const float* gate, const float* up, int M, int I,
  * evaluated term by term in fp64 (i ascending), ties to the lowest idx, then
  * the lowest code -- the brute-force choice, reached without evaluating every
  * pair (a filter with a proven error bound skips pairs that cannot win).
+ * With radius_lut (fp16 [N][2^b_r], b_r <= 4) the levels are r_code =
+ * radius_lut[n][code] and scale/offset are not read (may be NULL).
  * codebook: fp16 [2^b_d][8]; scale, offset: fp16 [N]; canonical: [N][row
  * bytes of svq_canonical_bytes] out, pad bits zero; row_err: fp64 [N] out or
  * NULL: sum_j e_j (W[n][perm[j]] - What[n][j])^2 over the row (What the exact
@@ -368,8 +377,8 @@ SVQ_API int svq_esg(const float* x_cal, int T, int K, double gamma, double* ener
 SVQ_API int svq_radius_grid(const float* W, int N, int K, const int32_t* perm, int b_d, uint16_t* scale,
                             uint16_t* offset, svq_stream_t stream);
 SVQ_API int svq_encode(const float* W, int N, int K, int b_d, const int32_t* perm, const float* weights,
-                       const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset, uint8_t* canonical,
-                       double* row_err, svq_stream_t stream);
+                       const uint16_t* codebook, const uint16_t* scale, const uint16_t* offset,
+                       const uint16_t* radius_lut, uint8_t* canonical, double* row_err, svq_stream_t stream);
 SVQ_API int svq_abs_select(const double* row_err, int n_cand, int N, double* totals, int32_t* best,
                            svq_stream_t stream);
 

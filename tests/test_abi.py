@@ -71,7 +71,7 @@ def test_header_compiles_as_c_and_links(tmp_path):
     src.write_text(
         '#include <stdio.h>\n#include "svq.h"\n'
         "int main(void) {\n"
-        "  svq_matrix m = {128, 128, 8, 0, 0, 0, 0, 0, 0};\n"
+        "  svq_matrix m = {128, 128, 8, 0, 0, 0, 0, 0, 0, 0};\n"
         "  size_t n = 0;\n"
         "  int st = svq_linear_gemv_workspace_size(&m, 1, &n);\n"
         '  printf("%zu %zu %d %s\\n", svq_packed_bytes(1024, 1024), svq_canonical_bytes(3, 40), st,\n'
