@@ -158,7 +158,8 @@ const char* svq_status_string(int status) {
   switch (status) {
     case SVQ_OK: return "ok";
     case SVQ_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad enum or batch size)";
-    case SVQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (needs K % 128 == 0, N % 4 == 0, 1 <= b_d <= 10)";
+    case SVQ_ERR_UNSUPPORTED_SHAPE:
+      return "unsupported shape (needs K % 8 == 0, 1 <= b_d <= 10; radius tables b_r <= 4; MoE K % 128 == 0 and N % 4 == 0)";
     case SVQ_ERR_WORKSPACE: return "workspace missing or too small";
     case SVQ_ERR_CUDA: return "CUDA runtime error";
     case SVQ_ERR_TIMEOUT: return "a kernel's bounded wait timed out";
@@ -313,7 +314,9 @@ int svq_moe_grouped_gemv(const svq_matrix* mats, int n_mats, int N, int K, int m
                          svq_stream_t stream) {
   if (!mats || !items || !x || !y || n_mats < 1 || n_items < 1 || n_out_rows < 1 || n_x_rows < 1)
     return SVQ_ERR_INVALID_ARG;
-  if (max_b_d < 1 || max_b_d > 10 || !svq::layout_supported(N, K)) return SVQ_ERR_UNSUPPORTED_SHAPE;
+  // the grouped MoE kernel takes only shapes that need no padding
+  if (max_b_d < 1 || max_b_d > 10 || !svq::layout_supported(N, K) || N % 4 != 0 || K % 128 != 0)
+    return SVQ_ERR_UNSUPPORTED_SHAPE;
   if (n_mats > 16384 || max_items_per_matrix < 1) return SVQ_ERR_INVALID_ARG;
   if (x_mode != SVQ_X_F16 && x_mode != SVQ_X_SWIGLU_F32) return SVQ_ERR_INVALID_ARG;
   if (!aligned(mats, 8) || !aligned(items, 4) || !aligned(y, 4) || !aligned(x, x_mode == SVQ_X_F16 ? 2 : 4))

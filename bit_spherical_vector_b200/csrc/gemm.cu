@@ -105,7 +105,7 @@ __device__ __forceinline__ Unit unit_of(const GemmKParams& p, int u) {
   const int rest = u / p.n_tiles;
   w.s = rest % p.S;
   w.mt = rest / p.S;
-  const int KB = p.K / 64;
+  const int KB = pad_cols(p.K) / 64;                  // 64-column blocks of the (padded) layout
   w.kb0 = (int)(((long long)KB * w.s) / p.S);
   w.kb1 = (int)(((long long)KB * (w.s + 1)) / p.S);
   return w;
@@ -199,7 +199,10 @@ __device__ __forceinline__ void decode_stage(const GemmKParams& p, int kb, const
     const uint4 cw = *reinterpret_cast<const uint4*>(cbq + id * cb_stride);
     const float scr = r0 == 0 ? sc[rr] : sc[2 + rr], ofr = r0 == 0 ? of[rr] : of[2 + rr];
     // the quantized radius: the row's table level (read through L1), or the affine form
-    const float rad = p.lut ? __half2float(__ushort_as_half(__ldg(p.lut + ((size_t)(row_base + r) << (10 - bd)) + code)))
+    const bool real_row = row_base + r < p.N;          // padding rows of a ragged N decode as zeros
+    const float rad = p.lut ? (real_row ? __half2float(__ushort_as_half(
+                                             __ldg(p.lut + ((size_t)(row_base + r) << (10 - bd)) + code)))
+                                       : 0.f)
                             : __fmaf_rn(scr, (float)code, ofr);
     const float2 rad2 = make_float2(rad, rad);
     const uint32_t c4[4] = {cw.x, cw.y, cw.z, cw.w};
@@ -302,10 +305,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           const int s = itp % NP;
           const uint32_t ph = (itp / NP) & 1;
           if (itp >= NP && !wait_bar(&bars->empty_p[s], ph ^ 1, p, bars)) { ok = false; break; }
-          const int L = tile_lanes(p.N, cp_.w.nt);
+          const int L = tile_lanes(pad_rows(p.N), cp_.w.nt);
           const uint32_t pbytes = (uint32_t)L * kLaneBlockBytes;
           mbar_arrive_expect_tx(&bars->full_p[s], pbytes);
-          bulk_load(p_st + s * kPTileBytes, p.packed + tile_offset(p.K, cp_.w.nt) + (size_t)(cp_.kb >> 1) * pbytes,
+          bulk_load(p_st + s * kPTileBytes, p.packed + tile_offset(pad_cols(p.K), cp_.w.nt) + (size_t)(cp_.kb >> 1) * pbytes,
                     pbytes, &bars->full_p[s]);
           advance(cp_);
           ++itp;
@@ -378,14 +381,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const Unit w = unit_of(p, u);
       // radius parameters of this lane's 4 rows of the unit's row tile
-      const int L = tile_lanes(p.N, w.nt);
+      const int L = tile_lanes(pad_rows(p.N), w.nt);
       float sc[4] = {0.f, 0.f, 0.f, 0.f}, of[4] = {0.f, 0.f, 0.f, 0.f};
       if (lane < L && !p.lut) {
         const int n0 = w.nt * kTileRows + 4 * lane;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          sc[r] = __half2float(__ushort_as_half(p.scale[n0 + r]));
-          of[r] = __half2float(__ushort_as_half(p.offset[n0 + r]));
+        for (int r = 0; r < 4; ++r) {                  // rows past N (padding) decode with zeros
+          sc[r] = n0 + r < p.N ? __half2float(__ushort_as_half(p.scale[n0 + r])) : 0.f;
+          of[r] = n0 + r < p.N ? __half2float(__ushort_as_half(p.offset[n0 + r])) : 0.f;
         }
       }
       for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
@@ -455,16 +458,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           };
           const float4 val = make_float4(pick(0), pick(1), pick(2), pick(3));
           const int n = n0 + 4 * lane;
-          if (split) {
-            float* dst = p.partial + ((size_t)w.s * p.M + m) * p.N + n;
-            *reinterpret_cast<float4*>(dst) = val;
-          } else if (p.y_f32) {
-            *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + (size_t)m * p.N + n) = val;
-          } else {
-            uint2 pk;
-            pk.x = pack2<true>(val.x, val.y);
-            pk.y = pack2<true>(val.z, val.w);
-            *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + (size_t)m * p.N + n) = pk;
+          const size_t o = (size_t)m * p.N + n;           // element of y (or of a partial slice)
+          if ((p.N & 3) == 0) {                           // rows of 4 stay 16-byte aligned
+            if (split) {
+              *reinterpret_cast<float4*>(p.partial + (size_t)w.s * p.part_stride + o) = val;
+            } else if (p.y_f32) {
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + o) = val;
+            } else {
+              uint2 pk;
+              pk.x = pack2<true>(val.x, val.y);
+              pk.y = pack2<true>(val.z, val.w);
+              *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + o) = pk;
+            }
+          } else {                                        // ragged N: element by element, rows < N
+            const float vv[4] = {val.x, val.y, val.z, val.w};
+            for (int r = 0; r < 4 && n + r < p.N; ++r) {
+              if (split) p.partial[(size_t)w.s * p.part_stride + o + r] = vv[r];
+              else if (p.y_f32) reinterpret_cast<float*>(p.y)[o + r] = vv[r];
+              else reinterpret_cast<uint16_t*>(p.y)[o + r] = __bfloat16_as_ushort(__float2bfloat16_rn(vv[r]));
+            }
           }
         }
         named_bar_sync(1, kNumEpi * 32);
@@ -506,23 +518,33 @@ __global__ void permute_kernel(const uint16_t* __restrict__ x, const int32_t* __
 // Split-K reduction: y[m][n] = sum over slices s = 0..S-1 of partial[s][m][n]
 // (in slice order, so the result does not depend on scheduling), four outputs
 // per thread.  Separate from the GEMM so that all SMs share it.
-__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int S, long long MN, void* __restrict__ y,
-                                     int y_f32) {
+// Slices are stride (= MN rounded up to 4) elements apart, so every slice is
+// 16-byte aligned; a last group of fewer than 4 elements is stored one by one.
+__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int S, long long MN, long long stride_el,
+                                     void* __restrict__ y, int y_f32) {
   const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = q; i < MN / 4; i += stride) {
+  for (long long i = q; i < (MN + 3) / 4; i += stride) {
     float4 acc = __ldcs(reinterpret_cast<const float4*>(partial) + i);
     for (int k = 1; k < S; ++k) {
-      const float4 t = __ldcs(reinterpret_cast<const float4*>(partial + (size_t)k * MN) + i);
+      const float4 t = __ldcs(reinterpret_cast<const float4*>(partial + (size_t)k * stride_el) + i);
       acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
     }
-    if (y_f32) {
-      reinterpret_cast<float4*>(y)[i] = acc;
+    if (4 * i + 4 <= MN) {
+      if (y_f32) {
+        reinterpret_cast<float4*>(y)[i] = acc;
+      } else {
+        uint2 pk;
+        pk.x = pack2<true>(acc.x, acc.y);
+        pk.y = pack2<true>(acc.z, acc.w);
+        reinterpret_cast<uint2*>(y)[i] = pk;
+      }
     } else {
-      uint2 pk;
-      pk.x = pack2<true>(acc.x, acc.y);
-      pk.y = pack2<true>(acc.z, acc.w);
-      reinterpret_cast<uint2*>(y)[i] = pk;
+      const float av[4] = {acc.x, acc.y, acc.z, acc.w};
+      for (long long e = 4 * i; e < MN; ++e) {
+        if (y_f32) reinterpret_cast<float*>(y)[e] = av[e - 4 * i];
+        else reinterpret_cast<uint16_t*>(y)[e] = __bfloat16_as_ushort(__float2bfloat16_rn(av[e - 4 * i]));
+      }
     }
   }
 }
@@ -580,9 +602,9 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   GemmPlan g{};
   g.BN = M >= 256 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : (M > 16 ? 32 : 16)));
   g.m_tiles = (M + g.BN - 1) / g.BN;
-  g.n_tiles = num_tiles(N);
+  g.n_tiles = num_tiles(pad_rows(N));
   const int T = g.n_tiles * g.m_tiles;
-  const int KB = K / 64;
+  const int KB = pad_cols(K) / 64;
   // Split K when it shortens the estimated time: waves of units times the
   // k-blocks per unit (about 1 us per 64-column k-block, set by the latency of
   // the staging ring rather than by the MMA), plus the reduction pass over the
@@ -608,7 +630,7 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   g.xp_offset = 0;
   g.wdec_offset = xp;
   g.partial_offset = xp + wdec;
-  const size_t part = g.S > 1 ? ((size_t)g.S * M * N * 4 + 255) / 256 * 256 : 0;
+  const size_t part = g.S > 1 ? ((size_t)g.S * (((size_t)M * N + 3) / 4 * 4) * 4 + 255) / 256 * 256 : 0;
   g.ws_bytes = xp + wdec + part;
   return g;
 }
@@ -666,6 +688,7 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.y = d.y;
   p.y_f32 = d.y_f32;
   p.partial = g.S > 1 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
+  p.part_stride = ((long long)d.M * d.N + 3) / 4 * 4;
   p.status = status;
   p.wait_polls = g_wait_polls.load(std::memory_order_relaxed);
   p.dense = g.dense;
@@ -673,8 +696,8 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
                            : launch_typed<false>(g.BN, tm, tw, p, g.grid, st);
   if (e != cudaSuccess || g.S == 1) return e;
   const long long mn = (long long)d.M * d.N;
-  const long long blocks = std::min<long long>((mn / 4 + 255) / 256, 148LL * 8);
-  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.partial, g.S, mn, d.y, d.y_f32);
+  const long long blocks = std::max<long long>(1, std::min<long long>(((mn + 3) / 4 + 255) / 256, 148LL * 8));
+  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.partial, g.S, mn, p.part_stride, d.y, d.y_f32);
   return cudaGetLastError();
 }
 

@@ -18,7 +18,8 @@ struct GemmKParams {
   int cb_replicas;
   void* y;
   int y_f32;
-  float* partial;       // [S][M][N] when S > 1
+  float* partial;       // [S][part_stride] when S > 1 (slice s: [M][N] row-major)
+  long long part_stride;  // elements between partial slices (M N rounded up to 4)
   int* status;          // device status word (bounded-wait timeouts)
   uint32_t wait_polls;  // polls before a bounded wait gives up (svq_debug_set_wait_polls)
   int dense;            // 1: weight tiles come pre-decoded from the workspace by TMA (decoders idle)

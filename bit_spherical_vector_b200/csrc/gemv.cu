@@ -64,8 +64,8 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
   long long T[kGemvMaxMats], total_blocks = 0;
   int B[kGemvMaxMats];
   for (int i = 0; i < n_mats; ++i) {
-    B[i] = mats[i].K / kBlockCols;
-    T[i] = (long long)num_tiles(mats[i].N) * B[i];
+    B[i] = pad_cols(mats[i].K) / kBlockCols;                    // the (padded) layout's blocks
+    T[i] = (long long)num_tiles(pad_rows(mats[i].N)) * B[i];
     if (T[i] < 1 || T[i] > (1LL << 30)) return false;
     total_blocks += T[i];
   }
@@ -109,7 +109,7 @@ bool plan_gemv(const GemvMatDesc* mats, int n_mats, int M, int num_sms, GemvPlan
       const long long cta_len = (Ti + Gi - 1) / Gi;                // longest CTA range
       const long long warp_len = (cta_len + W - 1) / W;            // longest warp range
       pm.ctas = ctas[i];
-      pm.n_tiles = num_tiles(mats[i].N);
+      pm.n_tiles = num_tiles(pad_rows(mats[i].N));
       pm.npw = (int)((warp_len - 1 + B[i] - 1) / B[i] + 1);
       int kmax = 1;
       for (int t = 0; t < pm.n_tiles; ++t) {

@@ -72,7 +72,7 @@ __device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, co
                                              const int* rb, int ta, bool whole, long long G, long long T,
                                              int npw, int y_f32, int lane) {
   constexpr int W = gemv_warps(MT);
-  const int N = g.N, B = g.K / kBlockCols, M = g.M;
+  const int N = g.N, B = pad_cols(g.K) / kBlockCols, M = g.M;   // blocks of the padded layout
   const int tq0 = t * B, tq1 = tq0 + B;               // blocks of tile t
   __threadfence_block();
   __syncwarp();
@@ -109,13 +109,14 @@ __device__ __noinline__ void tile_piece_done(const GemvKMat& g, int c, int t, co
       const float vv[4] = {v[m].x, v[m].y, v[m].z, v[m].w};
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
+        if (n0 + r >= N) break;                        // padding rows of a ragged N
         const size_t o = (size_t)m * N + n0 + r;
         if (y_f32) reinterpret_cast<float*>(g.y)[o] = vv[r];
         else reinterpret_cast<__half*>(g.y)[o] = __float2half_rn(vv[r]);
       }
     }
   };
-  const bool in_tile = lane < tile_lanes(N, t);
+  const bool in_tile = lane < tile_lanes(pad_rows(N), t);
   if (whole) {                                         // the tile lies wholly in this CTA's range
     if (in_tile) write_y();
     return;
@@ -165,8 +166,10 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   const int R = gemv_cb_replicas(BD);
   const CbShift cs = cb_shift(BD, R);
   const uint32_t CODEM = BR ? (((1u << BR) - 1u) << (23 - BR)) : 0u;
-  const int N = g.N, K = g.K, B = K / kBlockCols, M = g.M, npw = g.npw;
-  const long long T = (long long)num_tiles(N) * B, G = g.ctas;
+  // N, K: the matrix; Np, Kp: its (padded) layout -- columns >= K read x as 0,
+  // rows >= N are computed but never written
+  const int N = g.N, K = g.K, Np = pad_rows(N), Kp = pad_cols(K), B = Kp / kBlockCols, M = g.M, npw = g.npw;
+  const long long T = (long long)num_tiles(Np) * B, G = g.ctas;
   // this CTA's blocks [qa, qb) and this warp's blocks [wq0, wq0 + nb)
   const int qa = (int)(c * T / G), qb = (int)((c + 1) * T / G);
   const int n = qb - qa;
@@ -209,16 +212,24 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
   auto block_ptr = [&](int q, int L) -> const uint8_t* {
     const int t = q / B, kb = q - t * B;
-    return g.packed + tile_offset(K, t) + (size_t)kb * L * kLaneBlockBytes;
+    return g.packed + tile_offset(Kp, t) + (size_t)kb * L * kLaneBlockBytes;
   };
-  auto perm_ptr = [&](int q) -> const int32_t* { return g.perm + (size_t)(q % B) * kBlockCols + lane; };
-  auto cols = [&](int q, int (&pj)[4]) {
+  // x index of this lane's columns of block q (lane + 32u): perm[col], or col;
+  // -1 for padding columns (col >= K), whose activations read as zero
+  auto load_pj = [&](int q, int (&pj)[4]) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) pj[u] = (q % B) * kBlockCols + lane + 32 * u;
+    for (int u = 0; u < 4; ++u) {
+      const int col = (q % B) * kBlockCols + lane + 32 * u;
+      if constexpr (kPerm) pj[u] = col < K ? ldg_keep_i32(g.perm + col, pol_keep) : -1;
+      else pj[u] = col < K ? col : -1;
+    }
+  };
+  auto x_at = [&](int m, int pj) -> uint16_t {
+    return (m < M && pj >= 0) ? ldg_keep_u16(g.x + (size_t)m * K + pj, pol_keep) : (uint16_t)0;
   };
 
   int t_cur = nb > 0 ? q_of(0) / B : 0;
-  int L_cur = tile_lanes(N, t_cur);
+  int L_cur = tile_lanes(Np, t_cur);
   uint4 d0[kChunks], d1[kChunks];
   if (nb > 0 && lane < L_cur) load_block(d0, block_ptr(q_of(0), L_cur), L_cur, lane, pol_stream);
 
@@ -264,27 +275,17 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
   if (!kLut && nb > 0 && lane < L_cur) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      sc[r] = ldg_keep_u16(g.scale + t_cur * kTileRows + 4 * lane + r, pol_keep);
-      of[r] = ldg_keep_u16(g.offset + t_cur * kTileRows + 4 * lane + r, pol_keep);
+      const int n = t_cur * kTileRows + 4 * lane + r;
+      sc[r] = n < N ? ldg_keep_u16(g.scale + n, pol_keep) : (uint16_t)0;
+      of[r] = n < N ? ldg_keep_u16(g.offset + n, pol_keep) : (uint16_t)0;
     }
   }
   // x[perm] pipeline: lane l owns columns l, l+32, l+64, l+96 of a block.  The
   // permutation of block b+2 and the activations of block b+1 are loaded while
   // block b is decoded; the activations land in the other x slot.
-  const uint16_t* xg = g.x;
-  int pj_a[4], pj_b[4];
-  if constexpr (kPerm) {
-    const int32_t* pa = perm_ptr(nb > 0 ? q_of(0) : 0);
-    const int32_t* pb = perm_ptr(nb > 1 ? q_of(1) : 0);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      pj_a[u] = nb > 0 ? ldg_keep_i32(pa + 32 * u, pol_keep) : 0;
-      pj_b[u] = nb > 1 ? ldg_keep_i32(pb + 32 * u, pol_keep) : 0;
-    }
-  } else {
-    cols(nb > 0 ? q_of(0) : 0, pj_a);
-    cols(nb > 1 ? q_of(1) : 0, pj_b);
-  }
+  int pj_a[4] = {-1, -1, -1, -1}, pj_b[4] = {-1, -1, -1, -1};
+  if (nb > 0) load_pj(q_of(0), pj_a);
+  if (nb > 1) load_pj(q_of(1), pj_b);
   // The activations may be written by the previous kernel in the stream
   // (programmatic dependent launch): wait for it before reading x.
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -292,7 +293,7 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
-    for (int u = 0; u < 4; ++u) hx[m][u] = (m < M && nb > 0) ? ldg_keep_u16(xg + (size_t)m * K + pj_a[u], pol_keep) : 0;
+    for (int u = 0; u < 4; ++u) hx[m][u] = x_at(m, pj_a[u]);
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
@@ -339,30 +340,23 @@ __device__ __forceinline__ void gemv_cta(const GemvKMat& g, int c, unsigned char
 #pragma unroll
       for (int m = 0; m < MT; ++m)
 #pragma unroll
-        for (int u = 0; u < 4; ++u) hx[m][u] = m < M ? ldg_keep_u16(xg + (size_t)m * K + pj_b[u], pol_keep) : 0;
-      if (b + 2 < nb) {
-        if constexpr (kPerm) {
-          const int32_t* pn = perm_ptr(q_of(b + 2));
-#pragma unroll
-          for (int u = 0; u < 4; ++u) pj_b[u] = ldg_keep_i32(pn + 32 * u, pol_keep);
-        } else {
-          cols(q_of(b + 2), pj_b);
-        }
-      }
+        for (int u = 0; u < 4; ++u) hx[m][u] = x_at(m, pj_b[u]);
+      if (b + 2 < nb) load_pj(q_of(b + 2), pj_b);
     }
     // packed codes of block b+1, and the radius parameters of its tile if it is a new one
     int t_next = t_cur, L_next = L_cur;
     if (b + 1 < nb) {
       const int qn = q_of(b + 1);
       t_next = qn / B;
-      L_next = tile_lanes(N, t_next);
+      L_next = tile_lanes(Np, t_next);
       if (lane < L_next) {
         load_block(d1, block_ptr(qn, L_next), L_next, lane, pol_stream);
         if (!kLut && t_next != t_cur) {
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            sc[r] = ldg_keep_u16(g.scale + t_next * kTileRows + 4 * lane + r, pol_keep);
-            of[r] = ldg_keep_u16(g.offset + t_next * kTileRows + 4 * lane + r, pol_keep);
+            const int n = t_next * kTileRows + 4 * lane + r;
+            sc[r] = n < N ? ldg_keep_u16(g.scale + n, pol_keep) : (uint16_t)0;
+            of[r] = n < N ? ldg_keep_u16(g.offset + n, pol_keep) : (uint16_t)0;
           }
         }
       }

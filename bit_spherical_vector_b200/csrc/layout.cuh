@@ -9,6 +9,10 @@
 //
 //   tile      = 128 consecutive rows (the last tile may hold fewer; rows % 4 == 0)
 //   block     = 16 consecutive subvectors of every row of a tile (128 columns)
+//   Shapes whose N is not a multiple of 4 or whose K is not a multiple of 128
+//   are stored padded to Np = 4 ceil(N / 4) rows and Kp = 128 ceil(K / 128)
+//   columns with zero codes; the kernels read activation columns >= K as zero
+//   and write no output row >= N, so the padding never contributes.
 //   lane-block= 4 rows x 16 subvectors = 64 codes = 1152 bits = 144 bytes
 //               = 9 x 16-byte chunks, owned by one lane of a warp
 //   A tile with L lanes (L = rows/4) stores its blocks in order; inside a block
@@ -56,12 +60,18 @@ __host__ __device__ inline size_t chunk_offset(int N, int K, int t, int b, int c
   return tile_offset(K, t) + (size_t)b * L * kLaneBlockBytes + ((size_t)c * L + l) * 16;
 }
 
+// Padded layout dimensions (equal to N and K for the aligned shapes).
+__host__ __device__ inline int pad_rows(int N) { return (N + kRowsPerLane - 1) / kRowsPerLane * kRowsPerLane; }
+__host__ __device__ inline int pad_cols(int K) { return (K + kBlockCols - 1) / kBlockCols * kBlockCols; }
+
 __host__ __device__ inline bool layout_supported(int N, int K) {
-  return N > 0 && K > 0 && N % kRowsPerLane == 0 && K % kBlockCols == 0;
+  return N > 0 && K > 0 && K % 8 == 0;
 }
 
+// Bytes of the device layout: exactly N * K * 9 / 32 for aligned shapes, the
+// padded Np * Kp * 9 / 32 otherwise.
 __host__ __device__ inline size_t packed_bytes(int N, int K) {
-  return (size_t)N * (size_t)K * 9 / 32;
+  return (size_t)pad_rows(N) * (size_t)pad_cols(K) * 9 / 32;
 }
 
 }  // namespace svq

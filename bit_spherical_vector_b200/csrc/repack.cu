@@ -110,18 +110,20 @@ __device__ __forceinline__ long long num_lane_blocks(int N, int K) {
 
 __global__ void repack_kernel(const uint8_t* __restrict__ canon, int N, int K, int b_d,
                               uint8_t* __restrict__ out) {
+  const int Np = pad_rows(N), Kp = pad_cols(K), G = K / 8;
   const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= num_lane_blocks(N, K)) return;
-  const LaneBlockId lb = lane_block_id(N, K, id);
+  if (id >= num_lane_blocks(Np, Kp)) return;
+  const LaneBlockId lb = lane_block_id(Np, Kp, id);
   if (!lb.valid) return;
-  const size_t rb = (size_t)K * 9 / 32;               // canonical row bytes (K % 128 == 0)
+  const size_t rb = ((size_t)G * 18 + 7) / 8;         // canonical row bytes
   uint8_t s[16][4];
   uint32_t p[16][4];
   for (int r = 0; r < 4; ++r) {
     const int n = lb.t * kTileRows + 4 * lb.l + r;
     const uint8_t* seg = canon + (size_t)n * rb + (size_t)lb.b * 36;   // 16 codes = 36 bytes
     for (int j = 0; j < 16; ++j) {
-      const uint32_t code = read_code(seg, j);
+      // padding (row >= N or subvector >= K/8): a zero code
+      const uint32_t code = (n < N && lb.b * 16 + j < G) ? read_code(seg, j) : 0u;
       s[j][r] = (uint8_t)(code & 0xFFu);
       p[j][r] = code >> 8;                              // idx | radius << b_d
     }
@@ -131,7 +133,7 @@ __global__ void repack_kernel(const uint8_t* __restrict__ canon, int N, int K, i
   build_words(s, p, w);
   for (int c = 0; c < kChunks; ++c) {
     uint4 v = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
-    *reinterpret_cast<uint4*>(out + chunk_offset(N, K, lb.t, lb.b, c, lb.l)) = v;
+    *reinterpret_cast<uint4*>(out + chunk_offset(Np, Kp, lb.t, lb.b, c, lb.l)) = v;
   }
   // A GEMV launched next on the stream may start (programmatic dependent launch)
   // as soon as every block of this grid has exited, and it reads the packed codes
@@ -139,6 +141,7 @@ __global__ void repack_kernel(const uint8_t* __restrict__ canon, int N, int K, i
   __threadfence();
 }
 
+// (N, K: the padded layout dimensions)
 __device__ void load_words(const uint8_t* packed, int N, int K, const LaneBlockId& lb, uint32_t w[kWords]) {
   for (int c = 0; c < kChunks; ++c) {
     const uint4 v = *reinterpret_cast<const uint4*>(packed + chunk_offset(N, K, lb.t, lb.b, c, lb.l));
@@ -149,12 +152,13 @@ __device__ void load_words(const uint8_t* packed, int N, int K, const LaneBlockI
 __global__ void unpack_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d,
                               uint8_t* __restrict__ signs, uint16_t* __restrict__ idx,
                               uint16_t* __restrict__ code) {
+  const int Np = pad_rows(N), Kp = pad_cols(K);
   const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= num_lane_blocks(N, K)) return;
-  const LaneBlockId lb = lane_block_id(N, K, id);
+  if (id >= num_lane_blocks(Np, Kp)) return;
+  const LaneBlockId lb = lane_block_id(Np, Kp, id);
   if (!lb.valid) return;
   uint32_t w[kWords];
-  load_words(packed, N, K, lb, w);
+  load_words(packed, Np, Kp, lb, w);
   uint8_t s[16][4];
   uint32_t p[16][4];
   split_words(w, s, p);
@@ -162,7 +166,9 @@ __global__ void unpack_kernel(const uint8_t* __restrict__ packed, int N, int K, 
   const uint32_t imask = (1u << b_d) - 1u;
   for (int r = 0; r < 4; ++r) {
     const int n = lb.t * kTileRows + 4 * lb.l + r;
+    if (n >= N) break;
     for (int j = 0; j < 16; ++j) {
+      if (lb.b * 16 + j >= G) break;
       const size_t f = (size_t)n * G + (size_t)lb.b * 16 + j;
       signs[f] = s[j][r];
       idx[f] = (uint16_t)(p[j][r] & imask);
@@ -177,21 +183,24 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, int N, int K,
                                const uint16_t* __restrict__ codebook,
                                const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
                                const uint16_t* __restrict__ lut, int out_bf16, uint16_t* __restrict__ out) {
+  const int Np = pad_rows(N), Kp = pad_cols(K), G = K / 8;
   const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= num_lane_blocks(N, K)) return;
-  const LaneBlockId lb = lane_block_id(N, K, id);
+  if (id >= num_lane_blocks(Np, Kp)) return;
+  const LaneBlockId lb = lane_block_id(Np, Kp, id);
   if (!lb.valid) return;
   uint32_t w[kWords];
-  load_words(packed, N, K, lb, w);
+  load_words(packed, Np, Kp, lb, w);
   uint8_t s[16][4];
   uint32_t p[16][4];
   split_words(w, s, p);
   const uint32_t imask = (1u << b_d) - 1u;
   for (int r = 0; r < 4; ++r) {
     const int n = lb.t * kTileRows + 4 * lb.l + r;
+    if (n >= N) break;
     const float sc = lut ? 0.f : __half2float(__ushort_as_half(scale[n]));
     const float of = lut ? 0.f : __half2float(__ushort_as_half(offset[n]));
     for (int j = 0; j < 16; ++j) {
+      if (lb.b * 16 + j >= G) break;
       const uint32_t id_ = p[j][r] & imask;
       const uint32_t cd = p[j][r] >> b_d;
       // the quantized radius: per-row table level, or the affine form
@@ -223,14 +232,14 @@ inline unsigned grid_for(long long work, int threads) {
 }  // namespace
 
 cudaError_t launch_repack(const uint8_t* canon, int N, int K, int b_d, void* out, cudaStream_t st) {
-  const long long work = (long long)(N / kRowsPerLane) * (K / kBlockCols);
+  const long long work = (long long)(pad_rows(N) / kRowsPerLane) * (pad_cols(K) / kBlockCols);
   repack_kernel<<<grid_for(work, 128), 128, 0, st>>>(canon, N, K, b_d, (uint8_t*)out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpack(const void* packed, int N, int K, int b_d, uint8_t* signs, uint16_t* idx,
                           uint16_t* code, cudaStream_t st) {
-  const long long work = (long long)(N / kRowsPerLane) * (K / kBlockCols);
+  const long long work = (long long)(pad_rows(N) / kRowsPerLane) * (pad_cols(K) / kBlockCols);
   unpack_kernel<<<grid_for(work, 128), 128, 0, st>>>((const uint8_t*)packed, N, K, b_d, signs, idx, code);
   return cudaGetLastError();
 }
@@ -238,7 +247,7 @@ cudaError_t launch_unpack(const void* packed, int N, int K, int b_d, uint8_t* si
 cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
                            const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
                            uint16_t* out, cudaStream_t st) {
-  const long long work = (long long)(N / kRowsPerLane) * (K / kBlockCols);
+  const long long work = (long long)(pad_rows(N) / kRowsPerLane) * (pad_cols(K) / kBlockCols);
   dequant_kernel<<<grid_for(work, 128), 128, 0, st>>>((const uint8_t*)packed, N, K, b_d, codebook, scale,
                                                       offset, lut, out_bf16, out);
   return cudaGetLastError();

@@ -22,9 +22,11 @@
  *     runs asynchronously; the return value reports argument validation and
  *     launch errors only.
  *   - fp16 / bf16 values are passed as 16-bit bit patterns (uint16_t).
- *   - Shapes: K % 8 == 0 is the format's own rule.  The device layout and all
- *     kernels additionally need K % 128 == 0 and N % 4 == 0; other shapes return
- *     SVQ_ERR_UNSUPPORTED_SHAPE.  1 <= b_d <= 10.
+ *   - Shapes: K % 8 == 0 (the format's own rule), N >= 1, 1 <= b_d <= 10.
+ *     Shapes with N % 4 != 0 or K % 128 != 0 are stored padded to the next
+ *     multiple of 4 rows and 128 columns (zero codes, svq_packed_bytes counts
+ *     them); the padding never contributes to an output.  svq_moe_grouped_gemv
+ *     takes only K % 128 == 0 and N % 4 == 0.
  *   - Return codes: SVQ_OK or one of the SVQ_ERR_* values below; nothing is
  *     enqueued when an error is returned.
  */
@@ -89,8 +91,9 @@ SVQ_API const char* svq_status_string(int status);
 SVQ_API int svq_version(void);
 
 /* Bytes of the device layout of an N x K matrix: exactly N * K * 9 / 32 (18 bits
- * per 8 weights, Figure 2 caption), the same size as the canonical stream.
- * Returns 0 for shapes the layout does not support. */
+ * per 8 weights, Figure 2 caption), the same size as the canonical stream, for
+ * N % 4 == 0 and K % 128 == 0; otherwise Np * Kp * 9 / 32 with N and K rounded
+ * up to multiples of 4 and 128 (padding).  Returns 0 when K % 8 != 0. */
 SVQ_API size_t svq_packed_bytes(int N, int K);
 
 /* Bytes of the canonical stream: N * ceil(18 * (K/8) / 8). */

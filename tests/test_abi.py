@@ -25,8 +25,9 @@ def test_pure_host_queries():
     assert svq.lib().svq_version() >= 100
     assert svq.svq_packed_bytes(1024, 1024) == 1024 * 1024 * 9 // 32
     assert svq.svq_packed_bytes(2560, 9728) == 2560 * 9728 * 9 // 32
-    assert svq.svq_packed_bytes(1024, 1000) == 0          # K % 128 != 0: no device layout
-    assert svq.svq_packed_bytes(6, 128) == 0              # N % 4 != 0
+    assert svq.svq_packed_bytes(1024, 1000) == 1024 * 1024 * 9 // 32   # K padded to 1024 columns
+    assert svq.svq_packed_bytes(6, 128) == 8 * 128 * 9 // 32            # N padded to 8 rows
+    assert svq.svq_packed_bytes(1024, 1004) == 0          # K % 8 != 0: not an SVQ shape
     assert svq.svq_canonical_bytes(3, 40) == 3 * 12       # 5 codes * 18 bits = 90 bits -> 12 bytes
     for s in range(6):
         assert svq.status_string(s)
@@ -43,7 +44,7 @@ def test_validation_without_gpu():
     assert L.svq_repack(dummy, 128, 128, 0, dummy, nullp) == svq.SVQ_ERR_UNSUPPORTED_SHAPE
     assert L.svq_repack(dummy, 128, 128, 8, ctypes.c_void_p(0x1008), nullp) == svq.SVQ_ERR_INVALID_ARG
     m = svq.svq_matrix(128, 128, 8, 0, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
-    bad = svq.svq_matrix(128, 136, 8, 0, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+    bad = svq.svq_matrix(128, 132, 8, 0, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000)      # K % 8 != 0
     n = ctypes.c_size_t(0)
     assert L.svq_linear_gemv_workspace_size(ctypes.byref(bad), 1, ctypes.byref(n)) == svq.SVQ_ERR_UNSUPPORTED_SHAPE
     assert L.svq_linear_gemv_workspace_size(ctypes.byref(m), 0, ctypes.byref(n)) == svq.SVQ_ERR_INVALID_ARG
