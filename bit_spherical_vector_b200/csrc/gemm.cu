@@ -23,8 +23,12 @@
 //                   shared-memory replicas; the sixteen warps share every
 //                   stage (one of its eight subvector groups, half the rows)
 //       warps 18..21 epilogue: tcgen05.ld -> registers -> shared staging ->
-//                   coalesced stores of y (or of split-K partials)
-//   * pass 3 (split K only): y = sum of the partials in slice order.
+//                   coalesced stores of y (or of the fp32 partials of a
+//                   k-slice of a split tile)
+//   * pass 3 (split tiles only): y = sum of the slices' partials in slice order.
+//     Whole tiles fill complete rounds of the grid; the tiles of a last,
+//     partial round (or, where that estimates faster, every tile) are split
+//     along K so that their slices spread over all SMs.
 //   * weights are the A operand (swap-AB), so small token counts still map to
 //     the 128-row MMA; work units are (token tile, k-split, row tile).
 // Weight rows are placed in the A tile in the order rho = lane + 32 * r (lane
@@ -40,6 +44,7 @@
 #include <atomic>
 #include <cmath>
 
+#include "gemm_common.cuh"
 #include "gemm_params.h"
 #include "layout.cuh"
 #include "sm100.cuh"
@@ -49,6 +54,7 @@ namespace svq {
 namespace {
 
 using namespace sm100;
+using namespace gemm;
 
 constexpr int kDecWarp0 = 2, kNumDec = 16;
 constexpr int kEpiWarp0 = kDecWarp0 + kNumDec, kNumEpi = 4;
@@ -79,48 +85,6 @@ struct Bars {
   int abort_flag;
   int epi_ok;
 };
-
-__device__ __forceinline__ void record_timeout(const GemmKParams& p, Bars* bars) {
-  atomicExch(p.status, 5 /* SVQ_ERR_TIMEOUT */);
-  atomicExch(&bars->abort_flag, 1);
-}
-
-// Wait that gives up on timeout or when another role has aborted.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const GemmKParams& p, Bars* bars) {
-  for (uint32_t i = 0; i < p.wait_polls; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 63 && *(volatile int*)&bars->abort_flag) return false;
-  }
-  record_timeout(p, bars);
-  return false;
-}
-
-struct Unit {
-  int nt, mt, s, kb0, kb1;
-};
-
-__device__ __forceinline__ Unit unit_of(const GemmKParams& p, int u) {
-  Unit w;
-  w.nt = u % p.n_tiles;
-  const int rest = u / p.n_tiles;
-  w.s = rest % p.S;
-  w.mt = rest / p.S;
-  const int KB = pad_cols(p.K) / 64;                  // 64-column blocks of the (padded) layout
-  w.kb0 = (int)(((long long)KB * w.s) / p.S);
-  w.kb1 = (int)(((long long)KB * (w.s + 1)) / p.S);
-  return w;
-}
-
-template <bool BF16>
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  uint32_t r;
-  if constexpr (BF16) {
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  } else {
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  }
-  return r;
-}
 
 // Decode decoder warp dw's share of one 64-column stage of one 128-row tile
 // into the swizzled A tile: subvector group j = 8 * (kb & 1) + dw % 8 of the
@@ -274,7 +238,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const int n_units = p.n_tiles * p.m_tiles * p.S;
+  const int n_units = p.F + p.rem * p.S;
 
   if (warp == 0) {
     // ---------------- TMA producer: activation tiles into the A/B ring (slot
@@ -428,7 +392,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
       tc_fence_after();
       const int n0 = w.nt * kTileRows;
       const int rows = min(kTileRows, p.N - n0);
-      const bool split = p.S > 1;
+      const bool split = w.slot >= 0;
+      float* part = split ? p.partial + (size_t)w.slot * BN * kTileRows : nullptr;
       for (int c0 = 0; c0 < BN; c0 += kStageCols) {
         uint32_t v[32];
         tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * BN + c0, v);
@@ -458,11 +423,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           };
           const float4 val = make_float4(pick(0), pick(1), pick(2), pick(3));
           const int n = n0 + 4 * lane;
-          const size_t o = (size_t)m * p.N + n;           // element of y (or of a partial slice)
-          if ((p.N & 3) == 0) {                           // rows of 4 stay 16-byte aligned
-            if (split) {
-              *reinterpret_cast<float4*>(p.partial + (size_t)w.s * p.part_stride + o) = val;
-            } else if (p.y_f32) {
+          const size_t o = (size_t)m * p.N + n;           // element of y
+          if (split) {                                    // [token][row] of the tile's slot
+            *reinterpret_cast<float4*>(part + (size_t)(c0 + i) * kTileRows + 4 * lane) = val;
+          } else if ((p.N & 3) == 0) {                    // rows of 4 stay 16-byte aligned
+            if (p.y_f32) {
               *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + o) = val;
             } else {
               uint2 pk;
@@ -473,8 +438,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           } else {                                        // ragged N: element by element, rows < N
             const float vv[4] = {val.x, val.y, val.z, val.w};
             for (int r = 0; r < 4 && n + r < p.N; ++r) {
-              if (split) p.partial[(size_t)w.s * p.part_stride + o + r] = vv[r];
-              else if (p.y_f32) reinterpret_cast<float*>(p.y)[o + r] = vv[r];
+              if (p.y_f32) reinterpret_cast<float*>(p.y)[o + r] = vv[r];
               else reinterpret_cast<uint16_t*>(p.y)[o + r] = __bfloat16_as_ushort(__float2bfloat16_rn(vv[r]));
             }
           }
@@ -515,35 +479,78 @@ __global__ void permute_kernel(const uint16_t* __restrict__ x, const int32_t* __
   *reinterpret_cast<uint4*>(xp + (size_t)m * K + j0) = o;
 }
 
-// Split-K reduction: y[m][n] = sum over slices s = 0..S-1 of partial[s][m][n]
-// (in slice order, so the result does not depend on scheduling), four outputs
-// per thread.  Separate from the GEMM so that all SMs share it.
-// Slices are stride (= MN rounded up to 4) elements apart, so every slice is
-// 16-byte aligned; a last group of fewer than 4 elements is stored one by one.
-__global__ void splitk_reduce_kernel(const float* __restrict__ partial, int S, long long MN, long long stride_el,
-                                     void* __restrict__ y, int y_f32) {
-  const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  for (long long i = q; i < (MN + 3) / 4; i += stride) {
-    float4 acc = __ldcs(reinterpret_cast<const float4*>(partial) + i);
-    for (int k = 1; k < S; ++k) {
-      const float4 t = __ldcs(reinterpret_cast<const float4*>(partial + (size_t)k * stride_el) + i);
-      acc.x += t.x; acc.y += t.y; acc.z += t.z; acc.w += t.w;
+// The same gather with the row staged in shared memory: each CTA takes rows
+// m = blockIdx.x, + gridDim.x, ..., loads a row with 16-byte loads into one of
+// two buffers (the other may still be read by slower threads: one barrier per
+// row suffices), then every thread gathers eight columns from shared memory and
+// stores 16 bytes.  x, perm 16-byte aligned; 2 K 16-bit values of shared memory.
+__global__ void __launch_bounds__(256)
+permute_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int M, int K,
+                    uint16_t* __restrict__ xp) {
+  extern __shared__ uint4 prow[];
+  const int K8 = K / 8;
+  int it = 0;
+  for (int m = blockIdx.x; m < M; m += gridDim.x, ++it) {
+    uint4* row = prow + (it & 1) * K8;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)m * K);
+    for (int c = threadIdx.x; c < K8; c += blockDim.x) row[c] = __ldcs(src + c);
+    __syncthreads();
+    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)m * K);
+    // indices clamped to the row: a malformed perm cannot read past the buffer
+    const uint32_t last = (uint32_t)K - 1u;
+    auto at = [&](int j) -> uint32_t { return r16[min((uint32_t)j, last)]; };
+    for (int c = threadIdx.x; c < K8; c += blockDim.x) {
+      const int4 p0 = __ldg(reinterpret_cast<const int4*>(perm) + 2 * c);
+      const int4 p1 = __ldg(reinterpret_cast<const int4*>(perm) + 2 * c + 1);
+      uint4 o;
+      o.x = at(p0.x) | (at(p0.y) << 16);
+      o.y = at(p0.z) | (at(p0.w) << 16);
+      o.z = at(p1.x) | (at(p1.y) << 16);
+      o.w = at(p1.z) | (at(p1.w) << 16);
+      dst[c] = o;
     }
-    if (4 * i + 4 <= MN) {
+  }
+}
+
+// Split-tile reduction: for each of the rem split tiles (tile F + i, rows
+// nt * RM.., tokens mt * BN..), y = the sum of its S slot values in slice
+// order (so the result does not depend on scheduling); slot s * rem + i holds
+// BN x RM fp32 values [token][row].  Four outputs per thread, rows past N and
+// tokens past M skipped, ragged N stored element by element.
+__global__ void split_reduce_kernel(const float* __restrict__ partial, int S, int F, int rem, int n_tiles, int BN,
+                                    int RM, int M, int N, void* __restrict__ y, int y_f32) {
+  const int R4 = RM / 4;
+  const long long total = (long long)rem * BN * R4;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const size_t slot_el = (size_t)BN * RM;
+  for (long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x; q < total; q += stride) {
+    const int i = (int)(q / ((long long)BN * R4));
+    const int ml = (int)((q / R4) % BN), q4 = (int)(q % R4);
+    const int t = F + i;
+    const int m = (t / n_tiles) * BN + ml, n = (t % n_tiles) * RM + 4 * q4;
+    if (m >= M || n >= N) continue;
+    const size_t e = (size_t)ml * RM + 4 * q4;
+    float4 acc = __ldcs(reinterpret_cast<const float4*>(partial + (size_t)i * slot_el + e));
+    for (int s = 1; s < S; ++s) {
+      const float4 v = __ldcs(reinterpret_cast<const float4*>(partial + ((size_t)s * rem + i) * slot_el + e));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    const size_t o = (size_t)m * N + n;
+    if ((N & 3) == 0) {
       if (y_f32) {
-        reinterpret_cast<float4*>(y)[i] = acc;
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + o) = acc;
       } else {
         uint2 pk;
         pk.x = pack2<true>(acc.x, acc.y);
         pk.y = pack2<true>(acc.z, acc.w);
-        reinterpret_cast<uint2*>(y)[i] = pk;
+        *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(y) + o) = pk;
       }
     } else {
       const float av[4] = {acc.x, acc.y, acc.z, acc.w};
-      for (long long e = 4 * i; e < MN; ++e) {
-        if (y_f32) reinterpret_cast<float*>(y)[e] = av[e - 4 * i];
-        else reinterpret_cast<uint16_t*>(y)[e] = __bfloat16_as_ushort(__float2bfloat16_rn(av[e - 4 * i]));
+      for (int r = 0; r < 4 && n + r < N; ++r) {
+        if (y_f32) reinterpret_cast<float*>(y)[o + r] = av[r];
+        else reinterpret_cast<uint16_t*>(y)[o + r] = __bfloat16_as_ushort(__float2bfloat16_rn(av[r]));
       }
     }
   }
@@ -602,35 +609,49 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   GemmPlan g{};
   g.BN = M >= 256 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : (M > 16 ? 32 : 16)));
   g.m_tiles = (M + g.BN - 1) / g.BN;
-  g.n_tiles = num_tiles(pad_rows(N));
+  // From two token tiles on, the matrix is decoded once into the workspace
+  // (N x K 16-bit values, the activations' type) and the kernel loads weight
+  // tiles by TMA instead of decoding every stage once per token tile; with one
+  // token tile the decode pass would only add its own cost.
+  g.dense = g.m_tiles >= 2 ? 1 : 0;
+  // Pre-decoded tiles of 256 rows (1.5x fewer L2 bytes per output) once they
+  // still fill every SM at least once; below that 128-row tiles keep more SMs busy.
+  const int nt256 = (pad_rows(N) + kDenseTileRows - 1) / kDenseTileRows;
+  g.RM = g.dense && (long long)nt256 * g.m_tiles >= num_sms ? kDenseTileRows : kTileRows;
+  g.n_tiles = g.RM == kTileRows ? num_tiles(pad_rows(N)) : nt256;
   const int T = g.n_tiles * g.m_tiles;
   const int KB = pad_cols(K) / 64;
-  // Split K when it shortens the estimated time: waves of units times the
-  // k-blocks per unit (about 1 us per 64-column k-block, set by the latency of
-  // the staging ring rather than by the MMA), plus the reduction pass over the
-  // S fp32 partials (S + 1) * M * N * 4 bytes at ~4 TB/s and one launch.
-  g.S = 1;
-  {
-    double best = 1e30;
-    for (int S = 1; S <= std::min(16, std::max(1, KB / 8)); ++S) {
-      const double waves = std::ceil((double)T * S / num_sms);
-      double est = waves * std::ceil((double)KB / S) * 1.0e-6;
-      if (S > 1) est += (double)(S + 1) * M * N * 4.0 / 4.0e12 + 3.0e-6;
-      if (est < best * 0.97) { best = est; g.S = S; }
+  // Work split, by the estimated time: whole tiles round-robin over the SMs
+  // (rounds of tiles times the k-blocks of a tile), optionally with every tile
+  // split into S k-slices (more, shorter units), or with only the tiles of the
+  // last, partial round split S ways so that they spread over all SMs.  A
+  // 64-column k-block takes about 1 us with on-chip decode and 0.6 us with
+  // pre-decoded tiles (set by the staging ring's latency, not the MMA); a split
+  // adds the reduction pass over its S + 1 fp32 copies of the split tiles
+  // (~4 TB/s) and one launch.
+  const double t_kb = g.RM == kDenseTileRows ? 0.9e-6 : (g.dense ? 0.6e-6 : 1.0e-6);
+  const double tile_bytes = (double)g.BN * g.RM * 4.0;
+  auto red = [&](int S, int tiles) { return (double)(S + 1) * tiles * tile_bytes / 4.0e12 + 3.0e-6; };
+  g.S = 1; g.F = T; g.rem = 0;
+  double best = std::ceil((double)T / num_sms) * KB * t_kb;
+  for (int S = 2; S <= std::min(16, std::max(1, KB / 8)); ++S) {
+    const double est = std::ceil((double)T * S / num_sms) * std::ceil((double)KB / S) * t_kb + red(S, T);
+    if (est < best * 0.97) { best = est; g.S = S; g.F = 0; g.rem = T; }
+  }
+  const int rem = T % num_sms;
+  if (T > num_sms && rem > 0) {
+    for (int S = 2; S <= std::min(num_sms / rem, std::max(1, KB / 4)); ++S) {
+      const double est = (double)(T / num_sms) * KB * t_kb + std::ceil((double)KB / S) * t_kb + red(S, rem);
+      if (est < best * 0.97) { best = est; g.S = S; g.F = T - rem; g.rem = rem; }
     }
   }
-  g.grid = std::min(T * g.S, num_sms);
-  // From four token tiles on, the matrix is decoded once into the workspace
-  // (N x K 16-bit values, the activations' type) and the kernel loads weight
-  // tiles by TMA instead of decoding every stage once per token tile; below
-  // that the decode pass costs more than the repeated on-chip decodes.
-  g.dense = g.m_tiles >= 4 ? 1 : 0;
+  g.grid = std::min(g.F + g.rem * g.S, num_sms);
   const size_t xp = ((size_t)M * K * 2 + 255) / 256 * 256;
   const size_t wdec = g.dense ? ((size_t)N * K * 2 + 255) / 256 * 256 : 0;
   g.xp_offset = 0;
   g.wdec_offset = xp;
   g.partial_offset = xp + wdec;
-  const size_t part = g.S > 1 ? ((size_t)g.S * (((size_t)M * N + 3) / 4 * 4) * 4 + 255) / 256 * 256 : 0;
+  const size_t part = g.rem > 0 ? (size_t)g.S * g.rem * (size_t)g.BN * g.RM * 4 : 0;
   g.ws_bytes = xp + wdec + part;
   return g;
 }
@@ -642,8 +663,22 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   const uint16_t* xp = d.x;
   if (d.perm) {
     uint16_t* xw = reinterpret_cast<uint16_t*>(wsb + g.xp_offset);
-    const long long work = (long long)d.M * (d.K / 8);
-    permute_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(d.x, d.perm, d.M, d.K, xw);
+    const size_t row_smem = (size_t)4 * d.K;           // two staged rows
+    const bool al16 = ((reinterpret_cast<uintptr_t>(d.x) | reinterpret_cast<uintptr_t>(d.perm)) & 15) == 0;
+    if (al16 && row_smem <= 96 * 1024) {
+      static std::atomic<bool> attr_set{false};
+      if (!attr_set.load(std::memory_order_acquire)) {
+        const cudaError_t ea = cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                    96 * 1024);
+        if (ea != cudaSuccess) return ea;
+        attr_set.store(true, std::memory_order_release);
+      }
+      const int ctas = std::max(1, std::min(d.M, 148 * 4));
+      permute_rows_kernel<<<ctas, 256, row_smem, st>>>(d.x, d.perm, d.M, d.K, xw);
+    } else {
+      const long long work = (long long)d.M * (d.K / 8);
+      permute_kernel<<<(unsigned)((work + 255) / 256), 256, 0, st>>>(d.x, d.perm, d.M, d.K, xw);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     xp = xw;
@@ -669,7 +704,7 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
                                    st);
     if (e != cudaSuccess) return e;
     const cuuint64_t wdims[2] = {(cuuint64_t)d.K, (cuuint64_t)d.N};
-    const cuuint32_t wbox[2] = {64, (cuuint32_t)kTileRows};
+    const cuuint32_t wbox[2] = {64, (cuuint32_t)g.RM};
     const CUresult rw = enc(&tw, d.x_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                             wdec, wdims, strides, wbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -683,21 +718,22 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.offset = d.offset;
   p.lut = d.lut;
   p.N = d.N; p.K = d.K; p.b_d = d.b_d; p.M = d.M;
-  p.n_tiles = g.n_tiles; p.m_tiles = g.m_tiles; p.S = g.S;
+  p.n_tiles = g.n_tiles; p.m_tiles = g.m_tiles; p.S = g.S; p.F = g.F; p.rem = g.rem;
   p.cb_replicas = d.b_d <= 8 ? 8 : (d.b_d == 9 ? 4 : 2);
   p.y = d.y;
   p.y_f32 = d.y_f32;
-  p.partial = g.S > 1 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
-  p.part_stride = ((long long)d.M * d.N + 3) / 4 * 4;
+  p.partial = g.rem > 0 ? reinterpret_cast<float*>(wsb + g.partial_offset) : nullptr;
   p.status = status;
   p.wait_polls = g_wait_polls.load(std::memory_order_relaxed);
   p.dense = g.dense;
-  cudaError_t e = d.x_bf16 ? launch_typed<true>(g.BN, tm, tw, p, g.grid, st)
-                           : launch_typed<false>(g.BN, tm, tw, p, g.grid, st);
-  if (e != cudaSuccess || g.S == 1) return e;
-  const long long mn = (long long)d.M * d.N;
-  const long long blocks = std::max<long long>(1, std::min<long long>(((mn + 3) / 4 + 255) / 256, 148LL * 8));
-  splitk_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.partial, g.S, mn, p.part_stride, d.y, d.y_f32);
+  cudaError_t e = g.RM == kDenseTileRows ? launch_gemm_dense256(tm, tw, p, g.grid, d.x_bf16, st)
+                  : d.x_bf16 ? launch_typed<true>(g.BN, tm, tw, p, g.grid, st)
+                             : launch_typed<false>(g.BN, tm, tw, p, g.grid, st);
+  if (e != cudaSuccess || g.rem == 0) return e;
+  const long long work = (long long)g.rem * g.BN * (g.RM / 4);
+  const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 148LL * 8));
+  split_reduce_kernel<<<(unsigned)blocks, 256, 0, st>>>(p.partial, g.S, g.F, g.rem, g.n_tiles, g.BN, g.RM, d.M, d.N,
+                                                        d.y, d.y_f32);
   return cudaGetLastError();
 }
 

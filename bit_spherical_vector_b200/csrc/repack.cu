@@ -1,12 +1,16 @@
 // repack.cu -- canonical stream -> device layout, its inverse (field export)
 // and the bit-exact dense dequantisation.
 //
-// One thread owns one lane-block (4 rows x 16 subvectors, 144 bytes); see
-// layout.cuh.  These kernels run once per matrix (repack) or in tests and
-// exports (unpack, dequantize), so they favour plainness over speed.
+// In repack and unpack one thread owns one lane-block (4 rows x 16 subvectors,
+// 144 bytes; see layout.cuh).  They run once per matrix (repack) or in tests
+// and exports (unpack), so they favour plainness over speed; dequantize is
+// organised per warp (below) since the GEMM runs it per call.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
 
 #include "layout.cuh"
 #include "svq_internal.h"
@@ -177,51 +181,123 @@ __global__ void unpack_kernel(const uint8_t* __restrict__ packed, int N, int K, 
   }
 }
 
-// Dense export, bit-exact: r = fmaf(scale, code, offset); w = RNE(r * c) in the
-// output format; sign bit set from the code afterwards.
-__global__ void dequant_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d,
-                               const uint16_t* __restrict__ codebook,
-                               const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
-                               const uint16_t* __restrict__ lut, int out_bf16, uint16_t* __restrict__ out) {
-  const int Np = pad_rows(N), Kp = pad_cols(K), G = K / 8;
-  const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= num_lane_blocks(Np, Kp)) return;
-  const LaneBlockId lb = lane_block_id(Np, Kp, id);
-  if (!lb.valid) return;
-  uint32_t w[kWords];
-  load_words(packed, Np, Kp, lb, w);
-  uint8_t s[16][4];
-  uint32_t p[16][4];
-  split_words(w, s, p);
+// Dense export, bit-exact: r = fmaf(scale, code, offset) (or the row's table
+// level); w = RNE(r * c) in the output format; sign bit set from the code
+// afterwards.  It also runs on every call of the GEMM's pre-decoded plan, so it
+// is written for bandwidth: one warp per (tile, block, row r of the lanes)
+// item, dealt round-robin over the CTAs; the 32 lanes load their lane-blocks
+// with coalesced 16-byte loads, decode row r of their four into a shared-memory
+// stage (rows of 16 x 16 bytes, the column XOR the row, so that both the
+// decoders' column writes and the row reads below are conflict free), and the
+// warp stores two 256-byte output rows per instruction.
+constexpr int kDqWarps = 8;
+constexpr int kDqStageU4 = 32 * 16;                 // 32 rows x 16 subvectors of 16 bytes per warp
+
+__device__ __forceinline__ uint32_t payload_of(const uint32_t w[kWords], int v) {
+  if (v < 60) return (w[16 + v / 3] >> (10 * (v % 3))) & 0x3FFu;
+  const int a = v - 60;
+  uint32_t pay = 0;
+#pragma unroll
+  for (int i = 0; i < 5; ++i) pay |= (w[16 + 5 * a + i] >> 30) << (8 - 2 * i);
+  return pay;
+}
+
+// One element pair: RNE(r * c) of both halves in the output format (binary32
+// products, then one conversion), then the two sign bits of pair t (bit 15 - t:
+// low element, bit 31 - t: high element).
+template <bool BF16>
+__device__ __forceinline__ uint32_t dq_pair(float2 rad2, uint32_t cw, uint32_t S, int t) {
+  const float2 pr = __fmul2_rn(rad2, __half22float2(*reinterpret_cast<const __half2*>(&cw)));
+  uint32_t bits;
+  if constexpr (BF16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(pr.x, pr.y);
+    bits = *reinterpret_cast<const uint32_t*>(&h);
+  } else {
+    const __half2 h = __floats2half2_rn(pr.x, pr.y);
+    bits = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  return bits ^ ((S << t) & 0x80008000u);
+}
+
+// Row R of the lane's four: its 16 subvectors into the lane's stage row.
+template <int R, bool BF16, bool LUT>
+__device__ __forceinline__ void dq_row(const uint32_t (&w)[kWords], float sc, float of, const uint16_t* lut_row,
+                                       int b_d, uint32_t imask, const uint4* cb, uint4* stg_row, int swz) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t pay = payload_of(w, 4 * j + R);
+    const uint32_t cd = pay >> b_d;
+    float rad;
+    if constexpr (LUT) rad = lut_row ? __half2float(__ushort_as_half(__ldg(lut_row + cd))) : 0.f;
+    else rad = __fmaf_rn(sc, (float)cd, of);
+    const float2 rad2 = make_float2(rad, rad);
+    const uint4 cw = cb[pay & imask];
+    const uint32_t S = w[j];
+    uint4 o;
+    o.x = dq_pair<BF16>(rad2, cw.x, S, 4 * R + 0);
+    o.y = dq_pair<BF16>(rad2, cw.y, S, 4 * R + 1);
+    o.z = dq_pair<BF16>(rad2, cw.z, S, 4 * R + 2);
+    o.w = dq_pair<BF16>(rad2, cw.w, S, 4 * R + 3);
+    stg_row[j ^ swz] = o;
+  }
+}
+
+template <bool BF16, bool LUT>
+__global__ void __launch_bounds__(kDqWarps * 32, 2)
+dequant_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d, const uint16_t* __restrict__ codebook,
+               const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
+               const uint16_t* __restrict__ lut, uint16_t* __restrict__ out) {
+  extern __shared__ uint4 dq_smem[];
+  const int ncw = 1 << b_d;
+  uint4* cb = dq_smem;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint4* stg = dq_smem + ncw + warp * kDqStageU4;
+  for (int i = threadIdx.x; i < ncw; i += blockDim.x) cb[i] = __ldg(reinterpret_cast<const uint4*>(codebook) + i);
+  __syncthreads();
+  const int Np = pad_rows(N), Kp = pad_cols(K), G = K / 8, B = Kp / kBlockCols;
+  const long long items = (long long)num_tiles(Np) * B * 4;
   const uint32_t imask = (1u << b_d) - 1u;
-  for (int r = 0; r < 4; ++r) {
-    const int n = lb.t * kTileRows + 4 * lb.l + r;
-    if (n >= N) break;
-    const float sc = lut ? 0.f : __half2float(__ushort_as_half(scale[n]));
-    const float of = lut ? 0.f : __half2float(__ushort_as_half(offset[n]));
-    for (int j = 0; j < 16; ++j) {
-      if (lb.b * 16 + j >= G) break;
-      const uint32_t id_ = p[j][r] & imask;
-      const uint32_t cd = p[j][r] >> b_d;
-      // the quantized radius: per-row table level, or the affine form
-      const float rad = lut ? __half2float(__ushort_as_half(lut[((size_t)n << (10 - b_d)) + cd]))
-                            : __fmaf_rn(sc, (float)cd, of);
-      uint16_t vals[8];
-      for (int i = 0; i < 8; ++i) {
-        const float c = __half2float(__ushort_as_half(codebook[id_ * 8 + i]));
-        const float prod = __fmul_rn(rad, c);
-        uint16_t bits = out_bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(prod))
-                                 : __half_as_ushort(__float2half_rn(prod));
-        if ((s[j][r] >> i) & 1u) bits ^= 0x8000u;
-        vals[i] = bits;
-      }
-      uint4 v;
-      v.x = vals[0] | ((uint32_t)vals[1] << 16);
-      v.y = vals[2] | ((uint32_t)vals[3] << 16);
-      v.z = vals[4] | ((uint32_t)vals[5] << 16);
-      v.w = vals[6] | ((uint32_t)vals[7] << 16);
-      *reinterpret_cast<uint4*>(out + (size_t)n * K + (size_t)lb.b * kBlockCols + 8 * j) = v;
+  const int lut_shift = 10 - b_d;
+  for (long long it = blockIdx.x + (long long)warp * gridDim.x; it < items; it += (long long)gridDim.x * kDqWarps) {
+    const int r = (int)(it & 3);
+    const long long tb = it >> 2;
+    const int t = (int)(tb / B), b = (int)(tb % B);
+    const int L = tile_lanes(Np, t);
+    uint32_t w[kWords];
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (lane < L) v = __ldg(reinterpret_cast<const uint4*>(packed + chunk_offset(Np, Kp, t, b, c, lane)));
+      w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
     }
+    const int n = t * kTileRows + 4 * lane + r;
+    const bool row_ok = lane < L && n < N;
+    float sc = 0.f, of = 0.f;
+    if (!LUT && row_ok) {
+      sc = __half2float(__ushort_as_half(__ldg(scale + n)));
+      of = __half2float(__ushort_as_half(__ldg(offset + n)));
+    }
+    // rows past N (padding, never stored) read no table: a zero radius
+    const uint16_t* lut_row = LUT && row_ok ? lut + ((size_t)n << lut_shift) : nullptr;
+    uint4* srow = stg + lane * 16;
+    const int swz = lane & 15;
+    switch (r) {
+      case 0: dq_row<0, BF16, LUT>(w, sc, of, lut_row, b_d, imask, cb, srow, swz); break;
+      case 1: dq_row<1, BF16, LUT>(w, sc, of, lut_row, b_d, imask, cb, srow, swz); break;
+      case 2: dq_row<2, BF16, LUT>(w, sc, of, lut_row, b_d, imask, cb, srow, swz); break;
+      default: dq_row<3, BF16, LUT>(w, sc, of, lut_row, b_d, imask, cb, srow, swz); break;
+    }
+    __syncwarp();
+    // rows of lanes 2i and 2i + 1 (output rows 4 lane + r), 16 subvectors each
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+      const int rl = 2 * i + (lane >> 4), col = lane & 15;
+      const int nrow = t * kTileRows + 4 * rl + r;
+      const int g = b * 16 + col;
+      if (rl < L && nrow < N && g < G)
+        *reinterpret_cast<uint4*>(out + (size_t)nrow * K + (size_t)g * 8) = stg[rl * 16 + (col ^ (rl & 15))];
+    }
+    __syncwarp();
   }
 }
 
@@ -244,13 +320,40 @@ cudaError_t launch_unpack(const void* packed, int N, int K, int b_d, uint8_t* si
   return cudaGetLastError();
 }
 
+namespace {
+
+template <bool BF16, bool LUT>
+cudaError_t launch_dequant_t(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
+                             const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, uint16_t* out,
+                             cudaStream_t st) {
+  const size_t smem = ((size_t)(1 << b_d) + (size_t)kDqWarps * kDqStageU4) * 16;
+  static std::atomic<bool> attr_set{false};
+  if (!attr_set.load(std::memory_order_acquire)) {
+    // the largest codebook (b_d = 10) sets the bound for every launch
+    const cudaError_t e = cudaFuncSetAttribute(dequant_kernel<BF16, LUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(((size_t)1024 + (size_t)kDqWarps * kDqStageU4) * 16));
+    if (e != cudaSuccess) return e;
+    attr_set.store(true, std::memory_order_release);
+  }
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long items = (long long)num_tiles(pad_rows(N)) * (pad_cols(K) / kBlockCols) * 4;
+  const long long ctas = std::min<long long>((items + kDqWarps - 1) / kDqWarps, 2LL * sms);
+  dequant_kernel<BF16, LUT><<<(unsigned)std::max<long long>(1, ctas), kDqWarps * 32, smem, st>>>(
+      (const uint8_t*)packed, N, K, b_d, codebook, scale, offset, lut, out);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
                            const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
                            uint16_t* out, cudaStream_t st) {
-  const long long work = (long long)(pad_rows(N) / kRowsPerLane) * (pad_cols(K) / kBlockCols);
-  dequant_kernel<<<grid_for(work, 128), 128, 0, st>>>((const uint8_t*)packed, N, K, b_d, codebook, scale,
-                                                      offset, lut, out_bf16, out);
-  return cudaGetLastError();
+  if (out_bf16)
+    return lut ? launch_dequant_t<true, true>(packed, N, K, b_d, codebook, scale, offset, lut, out, st)
+               : launch_dequant_t<true, false>(packed, N, K, b_d, codebook, scale, offset, lut, out, st);
+  return lut ? launch_dequant_t<false, true>(packed, N, K, b_d, codebook, scale, offset, lut, out, st)
+             : launch_dequant_t<false, false>(packed, N, K, b_d, codebook, scale, offset, lut, out, st);
 }
 
 }  // namespace svq

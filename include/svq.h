@@ -225,11 +225,13 @@ SVQ_API int svq_linear_gemv_noalloc(const svq_matrix* W /* host */, const uint16
  * Tensor Memory Accelerator (TMA) reads it directly).  y: [M][N] of y_dtype SVQ_F32
  * or SVQ_BF16.
  * Workspace (svq_linear_gemm_workspace_size): the permuted activations
- * x[:, perm] (unused when perm is NULL); from 4 tiles of 256 tokens on
- * (M > 768) the matrix decoded once (N x K values of x_dtype, the weights
+ * x[:, perm] (unused when perm is NULL); from 2 tiles of 256 tokens on
+ * (M > 256) the matrix decoded once (N x K values of x_dtype, the weights
  * svq_dequantize exports), which the tensor cores then read in place of
- * decoding every weight tile once per token tile; and, when K is split across
- * CTAs, the fp32 partial sums (summed by a second kernel in split order).  It
+ * decoding every weight tile once per token tile; and, when tiles are split
+ * along K across CTAs (the tiles of a last, partial round over the SMs, or all
+ * of them), the fp32 partial sums of those tiles (summed by a second kernel in
+ * slice order).  It
  * carries no state between calls and needs no initialisation.  Error bound used by the tests:
  * |y - y_ref| <= 1e-2 * sum_j |W[n][j]||x[m][perm[j]]|.
  */

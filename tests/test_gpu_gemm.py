@@ -123,7 +123,7 @@ def test_gemm_metamorphic_permutation():
 
 @pytest.mark.parametrize("x_dtype", ["bf16", "f16"])
 def test_gemm_pre_decoded_plan_matches_decoded_tiles(x_dtype):
-    """Four or more 256-token tiles switch the GEMM to weights decoded once into the workspace and
+    """Two or more 256-token tiles switch the GEMM to weights decoded once into the workspace and
     loaded by TMA; one tile decodes on chip.  Both place the same 16-bit weights in the MMA (the export
     reading), so the first 256 tokens of a 1100-token call equal a 256-token call bit for bit (K = 512:
     no K split in either plan), and every output is within the bound of the oracle.  N = 1028 ends in a
@@ -138,3 +138,33 @@ def test_gemm_pre_decoded_plan_matches_decoded_tiles(x_dtype):
     assert torch.equal(yb[:256], y256)
     y_ref, den = oracle.linear(m, x, x_dtype)
     assert rel_err(yb.cpu().numpy(), y_ref, den) <= TOL
+
+
+@pytest.mark.parametrize("N,K,M,kind,y_dtype", [
+    (4100, 4096, 1300, "bf16", torch.float32),    # pre-decoded tiles: 33 x 6 = 198 tiles, the last 50 split
+    (4100, 4096, 1300, "f16", torch.bfloat16),
+    (20478, 2048, 128, "bf16", torch.float32),    # on-chip decode, one token tile: 160 row tiles, the last 12 split
+    (4100, 1024, 2300, "bf16", torch.float32),    # pre-decoded 256-row tiles: 17 x 9 = 153 tiles, the last 5 split
+    (4100, 1024, 2300, "f16", torch.bfloat16),
+])
+def test_gemm_split_last_round(N, K, M, kind, y_dtype):
+    """On a 148-SM part these shapes have more tiles than SMs and a last, partial round; its tiles are
+    split along K into slices that spread over all SMs, and a second kernel sums their fp32 partials in
+    slice order (ragged N: the last row tile holds 4 or 126 rows).  The 2300-token shape runs the
+    pre-decoded kernel with 256-row tiles.  Checked on token rows that fall in split tiles and in whole
+    tiles, every output row n."""
+    need_gpu()
+    m = synth.make_matrix(77, N + M, N, K, 8)
+    x = synth.make_x(77, N + M, M, K, dtype=kind)
+    W = svq.SvqWeight.from_synth(m)
+    y, _, _ = _gemm(W, x, kind=kind, y_dtype=y_dtype)
+    rng = np.random.default_rng(N + M)
+    if M > 256:
+        lo = M - 256 - M % 256                      # the last two token tiles hold the split tiles
+        rows = np.concatenate([rng.choice(np.arange(lo, M), 12, replace=False),
+                               rng.choice(lo, 8, replace=False)])
+    else:
+        rows = rng.choice(M, 16, replace=False)
+    y_ref, den = oracle.linear(m, np.ascontiguousarray(x[rows]), kind)
+    tol = TOL + (2.0 ** -8 if y_dtype == torch.bfloat16 else 0.0)
+    assert rel_err(y.float().cpu().numpy()[rows], y_ref, den) <= tol
