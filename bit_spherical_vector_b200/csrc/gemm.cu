@@ -259,6 +259,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
           if (c.u < n_units) { c.w = unit_of(p, c.u); c.kb = c.w.kb0; }
         }
       };
+      // X_p (and the decoded weights) come from the grids launched before this
+      // one in the same call (programmatic dependent launch): wait for them
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       Cursor cb_, cp_;
       start(cb_);
       start(cp_);
@@ -462,6 +465,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
 // X_p[m][j] = X[m][perm[j]] (16-bit values), eight columns per thread.
 __global__ void permute_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int M, int K,
                                uint16_t* __restrict__ xp) {
+  // the next grid of the call (dequantisation or GEMM) may start beside this one
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long per_row = K / 8;
   if (i >= (long long)M * per_row) return;
@@ -488,6 +493,7 @@ __global__ void __launch_bounds__(256)
 permute_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int M, int K,
                     uint16_t* __restrict__ xp) {
   extern __shared__ uint4 prow[];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int K8 = K / 8;
   int it = 0;
   for (int m = blockIdx.x; m < M; m += gridDim.x, ++it) {
@@ -557,26 +563,39 @@ __global__ void split_reduce_kernel(const float* __restrict__ partial, int S, in
 }
 
 template <int BN, int NS, bool BF16, bool DENSE = false>
-cudaError_t launch_bn(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_bn(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid, bool pdl,
+                      cudaStream_t st) {
   constexpr uint32_t smem = smem_bytes<BN, NS, DENSE>();
   static_assert(smem <= 227 * 1024, "shared memory");
   cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN, NS, BF16, DENSE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gemm_kernel<BN, NS, BF16, DENSE><<<grid, kThreads, smem, st>>>(tm, tw, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_kernel<BN, NS, BF16, DENSE>, tm, tw, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <bool BF16>
 cudaError_t launch_typed(int BN, const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid,
-                         cudaStream_t st) {
+                         bool pdl, cudaStream_t st) {
   switch (BN) {
-    case 16: return launch_bn<16, 6, BF16>(tm, tw, p, grid, st);
-    case 32: return launch_bn<32, 6, BF16>(tm, tw, p, grid, st);
-    case 64: return launch_bn<64, 5, BF16>(tm, tw, p, grid, st);
-    case 128: return launch_bn<128, 4, BF16>(tm, tw, p, grid, st);
+    case 16: return launch_bn<16, 6, BF16>(tm, tw, p, grid, pdl, st);
+    case 32: return launch_bn<32, 6, BF16>(tm, tw, p, grid, pdl, st);
+    case 64: return launch_bn<64, 5, BF16>(tm, tw, p, grid, pdl, st);
+    case 128: return launch_bn<128, 4, BF16>(tm, tw, p, grid, pdl, st);
     default:
-      return p.dense ? launch_bn<256, 4, BF16, true>(tm, tw, p, grid, st) : launch_bn<256, 3, BF16>(tm, tw, p, grid, st);
+      return p.dense ? launch_bn<256, 4, BF16, true>(tm, tw, p, grid, pdl, st)
+                     : launch_bn<256, 3, BF16>(tm, tw, p, grid, pdl, st);
   }
 }
 
@@ -700,8 +719,11 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   CUtensorMap tw = tm;
   if (g.dense) {
     uint16_t* wdec = reinterpret_cast<uint16_t*>(wsb + g.wdec_offset);
-    cudaError_t e = launch_dequant(d.packed, d.N, d.K, d.b_d, d.codebook, d.scale, d.offset, d.lut, d.x_bf16, wdec,
-                                   st);
+    // after the permute it runs beside it (programmatic dependent launch)
+    cudaError_t e = d.perm ? launch_dequant_chained(d.packed, d.N, d.K, d.b_d, d.codebook, d.scale, d.offset, d.lut,
+                                                    d.x_bf16, wdec, st)
+                           : launch_dequant(d.packed, d.N, d.K, d.b_d, d.codebook, d.scale, d.offset, d.lut,
+                                            d.x_bf16, wdec, st);
     if (e != cudaSuccess) return e;
     const cuuint64_t wdims[2] = {(cuuint64_t)d.K, (cuuint64_t)d.N};
     const cuuint32_t wbox[2] = {64, (cuuint32_t)g.RM};
@@ -726,9 +748,12 @@ cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* 
   p.status = status;
   p.wait_polls = g_wait_polls.load(std::memory_order_relaxed);
   p.dense = g.dense;
-  cudaError_t e = g.RM == kDenseTileRows ? launch_gemm_dense256(tm, tw, p, g.grid, d.x_bf16, st)
-                  : d.x_bf16 ? launch_typed<true>(g.BN, tm, tw, p, g.grid, st)
-                             : launch_typed<false>(g.BN, tm, tw, p, g.grid, st);
+  // A grid of this call precedes the GEMM (permute and/or dequantisation): let
+  // the GEMM's prologue start beside it; its producer waits before reading.
+  const bool pdl = d.perm != nullptr || g.dense;
+  cudaError_t e = g.RM == kDenseTileRows ? launch_gemm_dense256(tm, tw, p, g.grid, d.x_bf16, pdl, st)
+                  : d.x_bf16 ? launch_typed<true>(g.BN, tm, tw, p, g.grid, pdl, st)
+                             : launch_typed<false>(g.BN, tm, tw, p, g.grid, pdl, st);
   if (e != cudaSuccess || g.rem == 0) return e;
   const long long work = (long long)g.rem * g.BN * (g.RM / 4);
   const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 148LL * 8));

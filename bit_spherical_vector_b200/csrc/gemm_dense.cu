@@ -93,6 +93,9 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
   if (warp == 0) {
     // ---------------- TMA producer
     if (lane == 0) {
+      // the decoded weights and X_p come from the grids launched before this one
+      // in the same call (programmatic dependent launch): wait for them
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       int it = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -199,20 +202,31 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
 }
 
 template <bool BF16>
-cudaError_t launch_dense(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid,
+cudaError_t launch_dense(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid, bool pdl,
                          cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(gemm_dense_kernel<BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  gemm_dense_kernel<BF16><<<grid, kThreads, kSmemBytes, st>>>(tm, tw, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_dense_kernel<BF16>, tm, tw, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_dense256(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid,
-                                 int x_bf16, cudaStream_t st) {
-  return x_bf16 ? launch_dense<true>(tm, tw, p, grid, st) : launch_dense<false>(tm, tw, p, grid, st);
+                                 int x_bf16, bool pdl, cudaStream_t st) {
+  return x_bf16 ? launch_dense<true>(tm, tw, p, grid, pdl, st) : launch_dense<false>(tm, tw, p, grid, pdl, st);
 }
 
 }  // namespace svq

@@ -58,9 +58,15 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms);
 // to make a wait give up at once); returns the previous value.
 uint32_t set_wait_polls(uint32_t polls);
 cudaError_t launch_gemm(const GemmMatDesc& d, const GemmPlan& g, void* ws, int* status, cudaStream_t st);
+// The dequantisation pass of the pre-decoded plan (repack.cu), launched as a
+// programmatic dependent of the activation permute before it: it runs beside
+// that grid and completes only after it.
+cudaError_t launch_dequant_chained(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
+                                   const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
+                                   uint16_t* out, cudaStream_t st);
 // The 256 x 256-tile kernel on pre-decoded weights (gemm_dense.cu); tm: 256-token
 // boxes of X_p, tw: 256-row boxes of the decoded weights, both 64 columns wide.
 cudaError_t launch_gemm_dense256(const CUtensorMap& tm, const CUtensorMap& tw, const GemmKParams& p, int grid,
-                                 int x_bf16, cudaStream_t st);
+                                 int x_bf16, bool pdl, cudaStream_t st);
 
 }  // namespace svq

@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "gemm_params.h"
 #include "layout.cuh"
 #include "svq_internal.h"
 
@@ -248,6 +249,10 @@ dequant_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d, const 
                const uint16_t* __restrict__ scale, const uint16_t* __restrict__ offset,
                const uint16_t* __restrict__ lut, uint16_t* __restrict__ out) {
   extern __shared__ uint4 dq_smem[];
+  // In the GEMM's pre-decoded plan this grid follows the activation permute as
+  // a programmatic dependent launch and runs beside it (it reads only weights);
+  // the GEMM after it may likewise start its prologue early.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int ncw = 1 << b_d;
   uint4* cb = dq_smem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -299,6 +304,9 @@ dequant_kernel(const uint8_t* __restrict__ packed, int N, int K, int b_d, const 
     }
     __syncwarp();
   }
+  // Complete only after the grid this one overlapped (the permute): a kernel
+  // that waits for this grid then sees both outputs.  No-op in a plain launch.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 inline unsigned grid_for(long long work, int threads) {
@@ -325,7 +333,7 @@ namespace {
 template <bool BF16, bool LUT>
 cudaError_t launch_dequant_t(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
                              const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, uint16_t* out,
-                             cudaStream_t st) {
+                             bool pdl, cudaStream_t st) {
   const size_t smem = ((size_t)(1 << b_d) + (size_t)kDqWarps * kDqStageU4) * 16;
   static std::atomic<bool> attr_set{false};
   if (!attr_set.load(std::memory_order_acquire)) {
@@ -339,9 +347,34 @@ cudaError_t launch_dequant_t(const void* packed, int N, int K, int b_d, const ui
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = (long long)num_tiles(pad_rows(N)) * (pad_cols(K) / kBlockCols) * 4;
   const long long ctas = std::min<long long>((items + kDqWarps - 1) / kDqWarps, 2LL * sms);
-  dequant_kernel<BF16, LUT><<<(unsigned)std::max<long long>(1, ctas), kDqWarps * 32, smem, st>>>(
-      (const uint8_t*)packed, N, K, b_d, codebook, scale, offset, lut, out);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::max<long long>(1, ctas));
+  cfg.blockDim = dim3(kDqWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, dequant_kernel<BF16, LUT>, (const uint8_t*)packed, N, K, b_d,
+                                           codebook, scale, offset, lut, out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+namespace {
+
+cudaError_t dequant_dispatch(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
+                             const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
+                             uint16_t* out, cudaStream_t st, bool pdl) {
+  if (out_bf16)
+    return lut ? launch_dequant_t<true, true>(packed, N, K, b_d, codebook, scale, offset, lut, out, pdl, st)
+               : launch_dequant_t<true, false>(packed, N, K, b_d, codebook, scale, offset, lut, out, pdl, st);
+  return lut ? launch_dequant_t<false, true>(packed, N, K, b_d, codebook, scale, offset, lut, out, pdl, st)
+             : launch_dequant_t<false, false>(packed, N, K, b_d, codebook, scale, offset, lut, out, pdl, st);
 }
 
 }  // namespace
@@ -349,11 +382,13 @@ cudaError_t launch_dequant_t(const void* packed, int N, int K, int b_d, const ui
 cudaError_t launch_dequant(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
                            const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
                            uint16_t* out, cudaStream_t st) {
-  if (out_bf16)
-    return lut ? launch_dequant_t<true, true>(packed, N, K, b_d, codebook, scale, offset, lut, out, st)
-               : launch_dequant_t<true, false>(packed, N, K, b_d, codebook, scale, offset, lut, out, st);
-  return lut ? launch_dequant_t<false, true>(packed, N, K, b_d, codebook, scale, offset, lut, out, st)
-             : launch_dequant_t<false, false>(packed, N, K, b_d, codebook, scale, offset, lut, out, st);
+  return dequant_dispatch(packed, N, K, b_d, codebook, scale, offset, lut, out_bf16, out, st, false);
+}
+
+cudaError_t launch_dequant_chained(const void* packed, int N, int K, int b_d, const uint16_t* codebook,
+                                   const uint16_t* scale, const uint16_t* offset, const uint16_t* lut, int out_bf16,
+                                   uint16_t* out, cudaStream_t st) {
+  return dequant_dispatch(packed, N, K, b_d, codebook, scale, offset, lut, out_bf16, out, st, true);
 }
 
 }  // namespace svq
