@@ -485,26 +485,35 @@ __global__ void permute_kernel(const uint16_t* __restrict__ x, const int32_t* __
 }
 
 // The same gather with the row staged in shared memory: each CTA takes rows
-// m = blockIdx.x, + gridDim.x, ..., loads a row with 16-byte loads into one of
-// two buffers (the other may still be read by slower threads: one barrier per
-// row suffices), then every thread gathers eight columns from shared memory and
+// m = blockIdx.x, + gridDim.x, ...; row m is copied into one of two buffers by
+// asynchronous 16-byte copies (cp.async) issued while the previous row is being
+// gathered, then every thread gathers eight columns from shared memory and
 // stores 16 bytes.  x, perm 16-byte aligned; 2 K 16-bit values of shared memory.
+__device__ __forceinline__ void row_copy_async(uint4* dst, const uint4* src, int K8) {
+  for (int c = threadIdx.x; c < K8; c += blockDim.x)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_u32(dst + c)), "l"(src + c)
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(256)
 permute_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int M, int K,
                     uint16_t* __restrict__ xp) {
   extern __shared__ uint4 prow[];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int K8 = K / 8;
-  int it = 0;
-  for (int m = blockIdx.x; m < M; m += gridDim.x, ++it) {
-    uint4* row = prow + (it & 1) * K8;
-    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)m * K);
-    for (int c = threadIdx.x; c < K8; c += blockDim.x) row[c] = __ldcs(src + c);
+  const uint32_t last = (uint32_t)K - 1u;
+  int m = blockIdx.x;
+  if (m < M) row_copy_async(prow, reinterpret_cast<const uint4*>(x + (size_t)m * K), K8);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int it = 0; m < M; m += gridDim.x, ++it) {
+    const int mn = m + gridDim.x;
+    if (mn < M) row_copy_async(prow + ((it + 1) & 1) * K8, reinterpret_cast<const uint4*>(x + (size_t)mn * K), K8);
+    asm volatile("cp.async.commit_group;" ::: "memory");    // possibly empty: one group per row
+    asm volatile("cp.async.wait_group 1;" ::: "memory");    // this row's copies have landed
     __syncthreads();
-    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
+    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(prow + (it & 1) * K8);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)m * K);
     // indices clamped to the row: a malformed perm cannot read past the buffer
-    const uint32_t last = (uint32_t)K - 1u;
     auto at = [&](int j) -> uint32_t { return r16[min((uint32_t)j, last)]; };
     for (int c = threadIdx.x; c < K8; c += blockDim.x) {
       const int4 p0 = __ldg(reinterpret_cast<const int4*>(perm) + 2 * c);
@@ -516,7 +525,9 @@ permute_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ 
       o.w = at(p1.z) | (at(p1.w) << 16);
       dst[c] = o;
     }
+    __syncthreads();                                        // this buffer is refilled two rows on
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // Split-tile reduction: for each of the rem split tiles (tile F + i, rows
