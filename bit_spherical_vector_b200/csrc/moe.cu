@@ -59,8 +59,6 @@ __device__ __forceinline__ int moe_matrix_cost(int ni, int mt) {
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(MoeKParams p) {
   extern __shared__ int sh[];                   // [n_mats] counts, then scan scratch
   int* cnt = sh;
-  __shared__ int s_warp[kRouteThreads / 32];
-  __shared__ int s_total;
   for (int i = threadIdx.x; i < p.n_mats; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   for (int i = threadIdx.x; i < p.n_items; i += blockDim.x) {
@@ -112,9 +110,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(MoeKParams p) {
   if (threadIdx.x == 0) {
     p.offsets[p.n_mats] = base_items;
     *p.n_active = base_active;
-    s_total = base_items;
   }
-  (void)s_warp;
   __syncthreads();
   // Group item indices by matrix (order inside a matrix does not affect any
   // result: every item is computed on its own).
