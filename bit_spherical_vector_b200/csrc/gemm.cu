@@ -431,12 +431,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ 
             *reinterpret_cast<float4*>(part + (size_t)(c0 + i) * kTileRows + 4 * lane) = val;
           } else if ((p.N & 3) == 0) {                    // rows of 4 stay 16-byte aligned
             if (p.y_f32) {
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + o) = val;
+              __stcs(reinterpret_cast<float4*>(reinterpret_cast<float*>(p.y) + o), val);   // streaming: y is not re-read
             } else {
               uint2 pk;
               pk.x = pack2<true>(val.x, val.y);
               pk.y = pack2<true>(val.z, val.w);
-              *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + o) = pk;
+              __stcs(reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p.y) + o), pk);
             }
           } else {                                        // ragged N: element by element, rows < N
             const float vv[4] = {val.x, val.y, val.z, val.w};

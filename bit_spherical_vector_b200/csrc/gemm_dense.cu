@@ -181,8 +181,9 @@ gemm_dense_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_const
               part[(size_t)(c0 + i) * kRM + rt] = val;                  // [token][row] of the slot
             } else if (n < p.N) {
               const size_t o = (size_t)(m0 + i) * p.N + n;
-              if (p.y_f32) reinterpret_cast<float*>(p.y)[o] = val;
-              else reinterpret_cast<uint16_t*>(p.y)[o] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+              // streaming stores: y is not re-read here, the operand tiles are
+              if (p.y_f32) __stcs(reinterpret_cast<float*>(p.y) + o, val);
+              else __stcs(reinterpret_cast<unsigned short*>(p.y) + o, __bfloat16_as_ushort(__float2bfloat16_rn(val)));
             }
           }
         }
