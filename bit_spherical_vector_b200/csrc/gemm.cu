@@ -603,7 +603,9 @@ cudaError_t launch_typed(int BN, const CUtensorMap& tm, const CUtensorMap& tw, c
     case 16: return launch_bn<16, 6, BF16>(tm, tw, p, grid, pdl, st);
     case 32: return launch_bn<32, 6, BF16>(tm, tw, p, grid, pdl, st);
     case 64: return launch_bn<64, 5, BF16>(tm, tw, p, grid, pdl, st);
-    case 128: return launch_bn<128, 4, BF16>(tm, tw, p, grid, pdl, st);
+    case 128:
+      return p.dense ? launch_bn<128, 6, BF16, true>(tm, tw, p, grid, pdl, st)
+                     : launch_bn<128, 4, BF16>(tm, tw, p, grid, pdl, st);
     default:
       return p.dense ? launch_bn<256, 4, BF16, true>(tm, tw, p, grid, pdl, st)
                      : launch_bn<256, 3, BF16>(tm, tw, p, grid, pdl, st);
@@ -639,10 +641,12 @@ GemmPlan plan_gemm(int N, int K, int M, int num_sms) {
   GemmPlan g{};
   g.BN = M >= 256 ? 256 : (M > 64 ? 128 : (M > 32 ? 64 : (M > 16 ? 32 : 16)));
   g.m_tiles = (M + g.BN - 1) / g.BN;
-  // From two token tiles on, the matrix is decoded once into the workspace
-  // (N x K 16-bit values, the activations' type) and the kernel loads weight
-  // tiles by TMA instead of decoding every stage once per token tile; with one
-  // token tile the decode pass would only add its own cost.
+  // From two token tiles on (M > 128, except exactly 256: one tile of 256),
+  // the matrix is decoded once into the workspace (N x K 16-bit values, the
+  // activations' type) and the kernel loads weight tiles by TMA instead of
+  // decoding every stage once per token tile; with one token tile the decode
+  // pass would only add its own cost (at 256 tokens the decode pass of a
+  // 2560 x 9728 matrix costs more than the on-chip decode it replaces).
   g.dense = g.m_tiles >= 2 ? 1 : 0;
   // Pre-decoded tiles of 256 rows (1.5x fewer L2 bytes per output) once they
   // still fill every SM at least once; below that 128-row tiles keep more SMs busy.

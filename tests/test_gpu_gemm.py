@@ -123,19 +123,24 @@ def test_gemm_metamorphic_permutation():
 
 @pytest.mark.parametrize("x_dtype", ["bf16", "f16"])
 def test_gemm_pre_decoded_plan_matches_decoded_tiles(x_dtype):
-    """Two or more 256-token tiles switch the GEMM to weights decoded once into the workspace and
-    loaded by TMA; one tile decodes on chip.  Both place the same 16-bit weights in the MMA (the export
-    reading), so the first 256 tokens of a 1100-token call equal a 256-token call bit for bit (K = 512:
-    no K split in either plan), and every output is within the bound of the oracle.  N = 1028 ends in a
-    4-row tile (rows past N read as zeros by the TMA box)."""
+    """Two or more token tiles switch the GEMM to weights decoded once into the workspace and loaded
+    by TMA; one tile decodes on chip.  Both place the same 16-bit weights in the MMA (the export
+    reading), so the first 128 tokens of a 1100-token call (pre-decoded, 256-token tiles) and of a
+    200-token call (pre-decoded, 128-token tiles) equal a 128-token call (on-chip decode) bit for bit
+    (K = 512: no K split in any of them), and every output is within the bound of the oracle.
+    N = 1028 ends in a 4-row tile (rows past N read as zeros by the TMA box)."""
     need_gpu()
     N, K = 1028, 512
     m = synth.make_matrix(76, 1 if x_dtype == "f16" else 0, N, K, 7)
     x = synth.make_x(76, 2, 1100, K, dtype=x_dtype)
     W = svq.SvqWeight.from_synth(m)
     yb, _, _ = _gemm(W, x, kind=x_dtype)
-    y256, _, _ = _gemm(W, np.ascontiguousarray(x[:256]), kind=x_dtype)
-    assert torch.equal(yb[:256], y256)
+    y200, _, _ = _gemm(W, np.ascontiguousarray(x[:200]), kind=x_dtype)
+    y128, _, _ = _gemm(W, np.ascontiguousarray(x[:128]), kind=x_dtype)
+    assert torch.equal(yb[:128], y128)
+    assert torch.equal(y200[:128], y128)
+    y_ref200, den200 = oracle.linear(m, np.ascontiguousarray(x[:200]), x_dtype)
+    assert rel_err(y200.cpu().numpy(), y_ref200, den200) <= TOL
     y_ref, den = oracle.linear(m, x, x_dtype)
     assert rel_err(yb.cpu().numpy(), y_ref, den) <= TOL
 
