@@ -66,6 +66,7 @@ def lib():
         "svq_linear_gemv": ([MP, P, I, P, I, P, SZ, P], I),
         "svq_linear_gemv_batched_workspace_size": ([MP, I, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemv_batched": ([MP, I, ctypes.POINTER(P), I, ctypes.POINTER(P), I, P, SZ, P], I),
+        "svq_linear_gemv_batched_host": ([MP, I, P, P, I, P, P, I, P, SZ, P], I),
         "svq_linear_gemv_noalloc": ([MP, P, I, P, I, P], I),
         "svq_linear_gemm_workspace_size": ([MP, I, ctypes.POINTER(SZ)], I),
         "svq_linear_gemm": ([MP, P, I, I, P, I, P, SZ, P], I),
@@ -236,6 +237,23 @@ class GemvBatchCall:
 
     def __call__(self, stream=None):
         _check(self._fn(*self._args, _stream(stream)), "svq_linear_gemv_batched")
+
+
+class GemvBatchHostCall:
+    """svq_linear_gemv_batched_host with its arguments marshalled once: each call copies the step's
+    inputs x_host (pinned, the inputs back to back) into x_dev, runs the grouped launch and copies
+    y_dev (the outputs back to back) into y_host (pinned), all enqueued on the stream."""
+
+    def __init__(self, Ws, M, x_host, x_dev, y_host, y_dev, ws=None):
+        n = len(Ws)
+        self._keep = (list(Ws), x_host, x_dev, y_host, y_dev, ws)  # the buffers must outlive the calls
+        self._args = ((svq_matrix * n)(*[w.desc for w in Ws]), n, _ptr(x_host), _ptr(x_dev), M,
+                      _ptr(y_host), _ptr(y_dev), _dtype_code(y_dev.dtype), _ptr(ws),
+                      0 if ws is None else ws.numel() * ws.element_size())
+        self._fn = lib().svq_linear_gemv_batched_host
+
+    def __call__(self, stream=None):
+        _check(self._fn(*self._args, _stream(stream)), "svq_linear_gemv_batched_host")
 
 
 def svq_linear_gemv_noalloc(W: SvqWeight, x, y, stream=None):

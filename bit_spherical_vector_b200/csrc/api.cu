@@ -224,9 +224,10 @@ int svq_workspace_init(void* workspace, size_t bytes, svq_stream_t stream) {
   return cuda_status(cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream));
 }
 
-int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const uint16_t* const* x, int M,
-                            void* const* y, int y_dtype, void* workspace, size_t workspace_bytes,
-                            svq_stream_t stream) {
+// Checks and plans a grouped GEMV call (nothing is enqueued).
+static int prepare_batched(const svq_matrix* mats, int n_mats, const uint16_t* const* x, int M, void* const* y,
+                           int y_dtype, void* workspace, size_t workspace_bytes, svq::GemvPlan* plan,
+                           svq::GemvMatDesc* descs) {
   if (!x || !y) return SVQ_ERR_INVALID_ARG;
   if (y_dtype != SVQ_F16 && y_dtype != SVQ_F32) return SVQ_ERR_INVALID_ARG;
   if (n_mats < 1 || n_mats > svq::kGemvMaxMats) return SVQ_ERR_INVALID_ARG;
@@ -234,13 +235,51 @@ int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const uint16_t* 
     if (!x[i] || !y[i]) return SVQ_ERR_INVALID_ARG;
     if (!aligned(x[i], 2) || !aligned(y[i], y_dtype == SVQ_F32 ? 4 : 2)) return SVQ_ERR_INVALID_ARG;
   }
+  const int st = plan_group(mats, n_mats, M, plan, descs, x, y);
+  if (st != SVQ_OK) return st;
+  if (plan->ws_total > 0 && (!workspace || workspace_bytes < plan->ws_total || !aligned(workspace, 256)))
+    return SVQ_ERR_WORKSPACE;
+  return SVQ_OK;
+}
+
+int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const uint16_t* const* x, int M,
+                            void* const* y, int y_dtype, void* workspace, size_t workspace_bytes,
+                            svq_stream_t stream) {
   svq::GemvPlan plan;
   svq::GemvMatDesc descs[svq::kGemvMaxMats];
-  const int st = plan_group(mats, n_mats, M, &plan, descs, x, y);
+  const int st = prepare_batched(mats, n_mats, x, M, y, y_dtype, workspace, workspace_bytes, &plan, descs);
   if (st != SVQ_OK) return st;
-  if (plan.ws_total > 0 && (!workspace || workspace_bytes < plan.ws_total || !aligned(workspace, 256)))
-    return SVQ_ERR_WORKSPACE;
   return cuda_status(svq::launch_gemv(descs, plan, y_dtype == SVQ_F32, workspace, (cudaStream_t)stream));
+}
+
+int svq_linear_gemv_batched_host(const svq_matrix* mats, int n_mats, const uint16_t* x_host, uint16_t* x_dev,
+                                 int M, void* y_host, void* y_dev, int y_dtype, void* workspace,
+                                 size_t workspace_bytes, svq_stream_t stream) {
+  if (!mats || !x_host || !x_dev || !y_host || !y_dev) return SVQ_ERR_INVALID_ARG;
+  if (n_mats < 1 || n_mats > svq::kGemvMaxMats || M < 1) return SVQ_ERR_INVALID_ARG;
+  if (y_dtype != SVQ_F16 && y_dtype != SVQ_F32) return SVQ_ERR_INVALID_ARG;
+  const size_t ysz = y_dtype == SVQ_F32 ? 4 : 2;
+  const uint16_t* xs[svq::kGemvMaxMats];
+  void* ys[svq::kGemvMaxMats];
+  size_t xo = 0, yo = 0;                             // elements of x, bytes of y
+  for (int i = 0; i < n_mats; ++i) {
+    if (mats[i].N < 1 || mats[i].K < 1) return SVQ_ERR_INVALID_ARG;
+    xs[i] = x_dev + xo;
+    ys[i] = reinterpret_cast<char*>(y_dev) + yo;
+    xo += (size_t)M * mats[i].K;
+    yo += (size_t)M * mats[i].N * ysz;
+  }
+  svq::GemvPlan plan;
+  svq::GemvMatDesc descs[svq::kGemvMaxMats];
+  // every check passes before anything is enqueued
+  const int st = prepare_batched(mats, n_mats, xs, M, ys, y_dtype, workspace, workspace_bytes, &plan, descs);
+  if (st != SVQ_OK) return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xo * 2, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  e = svq::launch_gemv(descs, plan, y_dtype == SVQ_F32, workspace, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return cuda_status(cudaMemcpyAsync(y_host, y_dev, yo, cudaMemcpyDeviceToHost, s));
 }
 
 int svq_linear_gemv(const svq_matrix* W, const uint16_t* x, int M, void* y, int y_dtype, void* workspace,

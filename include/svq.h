@@ -185,6 +185,25 @@ SVQ_API int svq_linear_gemv_batched(const svq_matrix* mats, int n_mats, const ui
                             size_t workspace_bytes, svq_stream_t stream);
 
 /*
+ * svq_linear_gemv_batched_host -- svq_linear_gemv_batched for a decode step
+ * whose activations come from and whose results go to host memory: one call
+ * enqueues on `stream` the copy of x_host into x_dev, the grouped launch and
+ * the copy of y_dev into y_host (cudaMemcpyAsync each; nothing is allocated).
+ * x_host, x_dev: the n_mats inputs back to back, input i = M rows of
+ *   mats[i].K fp16 values (natural input order, as for svq_linear_gemv_batched).
+ * y_host, y_dev: the n_mats outputs back to back, output i = M rows of
+ *   mats[i].N values of y_dtype (SVQ_F16 or SVQ_F32).
+ * x_dev and y_dev are device buffers the caller owns; x_host and y_host should
+ * be page-locked, otherwise the copies are not asynchronous.  Every check of
+ * svq_linear_gemv_batched runs before anything is enqueued; the call returns
+ * once the three operations are enqueued, so y_host holds the results only
+ * after the stream has reached them (e.g. cudaStreamSynchronize).
+ */
+SVQ_API int svq_linear_gemv_batched_host(const svq_matrix* mats, int n_mats, const uint16_t* x_host,
+                                         uint16_t* x_dev, int M, void* y_host, void* y_dev, int y_dtype,
+                                         void* workspace, size_t workspace_bytes, svq_stream_t stream);
+
+/*
  * svq_linear_gemv_noalloc -- svq_linear_gemv for callers that cannot allocate
  * device memory.  The paper has no counterpart; this is a deployment aid.  Some
  * callers have no allocator to get a workspace from: a plugin that is handed

@@ -54,6 +54,17 @@ def test_validation_without_gpu():
     assert L.svq_dequantize(ctypes.byref(m), svq.SVQ_F32, dummy, nullp) == svq.SVQ_ERR_INVALID_ARG
     assert L.svq_linear_gemv(ctypes.byref(m), nullp, 1, dummy, svq.SVQ_F32, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
     assert L.svq_linear_gemv(ctypes.byref(m), dummy, 1, dummy, svq.SVQ_BF16, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    # host-buffer grouped call: every check runs before anything is enqueued
+    mats = (svq.svq_matrix * 1)(m)
+    hc = L.svq_linear_gemv_batched_host
+    assert hc(mats, 1, nullp, dummy, 1, dummy, dummy, svq.SVQ_F32, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert hc(mats, 0, dummy, dummy, 1, dummy, dummy, svq.SVQ_F32, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert hc(mats, 1, dummy, dummy, 0, dummy, dummy, svq.SVQ_F32, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert hc(mats, 1, dummy, dummy, 1, dummy, dummy, svq.SVQ_BF16, nullp, 0, nullp) == svq.SVQ_ERR_INVALID_ARG
+    assert hc(mats, 1, dummy, ctypes.c_void_p(0x1001), 1, dummy, dummy, svq.SVQ_F32, nullp, 0,
+              nullp) == svq.SVQ_ERR_INVALID_ARG
+    badm = (svq.svq_matrix * 1)(bad)
+    assert hc(badm, 1, dummy, dummy, 1, dummy, dummy, svq.SVQ_F32, nullp, 0, nullp) == svq.SVQ_ERR_UNSUPPORTED_SHAPE
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

@@ -219,3 +219,38 @@ def test_grouped_two_permuted_gate_shaped_matrices(N, M):
     for m, x, y in zip(mats, xs, ys):
         y_ref, den = oracle.linear(m, x)
         assert rel_err(y.cpu().numpy(), y_ref, den) <= TOL
+
+
+@pytest.mark.parametrize("M", [1, 3])
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.float16])
+def test_batched_host_call_matches_device_call(M, y_dtype):
+    """svq_linear_gemv_batched_host (pinned host x -> device copy, grouped launch, device -> pinned
+    host y copy in one call) on the seven decoder-layer linears: the host results equal the
+    device-buffer call bit for bit, and are within the bound of the oracle."""
+    need_gpu()
+    layer = synth.qwen3_4b_layer(0)
+    Ws = [svq.SvqWeight.from_synth(m) for m, _ in layer]
+    xs_np = [synth.make_x(90, i, M, m.K) for i, (m, _) in enumerate(layer)]
+    xs = [x_f16(x) for x in xs_np]
+    ys = [torch.empty((M, m.N), dtype=y_dtype, device="cuda") for m, _ in layer]
+    nb = svq.svq_linear_gemv_batched_workspace_size(Ws, M)
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device="cuda")
+    svq.svq_workspace_init(ws)
+    svq.svq_linear_gemv_batched(Ws, xs, ys, ws)
+    x_host = torch.cat([x.reshape(-1) for x in xs]).cpu().pin_memory()
+    x_dev = torch.empty_like(x_host, device="cuda")
+    n_out = sum(M * m.N for m, _ in layer)
+    y_host = torch.full((n_out,), float("nan"), dtype=y_dtype).pin_memory()
+    y_dev = torch.empty(n_out, dtype=y_dtype, device="cuda")
+    call = svq.GemvBatchHostCall(Ws, M, x_host, x_dev, y_host, y_dev, ws)
+    call()
+    call()                                        # twice: the workspace counters come back to zero
+    torch.cuda.synchronize()
+    assert torch.equal(y_host, torch.cat([y.reshape(-1) for y in ys]).cpu())
+    off = 0
+    for (m, _), x in zip(layer, xs_np):
+        y_ref, den = oracle.linear(m, x)
+        got = y_host[off:off + M * m.N].reshape(M, m.N).float().numpy()
+        tol = TOL + (2.0 ** -11 if y_dtype == torch.float16 else 0.0)
+        assert rel_err(got, y_ref, den) <= tol, m.name
+        off += M * m.N
