@@ -6,8 +6,8 @@
 // Once the weights need no on-chip decode the kernel is a plain tensor-core
 // GEMM whose speed is set by how many operand bytes each SM pulls from L2 per
 // MMA: a 128 x 256 tile takes 48 KB per 64-column k-block, a 256 x 256 tile
-// 64 KB for twice the outputs (1.5x fewer bytes per output), with no cluster
-// and no multicast.  Per CTA (persistent, one per SM, 18 warps):
+// 64 KB for twice the outputs (1.5x fewer bytes per output), with every CTA
+// loading its own tiles (no clusters).  Per CTA (persistent, one per SM, 18 warps):
 //   warp 0      TMA producer: per k-block one 256-row box of the decoded
 //               weights and one 256-token box of X_p (128-byte swizzle) into a
 //               three-stage ring, both completing on the stage's barrier
