@@ -487,7 +487,8 @@ def run_gpu(args, world, rank, local):
         del g_all, g_one
         line["secondary"] = {"sweep_8192": run_sweep(args, quiet=True), "prefill": run_prefill(args, quiet=True),
                              "moe": run_moe(args, quiet=True), "calibration": run_calib(args, quiet=True),
-                             "layer_radius_tables": run_lut_layer(args, quiet=True)}
+                             "layer_radius_tables": run_lut_layer(args, quiet=True),
+                             "shape_tails": run_tails(args, quiet=True)}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -683,6 +684,36 @@ def run_lut_layer(args, quiet=False):
     return [rec] if quiet else 0
 
 
+def run_tails(args, quiet=False):
+    """Shape tails: the batch-1 GEMV on a gate-shaped matrix whose N is not a multiple of 4 and whose K is
+    not a multiple of 128 (9726 x 2552, stored padded to 9728 x 2560 with zero codes), against the aligned
+    9728 x 2560; (8,2), 14 rotated copies each (larger than L2), one launch per copy."""
+    import torch
+    import bit_spherical_vector_b200 as svq
+    stream = torch.cuda.Stream()
+    recs = []
+    for N, K in ((9728, 2560), (9726, 2552)):
+        Ws, xs, ys = [], [], []
+        for L in range(N_LAYERS):
+            Ws.append(svq.SvqWeight.from_synth(synth.make_matrix(600 + L, 0, N, K, 8)))
+            xs.append(torch.from_numpy(synth.make_x(600 + L, 1, 1, K).view(np.int16)).cuda().view(torch.float16))
+            ys.append(torch.empty((1, N), dtype=torch.float32, device="cuda"))
+        ws = torch.zeros(max(svq.svq_linear_gemv_workspace_size(Ws[0], 1), 256), dtype=torch.uint8, device="cuda")
+        calls = [svq.GemvBatchCall([W], [x], [y], ws) for W, x, y in zip(Ws, xs, ys)]
+
+        def chain():
+            for c in calls:
+                c()
+        us = _time_graph(chain, 50, stream) / N_LAYERS
+        stored = svq.svq_packed_bytes(N, K)
+        recs.append({"workload": f"gemv {N}x{K} (8,2), batch 1", "us": round(us, 3),
+                     "packed_bytes_stored": stored, "packed_bytes_of_the_matrix": N * K * 9 // 32,
+                     "GBps_stored": round(stored / us / 1e3, 1)})
+        if not quiet:
+            print(json.dumps(recs[-1]), flush=True)
+    return recs if quiet else 0
+
+
 def run_calib(args, quiet=False):
     """Calibration side on one gate-projection-shaped matrix (9728 x 2560): ESG from 512 calibration rows,
     then for each candidate split b_d 6..9 the radius grid and the activation-weighted encode, then ABS.
@@ -827,12 +858,12 @@ def main():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the sweep / prefill / MoE / calibration measurements added to the headline line")
     ap.add_argument("--workload", default="layer",
-                    choices=["layer", "sweep", "prefill", "moe", "chain", "calib", "lut"],
+                    choices=["layer", "sweep", "prefill", "moe", "chain", "calib", "lut", "tails"],
                     help="layer = the headline line; the others print one JSON line per configuration")
     args = ap.parse_args()
     if args.workload != "layer":
         return {"sweep": run_sweep, "prefill": run_prefill, "moe": run_moe, "chain": run_chain,
-                "calib": run_calib, "lut": run_lut_layer}[args.workload](args)
+                "calib": run_calib, "lut": run_lut_layer, "tails": run_tails}[args.workload](args)
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_init() if args.impl == "svq" else (int(os.environ.get("WORLD_SIZE", "1")),
