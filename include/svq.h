@@ -244,8 +244,8 @@ SVQ_API int svq_linear_gemv_noalloc(const svq_matrix* W /* host */, const uint16
  * Tensor Memory Accelerator (TMA) reads it directly).  y: [M][N] of y_dtype SVQ_F32
  * or SVQ_BF16.
  * Workspace (svq_linear_gemm_workspace_size): the permuted activations
- * x[:, perm] (unused when perm is NULL); from 2 tiles of 256 tokens on
- * (M > 256) the matrix decoded once (N x K values of x_dtype, the weights
+ * x[:, perm] (unused when perm is NULL); from two token tiles on (M > 128,
+ * except M = 256, one tile) the matrix decoded once (N x K values of x_dtype, the weights
  * svq_dequantize exports), which the tensor cores then read in place of
  * decoding every weight tile once per token tile; and, when tiles are split
  * along K across CTAs (the tiles of a last, partial round over the SMs, or all
